@@ -1,0 +1,384 @@
+"""Benchmark of the FVAttn single-GPU hot path on B200.
+
+One step = one attention layer through the C ABI: reorder Q, K, V into
+spatio-temporal tiles -> route (block mean-pooling, block scores, Top-p with
+a Top-k floor) -> block-sparse attention -> inverse reorder.  Inputs are the
+seeded synthetic 720p-shaped layer (B=1, 40 heads, d=128, 21x45x80 latent,
+2x8x8 blocks, p=0.9, k=16) already resident in HBM.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl fvattn|reference]
+
+Prints one JSON line (rank 0).  With N > 1 (torchrun) every rank runs an
+independent replica layer with its own seed: there is no exchange step in
+this path, so scaling is weak and no collective touches the data.
+`--impl reference` times the CPU oracle instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "sparse-attn TFLOPS on executed blocks (% of bf16 peak) + end-to-end ms per layer"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+WORKLOAD = "720p"
+KERNELS_PER_STEP = 9   # reorder x3, pool, score/select, 2 work-list kernels, attention, inverse
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as fh:
+            d = json.load(fh)
+        return {k: float(d[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def workload_config(w, g):
+    return {
+        "workload": f"{w.name}-shaped layer: B={w.B}, H={w.H}, D={w.D}, latent {w.F}x{w.Hs}x{w.Ws} "
+                    f"= {w.N} tokens, {w.tf}x{w.th}x{w.tw} = {g.bs}-token blocks (nb={g.nb}), "
+                    f"p={w.p}, k={w.k}",
+        "global_batch": w.B, "seq_len": w.N, "heads": w.H, "head_dim": w.D,
+        "block": f"{w.tf}x{w.th}x{w.tw}", "nb": g.nb, "p": w.p, "k_floor": w.k,
+        "l2": "no flush: every input tensor (774 MB raster, 865 MB tiled) is larger than the 126 MB L2",
+        "parallelism": "replicas (independent layer per GPU)",
+    }
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples during the timed region."""
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- CPU oracle (baseline / reference arm)
+
+def oracle_sample_time(w, qt, kt, vt, q_raster, kv_idx_full, kv_cnt_full, heads=2, items_per_head=2):
+    """Time the oracle, as it stands, on a bounded sample of one layer and
+    extrapolate to the whole layer.
+
+    Sample: reorder of one raster tensor; routing (pool, scores, select) of
+    `heads` heads; masked attention on `items_per_head` query blocks of each
+    of those heads.  Extrapolation: reorder x4 (Q, K, V, inverse O), routing
+    x H/heads, attention x (executed block pairs of the layer / of the
+    sample).  Returns (seconds for the full layer, description, threads)."""
+    import numpy as np
+    from oracle import oracle as orc
+    from block_sparse_attention_aware_b200 import synth
+    orc.build_oracle()
+    threads = orc.num_threads()
+    t0 = time.perf_counter()
+    orc.reorder(synth.bf16_bits(q_raster), w)
+    t_reorder = time.perf_counter() - t0
+    sub = synth.custom_workload(**{**w.as_dict(), "H": heads, "name": "sample"})
+    hsel = list(range(heads))
+    qb = synth.bf16_bits(qt[:, hsel].contiguous())
+    kb = synth.bf16_bits(kt[:, hsel].contiguous())
+    vb = synth.bf16_bits(vt[:, hsel].contiguous())
+    t0 = time.perf_counter()
+    _, _, _, idx, cnt, _, _ = orc.route(qb, kb, sub, w.p, w.k, 1.0 / math.sqrt(w.D))
+    t_route = time.perf_counter() - t0
+    nb = idx.shape[-1]
+    items = []
+    for h in range(heads):
+        order = np.argsort(-cnt[0, h], kind="stable")
+        picks = [int(order[0]), int(order[len(order) // 2])][:items_per_head]
+        items += [h * nb + i for i in picks]
+    t0 = time.perf_counter()
+    orc.attention(qb, kb, vb, idx, cnt, items, sub, 1.0 / math.sqrt(w.D))
+    t_attn = time.perf_counter() - t0
+    sample_pairs = int(sum(cnt.reshape(-1)[i] for i in items))
+    layer_pairs = int(kv_cnt_full.sum())
+    full = 4 * t_reorder + t_route * (w.H * w.B / heads) + t_attn * layer_pairs / max(sample_pairs, 1)
+    desc = (f"oracle on {threads} host threads: reorder of 1 raster tensor (x4), routing of {heads} of "
+            f"{w.B * w.H} heads (x{w.B * w.H / heads:g}), masked attention on {len(items)} query blocks "
+            f"({sample_pairs} block pairs, scaled to the layer's {layer_pairs}); measured "
+            f"{t_reorder + t_route + t_attn:.1f} s, extrapolated to {full:.1f} s per layer")
+    return full, desc, threads, t_reorder + t_route + t_attn
+
+
+def run_reference(args):
+    """The oracle timed as the reference arm (rank 0; other ranks exit)."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import torch
+    from block_sparse_attention_aware_b200 import synth
+    w = synth.WORKLOADS[WORKLOAD]
+    q, k, v, _ = synth.make_qkv(w, device="cpu")
+    from oracle import oracle as orc
+    orc.build_oracle()
+    qt = torch.from_numpy(orc.reorder(synth.bf16_bits(q), w).view("int16")).view(torch.bfloat16)
+    kt = torch.from_numpy(orc.reorder(synth.bf16_bits(k), w).view("int16")).view(torch.bfloat16)
+    vt = torch.from_numpy(orc.reorder(synth.bf16_bits(v), w).view("int16")).view(torch.bfloat16)
+    # full-layer routing counts (needed for the executed-pair total)
+    _, _, _, _, cnt_full, _, _ = orc.route(synth.bf16_bits(qt), synth.bf16_bits(kt), w, w.p, w.k,
+                                           1.0 / math.sqrt(w.D))
+    geo = orc.geometry(w)
+    flops = 4.0 * geo["bs"] * geo["bs"] * w.D * float(cnt_full.sum())
+    times, descs = [], []
+    for i in range(args.warmup + args.steps):
+        full, desc, threads, _ = oracle_sample_time(w, qt, kt, vt, q, None, cnt_full)
+        if i >= args.warmup:
+            times.append(full)
+            descs.append(desc)
+    t = statistics.mean(times)
+    val = flops / t / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": val, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": t * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic (seeded, CPU generator)",
+        "config": {"workload": f"{w.name}-shaped layer", "global_batch": w.B, "seq_len": w.N},
+        "cpu_baseline": {"kind": "oracle", "value": val, "unit": "TFLOP/s", "cores": threads,
+                         "sample": descs[-1]},
+        "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- GPU arm
+
+def run_fvattn(args):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+    from block_sparse_attention_aware_b200 import fvattn, synth
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    fvattn.load()
+    w = synth.WORKLOADS[WORKLOAD]
+    g = fvattn.geom_of(w)
+    dev = torch.device("cuda", local)
+    # each rank: its own seeded replica layer
+    q, k, v, _ = synth.make_qkv(w, layer=rank, device=dev)
+    layer = fvattn.Layer(g, w.p, w.k, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    nsm = fvattn.num_sms()
+
+    def barrier():
+        if world > 1:
+            dist.barrier(device_ids=[local])
+
+    for _ in range(args.warmup):
+        layer(q, k, v, stats=True)
+    torch.cuda.synchronize()
+    assert fvattn.get_status() == 0, "device status after warm-up"
+
+    # timed region: K full steps, CUDA events per stage on the launching stream
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    start.record(stream)
+    for i in range(args.steps):
+        e = ev[i]
+        e[0].record(stream)
+        layer.reorder_qkv(q, k, v)
+        e[1].record(stream)
+        layer.route()
+        e[2].record(stream)
+        layer.attend(stats=True)
+        e[3].record(stream)
+        layer.restore()
+        e[4].record(stream)
+    end.record(stream)
+    torch.cuda.synchronize()
+    clock_info = clocks.stop()
+    barrier()
+    status = fvattn.get_status()
+    assert status == 0, f"device status {status}"
+    t_total = start.elapsed_time(end) / 1e3
+    t_max = torch.tensor([t_total], dtype=torch.float64, device=dev)
+    cnt = layer.routed.kv_cnt
+    pairs = int(cnt.sum())
+    flops = 4.0 * g.bs * g.bs * g.D * pairs
+    flops_t = torch.tensor([flops], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t_max, op=dist.ReduceOp.MAX)
+        dist.all_reduce(flops_t, op=dist.ReduceOp.SUM)
+    t_max = float(t_max.item())
+    flops_all = float(flops_t.item())
+
+    stage = {n: [] for n in ("reorder_qkv", "route", "attention", "inverse_reorder")}
+    for e in ev:
+        stage["reorder_qkv"].append(e[0].elapsed_time(e[1]))
+        stage["route"].append(e[1].elapsed_time(e[2]))
+        stage["attention"].append(e[2].elapsed_time(e[3]))
+        stage["inverse_reorder"].append(e[3].elapsed_time(e[4]))
+    ms = {kk: statistics.mean(vv) for kk, vv in stage.items()}
+    peaks, peak_src = load_peaks()
+    raster_bytes = g.B * g.N * g.H * g.D * 2
+    tiled_bytes = g.B * g.H * g.Npad * g.D * 2
+    attn_s = ms["attention"] / 1e3
+    attn_tflops = flops / attn_s / 1e12
+    route_bytes = 2 * tiled_bytes * (g.N / g.Npad) + 4 * pairs + 4 * cnt.numel()
+    route_gbs = route_bytes / (ms["route"] / 1e3) / 1e9
+    reorder_gbs = 3 * (raster_bytes + tiled_bytes) / (ms["reorder_qkv"] / 1e3) / 1e9
+    inverse_gbs = (raster_bytes + tiled_bytes) / (ms["inverse_reorder"] / 1e3) / 1e9
+    st = layer.sm_stats.cpu().numpy().astype(np.float64)
+    busy, blocks = st[:nsm], st[nsm:2 * nsm]
+    used = busy > 0
+    imb = float(busy[used].max() / busy[used].mean()) if used.any() else None
+    imb_pred = float(blocks[used].max() / blocks[used].mean()) if used.any() else None
+    per_head = cnt.view(g.B * g.H, g.nb).sum(dim=1).double().cpu().numpy()
+    sustained = peaks["bf16_tflops_sustained"]
+
+    line = {
+        "metric": METRIC,
+        "value": flops_all / (t_max / args.steps) / 1e12,
+        "unit": "TFLOP/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": t_max / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16",
+        "data": f"synthetic: seeded Gaussian Wan2.2 720p-shaped Q/K/V (seed {w.seed}+rank), "
+                "per-head log-uniform Q scales, shared rank-8 spatio-temporal component",
+        "config": workload_config(w, g),
+        "value_note": "executed-block attention FLOPs of all ranks / (max-over-ranks time of one whole "
+                      "layer step: reorder x3 + route + attention + inverse reorder)",
+        "attention": {
+            "tflops_executed_blocks": attn_tflops,
+            "pct_of_bf16_peak_burst": 100.0 * attn_tflops / peaks["bf16_tflops"],
+            "pct_of_bf16_peak_sustained": 100.0 * attn_tflops / sustained,
+            "ms": ms["attention"], "density": pairs / float(g.B * g.H * g.nb * g.nb),
+            "executed_block_pairs": pairs,
+            "sm_imbalance_max_over_mean": imb, "sm_imbalance_predicted_from_blocks": imb_pred,
+            "head_blocks_max_over_mean": float(per_head.max() / per_head.mean()),
+        },
+        "stages_ms": ms,
+        "stages_gbs": {"reorder_qkv": reorder_gbs, "route": route_gbs, "inverse_reorder": inverse_gbs,
+                       "route_pct_of_hbm": 100.0 * route_gbs / peaks["hbm_gbs"]},
+        "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": sustained, "unit": "TFLOP/s",
+                     "frac": attn_tflops / sustained, "traffic": None,
+                     "kernel": "sparse_attn_kernel<128>",
+                     "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside back-to-back steps)",
+                     "algorithmic_flops_per_launch": flops},
+        "gpu_launches": KERNELS_PER_STEP * args.steps,
+        "clocks": clock_info,
+    }
+
+    # end to end through the public API from pinned host buffers
+    if args.e2e_steps > 0:
+        qh = q.cpu().pin_memory()
+        kh = k.cpu().pin_memory()
+        vh = v.cpu().pin_memory()
+        oh = torch.empty_like(qh).pin_memory()
+        fvattn.attention_from_host(layer, qh, kh, vh, oh)
+        torch.cuda.synchronize()
+        barrier()
+        s0 = torch.cuda.Event(enable_timing=True)
+        s1 = torch.cuda.Event(enable_timing=True)
+        s0.record(stream)
+        for _ in range(args.e2e_steps):
+            fvattn.attention_from_host(layer, qh, kh, vh, oh)
+        s1.record(stream)
+        torch.cuda.synchronize()
+        te = torch.tensor([s0.elapsed_time(s1) / 1e3], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        te = float(te.item()) / args.e2e_steps
+        line["e2e"] = {"value": flops_all / te / 1e12, "unit": "TFLOP/s", "ms_per_step": te * 1e3,
+                       "h2d_bytes_per_step": 3 * raster_bytes, "d2h_bytes_per_step": raster_bytes,
+                       "steps": args.e2e_steps}
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        full, desc, threads, spent = oracle_sample_time(
+            w, layer.qt.cpu(), layer.kt.cpu(), layer.vt.cpu(), q.cpu(), None, cnt.cpu().numpy())
+        line["cpu_baseline"] = {"value": flops / full / 1e12, "unit": "TFLOP/s", "cores": threads,
+                                "kind": "oracle", "sample": desc, "sample_seconds": spent}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier(device_ids=[local])
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="fvattn", choices=["fvattn", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_fvattn(args)
+
+
+if __name__ == "__main__":
+    main()

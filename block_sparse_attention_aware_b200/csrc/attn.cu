@@ -1,0 +1,701 @@
+// Dynamic block-sparse attention on the materialised FVAttn mask
+// (paperlayer.ai summary, section 2 "Background and Related Work": dynamic
+// block-sparse attention; section 3 "FVAttn Design", item "Pipeline":
+// attention runs on the mask that routing materialised).
+//
+// Work list.  An item is (b, h, query block i) and costs kv_cnt[b,h,i] key
+// blocks.  Top-p makes costs uneven across heads (section 2, item on Top-p
+// producing heterogeneous workloads; section 3, "Runtime Load Balancing").
+// The pages balance that across GPUs by migrating heads; on one GPU the
+// analogue used here is a persistent kernel with one CTA per SM that takes
+// items from a shared counter in a fixed order: heads by total cost,
+// heaviest first, and inside a head query blocks longest first.  Taking
+// items dynamically in that order is a longest-processing-time greedy, and
+// keeping concurrent items inside one head keeps that head's K/V in L2.
+//
+// Kernel per CTA (192 threads, one CTA per SM):
+//   warp 0      producer: takes items, TMA-loads the Q tile and, per chunk of
+//               128 keys, the selected K and V blocks into a 2-stage ring,
+//               and writes the chunk's key-validity mask (padding tokens)
+//   warp 1      one lane issues tcgen05.mma: S = Q K^T into one of two TMEM
+//               S buffers, then O += P V into the TMEM O accumulator
+//   warps 2..5  softmax: one query row per thread (TMEM lane), online softmax
+//               in fp32 (exp2 on the MUFU), P rounded to bf16 into shared
+//               memory in the 128-byte-swizzled K-major layout, O rescaled
+//               in TMEM when the row maximum grows, and the epilogue
+//               (O / l -> bf16 -> global)
+// Every wait is bounded; a wait that runs out records FVATTN_ERR_TIMEOUT,
+// raises a CTA-wide abort flag and all roles leave their loops, so the CTA
+// always reaches the TMEM release.
+#include <cuda.h>
+
+#include "common.cuh"
+#include "ptx.cuh"
+
+namespace fv {
+
+constexpr int ATT_THREADS = 192;
+constexpr int STAGES = 2;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t O_COL = 256;          // S buffers at columns 0 and 128
+constexpr unsigned long long WAIT_LIMIT_NS = 4000000000ull;
+
+struct AttnArgs {
+    Geo g;
+    const int32_t* kv_idx;
+    const int32_t* kv_cnt;
+    const int32_t* head_order;   // [B*H] heads, heaviest first
+    const int32_t* item_order;   // [B*H][nb] query blocks of each head, longest first
+    int* counter;                // next item to hand out
+    __nv_bfloat16* o;            // [B, H, Npad, D]
+    unsigned long long* sm_stats;
+    float scale_log2;            // scale * log2(e)
+    int total_items;
+};
+
+struct __align__(8) Ctrl {
+    unsigned long long q_full, q_empty;
+    unsigned long long k_full[STAGES], v_full[STAGES], kv_empty[STAGES];
+    unsigned long long s_full[2], s_free[2];
+    unsigned long long p_full, pv_done, o_free;
+    unsigned long long item_full[2], item_empty[2];
+    int item[2][4];              // bh, qb, cnt, valid
+    uint32_t mask[STAGES][4];
+    uint32_t tmem_base;
+    int abort_flag;
+    unsigned long long blocks_done;
+};
+
+template <int D>
+struct Smem {
+    static constexpr uint32_t Q_BYTES = 128u * D * 2u;   // D/64 halves of 16 KB
+    static constexpr uint32_t KV_BYTES = 128u * D * 2u;
+    static constexpr uint32_t P_BYTES = 128u * 128u * 2u;
+    static constexpr uint32_t Q_OFF = 0;
+    static constexpr uint32_t K_OFF = Q_OFF + Q_BYTES;
+    static constexpr uint32_t V_OFF = K_OFF + STAGES * KV_BYTES;
+    static constexpr uint32_t P_OFF = V_OFF + STAGES * KV_BYTES;
+    static constexpr uint32_t CTRL_OFF = P_OFF + P_BYTES;
+    static constexpr uint32_t TOTAL = CTRL_OFF + static_cast<uint32_t>(sizeof(Ctrl));
+    // 1024 bytes of slack for the 1024-byte alignment; at least 120 KB so two
+    // CTAs never share an SM (each holds all 512 TMEM columns).
+    static constexpr uint32_t ALLOC = TOTAL + 1024 > 120u * 1024u ? TOTAL + 1024 : 120u * 1024u;
+};
+
+// Bounded mbarrier wait.  Returns false if the CTA aborted or the wait ran
+// past WAIT_LIMIT_NS (then it records the timeout and raises the abort flag).
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+    if (mbar_try_wait(bar, parity)) return true;
+    unsigned long long t0 = 0;
+    for (uint32_t it = 1;; ++it) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((it & 255u) == 0u) {
+            if (*abort_flag) return false;
+            unsigned long long now = global_timer_ns();
+            if (t0 == 0) {
+                t0 = now;
+            } else if (now - t0 > WAIT_LIMIT_NS) {
+                record_status(FVATTN_ERR_TIMEOUT);
+                *abort_flag = 1;
+                return false;
+            }
+        }
+    }
+}
+
+// Warp-uniform variant: every lane waits, and the warp leaves together if
+// any lane gave up (the .sync.aligned tcgen05 loads that follow need the
+// whole warp).
+__device__ __forceinline__ bool wait_warp(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+    const bool ok = wait_bar(bar, parity, abort_flag);
+    return __all_sync(0xffffffffu, ok);
+}
+
+__device__ __forceinline__ bool token_real(const Geo& g, int block, int off) {
+    int bx = block % g.nbx;
+    int rest = block / g.nbx;
+    int by = rest % g.nby;
+    int bf = rest / g.nby;
+    int ox = off % g.tw;
+    int r2 = off / g.tw;
+    int oy = r2 % g.th;
+    int of = r2 / g.th;
+    return bf * g.tf + of < g.F && by * g.th + oy < g.Hs && bx * g.tw + ox < g.Ws;
+}
+
+template <int D>
+__global__ void __launch_bounds__(ATT_THREADS, 1)
+    sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                       const __grid_constant__ CUtensorMap tmV, const AttnArgs a) {
+    using L = Smem<D>;
+    extern __shared__ unsigned char att_smem_raw[];
+    unsigned char* smem = reinterpret_cast<unsigned char*>(
+        (reinterpret_cast<uintptr_t>(att_smem_raw) + 1023u) & ~static_cast<uintptr_t>(1023u));
+    Ctrl& ctl = *reinterpret_cast<Ctrl*>(smem + L::CTRL_OFF);
+    const uint32_t sbase = smem_u32(smem);
+    const uint32_t sQ = sbase + L::Q_OFF;
+    const uint32_t sK = sbase + L::K_OFF;
+    const uint32_t sV = sbase + L::V_OFF;
+    const uint32_t sP = sbase + L::P_OFF;
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const Geo& g = a.g;
+    const int bs = g.bs;
+    const int bpc = 128 / bs;   // key blocks per 128-key chunk
+    volatile int* abort_flag = &ctl.abort_flag;
+    const unsigned long long t_start = global_timer_ns();
+
+    // ---- set-up: zero the operand tiles (stale rows must be finite), barriers, TMEM
+    {
+        uint4* z = reinterpret_cast<uint4*>(smem);
+        const uint32_t n16 = L::CTRL_OFF / 16u;
+        for (uint32_t i = threadIdx.x; i < n16; i += ATT_THREADS) z[i] = make_uint4(0, 0, 0, 0);
+        fence_proxy_async_smem();
+    }
+    if (threadIdx.x == 0) {
+        mbar_init(smem_u32(&ctl.q_full), 1);
+        mbar_init(smem_u32(&ctl.q_empty), 1);
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(smem_u32(&ctl.k_full[s]), 1);
+            mbar_init(smem_u32(&ctl.v_full[s]), 1);
+            mbar_init(smem_u32(&ctl.kv_empty[s]), 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(smem_u32(&ctl.s_full[b]), 1);
+            mbar_init(smem_u32(&ctl.s_free[b]), 4);
+            mbar_init(smem_u32(&ctl.item_full[b]), 1);
+            mbar_init(smem_u32(&ctl.item_empty[b]), 5);
+        }
+        mbar_init(smem_u32(&ctl.p_full), 4);
+        mbar_init(smem_u32(&ctl.pv_done), 1);
+        mbar_init(smem_u32(&ctl.o_free), 4);
+        ctl.abort_flag = 0;
+        ctl.blocks_done = 0ull;
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        prefetch_tmap(&tmQ);
+        prefetch_tmap(&tmK);
+        prefetch_tmap(&tmV);
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(&ctl.tmem_base), TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = ctl.tmem_base;
+
+    if (warp == 0) {
+        // =========================== producer
+        int item_seq = 0;
+        uint32_t c_seq = 0;
+        bool ok = true;
+        while (ok) {
+            const int slot = item_seq & 1;
+            if (!wait_warp(smem_u32(&ctl.item_empty[slot]), ((item_seq >> 1) & 1) ^ 1, abort_flag)) break;
+            int t = 0;
+            if (lane == 0) t = atomicAdd(a.counter, 1);
+            t = __shfl_sync(0xffffffffu, t, 0);
+            if (t >= a.total_items) {
+                if (lane == 0) {
+                    ctl.item[slot][3] = 0;
+                    mbar_arrive(smem_u32(&ctl.item_full[slot]));
+                }
+                break;
+            }
+            const int hs = t / g.nb;
+            const int r = t - hs * g.nb;
+            const int bh = __ldg(a.head_order + hs);
+            const int qb = __ldg(a.item_order + static_cast<long long>(bh) * g.nb + r);
+            int cnt = __ldg(a.kv_cnt + static_cast<long long>(bh) * g.nb + qb);
+            if (cnt < 1 || cnt > g.nb) {
+                if (lane == 0) record_status(FVATTN_ERR_BOUNDS);
+                cnt = cnt < 1 ? 1 : g.nb;
+            }
+            if (lane == 0) {
+                ctl.item[slot][0] = bh;
+                ctl.item[slot][1] = qb;
+                ctl.item[slot][2] = cnt;
+                ctl.item[slot][3] = 1;
+                mbar_arrive(smem_u32(&ctl.item_full[slot]));
+            }
+            // Q tile
+            if (!wait_warp(smem_u32(&ctl.q_empty), (item_seq & 1) ^ 1, abort_flag)) break;
+            const int row_base = bh * static_cast<int>(g.Npad);
+            if (lane == 0) {
+                mbar_arrive_expect_tx(smem_u32(&ctl.q_full), static_cast<uint32_t>(bs * D * 2));
+#pragma unroll
+                for (int h = 0; h < D / 64; ++h)
+                    tma_load_2d(sQ + h * 16384u, &tmQ, h * 64, row_base + qb * bs, smem_u32(&ctl.q_full));
+            }
+            const int32_t* list = a.kv_idx + (static_cast<long long>(bh) * g.nb + qb) * g.nb;
+            const int nc = (cnt + bpc - 1) / bpc;
+            for (int cl = 0; cl < nc; ++cl, ++c_seq) {
+                const int stage = c_seq % STAGES;
+                if (!wait_warp(smem_u32(&ctl.kv_empty[stage]), ((c_seq / STAGES) & 1) ^ 1, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                const int nblk = min(bpc, cnt - cl * bpc);
+                int j = 0;
+                if (lane < nblk) {
+                    j = __ldg(list + cl * bpc + lane);
+                    if (j < 0 || j >= g.nb) {
+                        record_status(FVATTN_ERR_BOUNDS);
+                        j = 0;
+                    }
+                }
+                uint32_t words[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int col = q * 32 + lane;
+                    const int s = col / bs;
+                    const int off = col - s * bs;
+                    const int jj = __shfl_sync(0xffffffffu, j, s < 8 ? s : 0);
+                    const bool valid = (s < nblk) && token_real(g, jj, off);
+                    words[q] = __ballot_sync(0xffffffffu, valid);
+                }
+                if (lane == 0) {
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) ctl.mask[stage][q] = words[q];
+                }
+                const uint32_t kb = sK + stage * L::KV_BYTES;
+                const uint32_t vb = sV + stage * L::KV_BYTES;
+                const uint32_t bytes = static_cast<uint32_t>(nblk * bs * D * 2);
+                // every lane < nblk holds one block id; lane 0 issues the copies
+                int jl[8];
+#pragma unroll
+                for (int s = 0; s < 8; ++s) jl[s] = __shfl_sync(0xffffffffu, j, s);
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(smem_u32(&ctl.k_full[stage]), bytes);
+                    for (int s = 0; s < nblk; ++s)
+#pragma unroll
+                        for (int h = 0; h < D / 64; ++h)
+                            tma_load_2d(kb + h * 16384u + s * bs * 128u, &tmK, h * 64, row_base + jl[s] * bs,
+                                        smem_u32(&ctl.k_full[stage]));
+                    mbar_arrive_expect_tx(smem_u32(&ctl.v_full[stage]), bytes);
+                    for (int s = 0; s < nblk; ++s)
+#pragma unroll
+                        for (int h = 0; h < D / 64; ++h)
+                            tma_load_2d(vb + h * 16384u + s * bs * 128u, &tmV, h * 64, row_base + jl[s] * bs,
+                                        smem_u32(&ctl.v_full[stage]));
+                }
+            }
+            ++item_seq;
+        }
+    } else if (warp == 1) {
+        // =========================== MMA issuer (one lane)
+        if (lane == 0) {
+            constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, 128, false);
+            constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, D, true);
+            int item_seq = 0;
+            uint32_t c_seq = 0;
+            unsigned long long blocks = 0;
+            bool ok = true;
+            // O += P V for global chunk c; `first` starts a new accumulation
+            auto issue_pv = [&](uint32_t c, bool first) -> bool {
+                const int stage = c % STAGES;
+                if (!wait_bar(smem_u32(&ctl.p_full), c & 1, abort_flag)) return false;
+                if (!wait_bar(smem_u32(&ctl.v_full[stage]), (c / STAGES) & 1, abort_flag)) return false;
+                if (first && !wait_bar(smem_u32(&ctl.o_free), (item_seq & 1) ^ 1, abort_flag)) return false;
+                tc_fence_after();
+                const uint32_t vb = sV + stage * L::KV_BYTES;
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint64_t ad = sw128_desc(sP + (kk >> 2) * 16384u + (kk & 3) * 32u, 16u, 1024u);
+                    const uint64_t bd = sw128_desc(vb + kk * 2048u, 16384u, 1024u);
+                    mma_bf16_ss(tmem + O_COL, ad, bd, IDESC_PV, (first && kk == 0) ? 0u : 1u);
+                }
+                mma_commit(smem_u32(&ctl.kv_empty[stage]));
+                mma_commit(smem_u32(&ctl.pv_done));
+                return true;
+            };
+            while (ok) {
+                const int slot = item_seq & 1;
+                if (!wait_bar(smem_u32(&ctl.item_full[slot]), (item_seq >> 1) & 1, abort_flag)) break;
+                const int valid = ctl.item[slot][3];
+                const int cnt = ctl.item[slot][2];
+                mbar_arrive(smem_u32(&ctl.item_empty[slot]));
+                if (!valid) break;
+                const int nc = (cnt + bpc - 1) / bpc;
+                blocks += static_cast<unsigned long long>(cnt);
+                if (!wait_bar(smem_u32(&ctl.q_full), item_seq & 1, abort_flag)) break;
+                tc_fence_after();
+                for (int cl = 0; cl < nc && ok; ++cl) {
+                    const uint32_t c = c_seq + cl;
+                    const int stage = c % STAGES;
+                    const int b = c & 1;
+                    if (!wait_bar(smem_u32(&ctl.k_full[stage]), (c / STAGES) & 1, abort_flag) ||
+                        !wait_bar(smem_u32(&ctl.s_free[b]), ((c >> 1) & 1) ^ 1, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t kb = sK + stage * L::KV_BYTES;
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint32_t off = (kk >> 2) * 16384u + (kk & 3) * 32u;
+                        const uint64_t ad = sw128_desc(sQ + off, 16u, 1024u);
+                        const uint64_t bd = sw128_desc(kb + off, 16u, 1024u);
+                        mma_bf16_ss(tmem + b * 128u, ad, bd, IDESC_QK, kk > 0 ? 1u : 0u);
+                    }
+                    mma_commit(smem_u32(&ctl.s_full[b]));
+                    if (cl == nc - 1) mma_commit(smem_u32(&ctl.q_empty));
+                    if (cl > 0 && !issue_pv(c - 1, cl == 1)) ok = false;
+                }
+                if (!ok) break;
+                if (!issue_pv(c_seq + nc - 1, nc == 1)) break;
+                c_seq += nc;
+                ++item_seq;
+            }
+            ctl.blocks_done = blocks;
+        }
+        __syncwarp();
+    } else {
+        // =========================== softmax / correction / epilogue
+        const int quad = warp & 3;                 // TMEM lanes 32*quad ..
+        const int row = quad * 32 + lane;          // query row in the 128-row tile
+        const uint32_t trow = tmem + (static_cast<uint32_t>(quad * 32) << 16);
+        const float sl2 = a.scale_log2;
+        int item_seq = 0;
+        uint32_t c_seq = 0;
+        bool ok = true;
+        while (ok) {
+            const int slot = item_seq & 1;
+            if (!wait_warp(smem_u32(&ctl.item_full[slot]), (item_seq >> 1) & 1, abort_flag)) break;
+            const int bh = ctl.item[slot][0];
+            const int qb = ctl.item[slot][1];
+            const int cnt = ctl.item[slot][2];
+            const int valid = ctl.item[slot][3];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&ctl.item_empty[slot]));
+            if (!valid) break;
+            const int nc = (cnt + bpc - 1) / bpc;
+            float m = -INFINITY, l = 0.f;
+            for (int cl = 0; cl < nc; ++cl) {
+                const uint32_t c = c_seq + cl;
+                const int stage = c % STAGES;
+                const int b = c & 1;
+                if (!wait_warp(smem_u32(&ctl.k_full[stage]), (c / STAGES) & 1, abort_flag) ||
+                    !wait_warp(smem_u32(&ctl.s_full[b]), (c >> 1) & 1, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                uint32_t mw[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) mw[q] = ctl.mask[stage][q];
+                tc_fence_after();
+                uint32_t sr[4][32];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) tmem_ld32(trow + b * 128u + q * 32u, sr[q]);
+                tmem_wait_ld();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(&ctl.s_free[b]));
+                // scale into log2 units, mask padding keys, row max
+                float mx = -INFINITY;
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        float v = __uint_as_float(sr[q][i]) * sl2;
+                        v = ((mw[q] >> i) & 1u) ? v : -INFINITY;
+                        sr[q][i] = __float_as_uint(v);
+                        mx = fmaxf(mx, v);
+                    }
+                const float m_new = fmaxf(m, mx);
+                const float alpha = ex2_approx(m - m_new);
+                float sum = 0.f;
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        float pv = ex2_approx(__uint_as_float(sr[q][i]) - m_new);
+                        sr[q][i] = __float_as_uint(pv);
+                        sum += pv;
+                    }
+                l = l * alpha + sum;
+                m = m_new;
+                if (cl > 0) {
+                    // O and the P buffer are free once the previous PV finished
+                    if (!wait_warp(smem_u32(&ctl.pv_done), (c - 1) & 1, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    if (__any_sync(0xffffffffu, alpha != 1.0f)) {
+#pragma unroll
+                        for (int q = 0; q < D / 32; ++q) {
+                            uint32_t o[32];
+                            tmem_ld32(trow + O_COL + q * 32u, o);
+                            tmem_wait_ld();
+#pragma unroll
+                            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+                            tmem_st32(trow + O_COL + q * 32u, o);
+                        }
+                        tmem_wait_st();
+                    }
+                }
+                // P row -> shared memory, bf16, 128-byte swizzle (K-major operand)
+                const uint32_t prow = sP + static_cast<uint32_t>(row) * 128u;
+#pragma unroll
+                for (int kc = 0; kc < 16; ++kc) {
+                    const int q = kc >> 2;
+                    const int i0 = (kc & 3) * 8;
+                    uint32_t w0 = pack_bf16x2(__uint_as_float(sr[q][i0 + 0]), __uint_as_float(sr[q][i0 + 1]));
+                    uint32_t w1 = pack_bf16x2(__uint_as_float(sr[q][i0 + 2]), __uint_as_float(sr[q][i0 + 3]));
+                    uint32_t w2 = pack_bf16x2(__uint_as_float(sr[q][i0 + 4]), __uint_as_float(sr[q][i0 + 5]));
+                    uint32_t w3 = pack_bf16x2(__uint_as_float(sr[q][i0 + 6]), __uint_as_float(sr[q][i0 + 7]));
+                    const int half = kc >> 3;
+                    const int chunk = (kc & 7) ^ (row & 7);
+                    const uint32_t addr = prow + half * 16384u + chunk * 16u;
+                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(w0), "r"(w1),
+                                 "r"(w2), "r"(w3)
+                                 : "memory");
+                }
+                fence_proxy_async_smem();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(&ctl.p_full));
+            }
+            if (!ok) break;
+            // epilogue: wait for the last PV, normalise, store bf16
+            const uint32_t c_last = c_seq + nc - 1;
+            if (!wait_warp(smem_u32(&ctl.pv_done), c_last & 1, abort_flag)) break;
+            tc_fence_after();
+            const float inv_l = 1.0f / l;
+            __nv_bfloat16* orow = a.o + ((static_cast<long long>(bh) * g.Npad) + static_cast<long long>(qb) * bs + row) * D;
+            const bool store = row < bs;
+#pragma unroll
+            for (int q = 0; q < D / 32; ++q) {
+                uint32_t o[32];
+                tmem_ld32(trow + O_COL + q * 32u, o);
+                tmem_wait_ld();
+                if (store) {
+#pragma unroll
+                    for (int v = 0; v < 4; ++v) {
+                        uint4 w;
+                        w.x = pack_bf16x2(__uint_as_float(o[v * 8 + 0]) * inv_l, __uint_as_float(o[v * 8 + 1]) * inv_l);
+                        w.y = pack_bf16x2(__uint_as_float(o[v * 8 + 2]) * inv_l, __uint_as_float(o[v * 8 + 3]) * inv_l);
+                        w.z = pack_bf16x2(__uint_as_float(o[v * 8 + 4]) * inv_l, __uint_as_float(o[v * 8 + 5]) * inv_l);
+                        w.w = pack_bf16x2(__uint_as_float(o[v * 8 + 6]) * inv_l, __uint_as_float(o[v * 8 + 7]) * inv_l);
+                        *reinterpret_cast<uint4*>(orow + q * 32 + v * 8) = w;
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&ctl.o_free));
+            c_seq += nc;
+            ++item_seq;
+        }
+    }
+
+    // ---- teardown
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem, TMEM_COLS);
+    if (threadIdx.x == 0 && a.sm_stats) {
+        const unsigned long long t_end = global_timer_ns();
+        a.sm_stats[blockIdx.x] = t_end - t_start;
+        a.sm_stats[gridDim.x + blockIdx.x] = ctl.blocks_done;
+    }
+}
+
+// ------------------------------------------------------------------ work list
+
+// One CTA per (b, h): order the head's query blocks by kv_cnt, longest first
+// (ties by lower block index), and record the head's total cost.
+__global__ void __launch_bounds__(256) worklist_head_kernel(Geo g, const int32_t* __restrict__ kv_cnt,
+                                                            int32_t* __restrict__ item_order,
+                                                            long long* __restrict__ head_cost) {
+    extern __shared__ int wl_hist[];   // [nb + 2]
+    const int nb = g.nb;
+    const long long bh = blockIdx.x;
+    const int32_t* cnt = kv_cnt + bh * nb;
+    for (int i = threadIdx.x; i < nb + 2; i += blockDim.x) wl_hist[i] = 0;
+    __syncthreads();
+    long long part = 0;
+    for (int i = threadIdx.x; i < nb; i += blockDim.x) {
+        int c = cnt[i];
+        c = c < 1 ? 1 : (c > nb ? nb : c);
+        atomicAdd(&wl_hist[c], 1);
+        part += c;
+    }
+    // block reduction of the cost
+    __shared__ long long red[8];
+    for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = part;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        long long tot = 0;
+        for (int w = 0; w < (int)(blockDim.x >> 5); ++w) tot += red[w];
+        head_cost[bh] = tot;
+        // descending exclusive scan: start[c] = #items with a larger count
+        int run = 0;
+        for (int c = nb; c >= 1; --c) {
+            int h = wl_hist[c];
+            wl_hist[c] = run;
+            run += h;
+        }
+        // stable placement in ascending block order
+        for (int i = 0; i < nb; ++i) {
+            int c = cnt[i];
+            c = c < 1 ? 1 : (c > nb ? nb : c);
+            item_order[bh * nb + wl_hist[c]++] = i;
+        }
+    }
+}
+
+// Single CTA: heads by total cost, heaviest first (ties by lower index);
+// resets the item counter.
+__global__ void __launch_bounds__(256) worklist_heads_kernel(int BH, const long long* __restrict__ head_cost,
+                                                             int32_t* __restrict__ head_order, int* counter) {
+    for (int h = threadIdx.x; h < BH; h += blockDim.x) {
+        const long long ch = head_cost[h];
+        int rank = 0;
+        for (int o = 0; o < BH; ++o) {
+            const long long co = head_cost[o];
+            rank += (co > ch) || (co == ch && o < h);
+        }
+        head_order[rank] = h;
+    }
+    if (threadIdx.x == 0) *counter = 0;
+}
+
+// ------------------------------------------------------------------ host side
+
+typedef CUresult (*PFN_encodeTiled)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                    const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                    CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static PFN_encodeTiled get_encode() {
+    static PFN_encodeTiled fn = nullptr;
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return nullptr;
+        fn = reinterpret_cast<PFN_encodeTiled>(p);
+    }
+    return fn;
+}
+
+// 2-D view [rows, D] of a tiled tensor, boxes of bs rows x 64 columns,
+// 128-byte swizzle (the tcgen05 K-major / MN-major SW128 operand layout).
+static bool make_tmap(CUtensorMap* m, const void* base, long long rows, int D, int bs) {
+    PFN_encodeTiled enc = get_encode();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(D) * 2u};
+    cuuint32_t box[2] = {64u, static_cast<cuuint32_t>(bs)};
+    cuuint32_t estr[2] = {1u, 1u};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+struct WsLayout {
+    size_t item_order, head_cost, head_order, counter, total;
+};
+
+static size_t al256(size_t x) { return (x + 255) / 256 * 256; }
+
+static WsLayout ws_layout(const fvattn_geom& g) {
+    WsLayout w;
+    size_t BH = static_cast<size_t>(g.B) * g.H;
+    w.item_order = 0;
+    w.head_cost = al256(sizeof(int32_t) * BH * g.nb);
+    w.head_order = w.head_cost + al256(sizeof(long long) * BH);
+    w.counter = w.head_order + al256(sizeof(int32_t) * BH);
+    w.total = w.counter + 256;
+    return w;
+}
+
+static int cached_num_sms() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    return n;
+}
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+template <int D>
+static int launch_attn(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const AttnArgs& args,
+                       int grid, cudaStream_t s) {
+    using L = Smem<D>;
+    if (cudaFuncSetAttribute(sparse_attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(L::ALLOC)) != cudaSuccess)
+        return FVATTN_ERR_CUDA;
+    sparse_attn_kernel<D><<<grid, ATT_THREADS, L::ALLOC, s>>>(tq, tk, tv, args);
+    FV_CHECK_LAUNCH();
+    return FVATTN_OK;
+}
+
+}  // namespace fv
+
+using namespace fv;
+
+extern "C" size_t fvattn_attn_workspace_size(const fvattn_geom* gp) {
+    if (!gp) return 0;
+    return ws_layout(*gp).total;
+}
+
+extern "C" int fvattn_num_sms(void) { return cached_num_sms(); }
+
+extern "C" int fvattn_sparse_attn(const fvattn_geom* gp, const void* q_t, const void* k_t, const void* v_t,
+                                  const int32_t* kv_idx, const int32_t* kv_cnt, float scale, void* o_t,
+                                  unsigned long long* sm_stats, void* workspace, size_t ws_bytes,
+                                  fvattn_stream_t stream) {
+    if (!gp || !q_t || !k_t || !v_t || !kv_idx || !kv_cnt || !o_t || !workspace) return FVATTN_ERR_INVALID;
+    if (!aligned16(q_t) || !aligned16(k_t) || !aligned16(v_t) || !aligned16(o_t) || !aligned16(kv_idx) ||
+        !aligned16(kv_cnt) || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+        return FVATTN_ERR_INVALID;
+    if (!isfinite(scale)) return FVATTN_ERR_INVALID;
+    if (gp->D != 64 && gp->D != 128) return FVATTN_ERR_UNSUPPORTED;
+    if (gp->bs != 16 && gp->bs != 32 && gp->bs != 64 && gp->bs != 128) return FVATTN_ERR_UNSUPPORTED;
+    if (gp->nb <= 0 || gp->nb > 2560) return FVATTN_ERR_UNSUPPORTED;
+    const WsLayout wl = ws_layout(*gp);
+    if (ws_bytes < wl.total) return FVATTN_ERR_INVALID;
+    const long long rows = static_cast<long long>(gp->B) * gp->H * gp->Npad;
+    if (rows >= (1ll << 31)) return FVATTN_ERR_UNSUPPORTED;
+    Geo g = to_geo(*gp);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    char* ws = static_cast<char*>(workspace);
+    int32_t* item_order = reinterpret_cast<int32_t*>(ws + wl.item_order);
+    long long* head_cost = reinterpret_cast<long long*>(ws + wl.head_cost);
+    int32_t* head_order = reinterpret_cast<int32_t*>(ws + wl.head_order);
+    int* counter = reinterpret_cast<int*>(ws + wl.counter);
+    const int BH = g.B * g.H;
+
+    worklist_head_kernel<<<BH, 256, sizeof(int) * (g.nb + 2), s>>>(g, kv_cnt, item_order, head_cost);
+    FV_CHECK_LAUNCH();
+    worklist_heads_kernel<<<1, 256, 0, s>>>(BH, head_cost, head_order, counter);
+    FV_CHECK_LAUNCH();
+
+    CUtensorMap tq, tk, tv;
+    if (!make_tmap(&tq, q_t, rows, g.D, g.bs) || !make_tmap(&tk, k_t, rows, g.D, g.bs) ||
+        !make_tmap(&tv, v_t, rows, g.D, g.bs))
+        return FVATTN_ERR_CUDA;
+    AttnArgs args;
+    args.g = g;
+    args.kv_idx = kv_idx;
+    args.kv_cnt = kv_cnt;
+    args.head_order = head_order;
+    args.item_order = item_order;
+    args.counter = counter;
+    args.o = static_cast<__nv_bfloat16*>(o_t);
+    args.sm_stats = sm_stats;
+    args.scale_log2 = scale * 1.4426950408889634f;
+    args.total_items = BH * g.nb;
+    int nsm = cached_num_sms();
+    if (nsm <= 0) return FVATTN_ERR_CUDA;
+    const int grid = nsm;
+    return g.D == 128 ? launch_attn<128>(tq, tk, tv, args, grid, s) : launch_attn<64>(tq, tk, tv, args, grid, s);
+}

@@ -1,0 +1,72 @@
+// Shared definitions of the CUDA path: geometry passed to kernels, the
+// device status word, and the tile <-> raster index maps.
+#pragma once
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <cstdint>
+
+#include "fvattn.h"
+
+namespace fv {
+
+// Kernel-side copy of the geometry (plain ints, passed by value).
+struct Geo {
+    int B, H, D, F, Hs, Ws, tf, th, tw;
+    int nbf, nby, nbx, bs, nb;
+    long long N, Npad;
+};
+
+inline Geo to_geo(const fvattn_geom& g) {
+    Geo k;
+    k.B = g.B; k.H = g.H; k.D = g.D; k.F = g.F; k.Hs = g.Hs; k.Ws = g.Ws;
+    k.tf = g.tf; k.th = g.th; k.tw = g.tw;
+    k.nbf = g.nbf; k.nby = g.nby; k.nbx = g.nbx; k.bs = g.bs; k.nb = g.nb;
+    k.N = g.N; k.Npad = g.Npad;
+    return k;
+}
+
+// Device status word (FVATTN_OK or the first error a kernel recorded).
+extern __device__ int g_fvattn_status;
+
+__device__ __forceinline__ void record_status(int code) {
+    atomicCAS(&g_fvattn_status, 0, code);
+}
+
+// Raster token (f, y, x) of tile-layout position `pos` of a head, and
+// whether it is a real token.
+__device__ __forceinline__ bool token_of_pos(const Geo& g, long long pos, int& f, int& y, int& x) {
+    int block = static_cast<int>(pos / g.bs);
+    int off = static_cast<int>(pos - static_cast<long long>(block) * g.bs);
+    int bx = block % g.nbx;
+    int rest = block / g.nbx;
+    int by = rest % g.nby;
+    int bf = rest / g.nby;
+    int ox = off % g.tw;
+    int r2 = off / g.tw;
+    int oy = r2 % g.th;
+    int of = r2 / g.th;
+    f = bf * g.tf + of;
+    y = by * g.th + oy;
+    x = bx * g.tw + ox;
+    return f < g.F && y < g.Hs && x < g.Ws;
+}
+
+// Number of real tokens in block `block`.
+__device__ __forceinline__ int block_real_tokens(const Geo& g, int block) {
+    int bx = block % g.nbx;
+    int rest = block / g.nbx;
+    int by = rest % g.nby;
+    int bf = rest / g.nby;
+    int nf = min(g.tf, g.F - bf * g.tf);
+    int ny = min(g.th, g.Hs - by * g.th);
+    int nx = min(g.tw, g.Ws - bx * g.tw);
+    return nf * ny * nx;
+}
+
+}  // namespace fv
+
+#define FV_CHECK_LAUNCH()                                      \
+    do {                                                       \
+        cudaError_t e_ = cudaGetLastError();                   \
+        if (e_ != cudaSuccess) return FVATTN_ERR_CUDA;         \
+    } while (0)

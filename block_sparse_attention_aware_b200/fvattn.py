@@ -1,0 +1,269 @@
+"""ctypes binding of libfvattn.so (the C ABI in include/fvattn.h).
+
+Argument marshalling only: every step of the path runs in the library's
+CUDA kernels.  torch provides device memory and the current CUDA stream.
+There is no CPU fallback: if the library is missing or no CUDA device is
+present, the calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from dataclasses import dataclass
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libfvattn.so")
+_lib = None
+
+OK, ERR_INVALID, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_BOUNDS = range(6)
+EXPORTED = ("fvattn_geom_init", "fvattn_reorder", "fvattn_inverse_reorder",
+            "fvattn_route_workspace_size", "fvattn_route", "fvattn_attn_workspace_size",
+            "fvattn_num_sms", "fvattn_sparse_attn", "fvattn_get_status", "fvattn_status_string")
+
+
+class FVAttnError(RuntimeError):
+    def __init__(self, what: str, code: int):
+        super().__init__(f"{what}: {status_string(code)} (code {code})")
+        self.code = code
+
+
+class Geom(ctypes.Structure):
+    """Mirror of fvattn_geom."""
+    _fields_ = [(n, ctypes.c_int) for n in
+                ("B", "H", "D", "F", "Hs", "Ws", "tf", "th", "tw",
+                 "Fp", "Hp", "Wp", "nbf", "nby", "nbx", "bs", "nb")] + \
+               [("N", ctypes.c_longlong), ("Npad", ctypes.c_longlong)]
+
+
+def load(path: str = LIB_PATH):
+    """Load libfvattn.so and declare its signatures (raises if missing)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"libfvattn.so not built at {path}; run "
+                           "`python -m block_sparse_attention_aware_b200.build`")
+    L = ctypes.CDLL(path)
+    P, I, S = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    G = ctypes.POINTER(Geom)
+    L.fvattn_geom_init.argtypes = [G]
+    L.fvattn_geom_init.restype = I
+    L.fvattn_reorder.argtypes = [G, P, P, P]
+    L.fvattn_reorder.restype = I
+    L.fvattn_inverse_reorder.argtypes = [G, P, P, P]
+    L.fvattn_inverse_reorder.restype = I
+    L.fvattn_route_workspace_size.argtypes = [G]
+    L.fvattn_route_workspace_size.restype = S
+    L.fvattn_route.argtypes = [G, P, P, ctypes.c_double, I, ctypes.c_float, P, P, P, P, P, P, S, P]
+    L.fvattn_route.restype = I
+    L.fvattn_attn_workspace_size.argtypes = [G]
+    L.fvattn_attn_workspace_size.restype = S
+    L.fvattn_num_sms.argtypes = []
+    L.fvattn_num_sms.restype = I
+    L.fvattn_sparse_attn.argtypes = [G, P, P, P, P, P, ctypes.c_float, P, P, P, S, P]
+    L.fvattn_sparse_attn.restype = I
+    L.fvattn_get_status.argtypes = [P]
+    L.fvattn_get_status.restype = I
+    L.fvattn_status_string.argtypes = [I]
+    L.fvattn_status_string.restype = ctypes.c_char_p
+    _lib = L
+    return L
+
+
+def status_string(code: int) -> str:
+    return load().fvattn_status_string(int(code)).decode()
+
+
+def _check(what: str, rc: int):
+    if rc != OK:
+        raise FVAttnError(what, rc)
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return ctypes.c_void_p(0 if t is None else t.data_ptr())
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None and (not t.is_cuda or not t.is_contiguous()):
+            raise ValueError("tensors must be contiguous CUDA tensors")
+
+
+def geom(B, H, D, F, Hs, Ws, tf, th, tw) -> Geom:
+    g = Geom(B=B, H=H, D=D, F=F, Hs=Hs, Ws=Ws, tf=tf, th=th, tw=tw)
+    _check("fvattn_geom_init", load().fvattn_geom_init(ctypes.byref(g)))
+    return g
+
+
+def geom_of(w) -> Geom:
+    """Geometry of a synth.Workload."""
+    return geom(w.B, w.H, w.D, w.F, w.Hs, w.Ws, w.tf, w.th, w.tw)
+
+
+def num_sms() -> int:
+    return load().fvattn_num_sms()
+
+
+def tiled_empty(g: Geom, device="cuda") -> torch.Tensor:
+    return torch.empty((g.B, g.H, g.Npad, g.D), dtype=torch.bfloat16, device=device)
+
+
+def reorder(g: Geom, x: torch.Tensor, out: Optional[torch.Tensor] = None, stream=None):
+    """fvattn_reorder: raster [B, N, H, D] bf16 -> tiled [B, H, Npad, D]."""
+    _need_cuda(x, out)
+    assert x.dtype == torch.bfloat16 and tuple(x.shape) == (g.B, g.N, g.H, g.D)
+    if out is None:
+        out = tiled_empty(g, x.device)
+    _check("fvattn_reorder", load().fvattn_reorder(ctypes.byref(g), _ptr(x), _ptr(out), _stream(stream)))
+    return out
+
+
+def inverse_reorder(g: Geom, ot: torch.Tensor, out: Optional[torch.Tensor] = None, stream=None):
+    """fvattn_inverse_reorder: tiled [B, H, Npad, D] -> raster [B, N, H, D]."""
+    _need_cuda(ot, out)
+    assert ot.dtype == torch.bfloat16 and tuple(ot.shape) == (g.B, g.H, g.Npad, g.D)
+    if out is None:
+        out = torch.empty((g.B, g.N, g.H, g.D), dtype=torch.bfloat16, device=ot.device)
+    _check("fvattn_inverse_reorder",
+           load().fvattn_inverse_reorder(ctypes.byref(g), _ptr(ot), _ptr(out), _stream(stream)))
+    return out
+
+
+@dataclass
+class RouteOut:
+    kv_idx: torch.Tensor
+    kv_cnt: torch.Tensor
+    q_pool: Optional[torch.Tensor] = None
+    k_pool: Optional[torch.Tensor] = None
+    logits: Optional[torch.Tensor] = None
+
+
+def route_workspace(g: Geom, device="cuda") -> torch.Tensor:
+    n = load().fvattn_route_workspace_size(ctypes.byref(g))
+    return torch.empty(max(n, 256), dtype=torch.uint8, device=device)
+
+
+def attn_workspace(g: Geom, device="cuda") -> torch.Tensor:
+    n = load().fvattn_attn_workspace_size(ctypes.byref(g))
+    return torch.empty(max(n, 256), dtype=torch.uint8, device=device)
+
+
+def route(g: Geom, qt: torch.Tensor, kt: torch.Tensor, p: float, k: int,
+          scale: Optional[float] = None, debug: bool = False, out: Optional[RouteOut] = None,
+          workspace: Optional[torch.Tensor] = None, stream=None) -> RouteOut:
+    """fvattn_route: pooled block scores -> Top-p (+ Top-k floor) kv lists."""
+    _need_cuda(qt, kt)
+    dev = qt.device
+    if scale is None:
+        scale = 1.0 / math.sqrt(g.D)
+    if out is None:
+        out = RouteOut(kv_idx=torch.empty((g.B, g.H, g.nb, g.nb), dtype=torch.int32, device=dev),
+                       kv_cnt=torch.empty((g.B, g.H, g.nb), dtype=torch.int32, device=dev))
+        if debug:
+            out.q_pool = torch.empty((g.B, g.H, g.nb, g.D), dtype=torch.float32, device=dev)
+            out.k_pool = torch.empty_like(out.q_pool)
+            out.logits = torch.empty((g.B, g.H, g.nb, g.nb), dtype=torch.float32, device=dev)
+    if workspace is None and (out.q_pool is None or out.k_pool is None):
+        workspace = route_workspace(g, dev)
+    rc = load().fvattn_route(ctypes.byref(g), _ptr(qt), _ptr(kt), float(p), int(k), float(scale),
+                             _ptr(out.kv_idx), _ptr(out.kv_cnt), _ptr(out.q_pool), _ptr(out.k_pool),
+                             _ptr(out.logits), _ptr(workspace),
+                             0 if workspace is None else workspace.numel(), _stream(stream))
+    _check("fvattn_route", rc)
+    return out
+
+
+def sparse_attn(g: Geom, qt, kt, vt, kv_idx, kv_cnt, scale: Optional[float] = None,
+                out: Optional[torch.Tensor] = None, sm_stats: Optional[torch.Tensor] = None,
+                workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """fvattn_sparse_attn: block-sparse attention on the kept blocks -> tiled O."""
+    _need_cuda(qt, kt, vt, kv_idx, kv_cnt, out, sm_stats)
+    if scale is None:
+        scale = 1.0 / math.sqrt(g.D)
+    if out is None:
+        out = tiled_empty(g, qt.device)
+    if workspace is None:
+        workspace = attn_workspace(g, qt.device)
+    if sm_stats is not None:
+        assert sm_stats.dtype == torch.int64 and sm_stats.numel() >= 2 * num_sms()
+    rc = load().fvattn_sparse_attn(ctypes.byref(g), _ptr(qt), _ptr(kt), _ptr(vt), _ptr(kv_idx),
+                                   _ptr(kv_cnt), float(scale), _ptr(out), _ptr(sm_stats),
+                                   _ptr(workspace), workspace.numel(), _stream(stream))
+    _check("fvattn_sparse_attn", rc)
+    return out
+
+
+def get_status(stream=None) -> int:
+    """Synchronise the stream and read/clear the device status word."""
+    return load().fvattn_get_status(_stream(stream))
+
+
+class Layer:
+    """One attention layer's buffers, allocated once and reused: the four C
+    ABI calls in order (reorder Q, K, V -> route -> sparse attention ->
+    inverse reorder)."""
+
+    def __init__(self, g: Geom, p: float, k: int, scale: Optional[float] = None, device="cuda",
+                 debug: bool = False):
+        self.g, self.p, self.k = g, p, k
+        self.scale = 1.0 / math.sqrt(g.D) if scale is None else scale
+        self.qt = tiled_empty(g, device)
+        self.kt = tiled_empty(g, device)
+        self.vt = tiled_empty(g, device)
+        self.ot = tiled_empty(g, device)
+        self.o = torch.empty((g.B, g.N, g.H, g.D), dtype=torch.bfloat16, device=device)
+        self.routed = RouteOut(kv_idx=torch.empty((g.B, g.H, g.nb, g.nb), dtype=torch.int32, device=device),
+                               kv_cnt=torch.empty((g.B, g.H, g.nb), dtype=torch.int32, device=device))
+        if debug:
+            self.routed.logits = torch.empty((g.B, g.H, g.nb, g.nb), dtype=torch.float32, device=device)
+        self.route_ws = route_workspace(g, device)
+        self.attn_ws = attn_workspace(g, device)
+        self.sm_stats = torch.zeros(2 * num_sms(), dtype=torch.int64, device=device)
+
+    def reorder_qkv(self, q, k, v, stream=None):
+        reorder(self.g, q, self.qt, stream)
+        reorder(self.g, k, self.kt, stream)
+        reorder(self.g, v, self.vt, stream)
+
+    def route(self, stream=None):
+        return route(self.g, self.qt, self.kt, self.p, self.k, self.scale, out=self.routed,
+                     workspace=self.route_ws, stream=stream)
+
+    def attend(self, stats: bool = False, stream=None):
+        return sparse_attn(self.g, self.qt, self.kt, self.vt, self.routed.kv_idx, self.routed.kv_cnt,
+                           self.scale, out=self.ot, sm_stats=self.sm_stats if stats else None,
+                           workspace=self.attn_ws, stream=stream)
+
+    def restore(self, stream=None):
+        return inverse_reorder(self.g, self.ot, self.o, stream)
+
+    def __call__(self, q, k, v, stats: bool = False, stream=None):
+        self.reorder_qkv(q, k, v, stream)
+        self.route(stream)
+        self.attend(stats, stream)
+        return self.restore(stream)
+
+
+def attention_from_host(layer: Layer, q_host, k_host, v_host, o_host, stream=None):
+    """End to end from pinned host buffers: H2D copies of raster Q, K, V, the
+    four library calls, and a D2H copy of the raster output, all on one stream."""
+    s = stream if stream is not None else torch.cuda.current_stream()
+    with torch.cuda.stream(s):
+        qd = torch.empty_like(q_host, device="cuda")
+        kd = torch.empty_like(k_host, device="cuda")
+        vd = torch.empty_like(v_host, device="cuda")
+        qd.copy_(q_host, non_blocking=True)
+        kd.copy_(k_host, non_blocking=True)
+        vd.copy_(v_host, non_blocking=True)
+        out = layer(qd, kd, vd, stream=s)
+        o_host.copy_(out, non_blocking=True)
+    return o_host

@@ -1,0 +1,172 @@
+/*
+ * fvattn.h -- C ABI of the FVAttn single-GPU hot path on B200 (sm_100a).
+ *
+ * FVAttn ("FVAttn: Adaptive Sparse Attention with Runtime Load Balancing
+ * for Video Generation", arXiv 2607.16190) builds, per attention layer, a
+ * video-aware block organisation, a Top-p plus Top-k-floor block mask from
+ * the current attention features, and then runs block-sparse attention on
+ * that mask (paperlayer.ai summary, section 3 "FVAttn Design", items
+ * "Pipeline" and "Sparse-routing frontend"; section 2 "Background and
+ * Related Work", items on Top-p, Top-k and dynamic block-sparse attention).
+ * This library exposes the four single-GPU steps of that path:
+ *
+ *   fvattn_reorder          raster tokens -> spatio-temporal tiles
+ *   fvattn_route            block mean-pooling, block scores, Top-p + Top-k
+ *   fvattn_sparse_attn      block-sparse flash attention on the kept blocks
+ *   fvattn_inverse_reorder  tiles -> raster tokens
+ *
+ * Conventions for every call:
+ *   - All tensor pointers are DEVICE pointers, 16-byte aligned, contiguous.
+ *     bf16 tensors are passed as void* holding IEEE bfloat16 values.
+ *   - The caller owns (allocates and frees) every buffer, including the
+ *     workspaces.  The library allocates and frees no device memory.
+ *   - Every call is asynchronous on the given stream (a cudaStream_t; NULL
+ *     is the legacy default stream) and never synchronises it, except
+ *     fvattn_get_status.
+ *   - Return value: FVATTN_OK or an error code below.  Argument errors are
+ *     detected on the host before anything is launched.  Errors raised
+ *     inside a kernel (a bounded wait that ran out, a kv index out of range)
+ *     are recorded in a device status word read by fvattn_get_status.
+ *   - Nothing here falls back to the CPU.
+ *
+ * Geometry (notation of the pages' video DiT setting): a layer has B
+ * sequences, H heads of dimension D, and a latent video of F frames of
+ * Hs x Ws tokens, in raster (frame, row, col) order: N = F*Hs*Ws tokens.
+ * Tiles are tf x th x tw tokens; the video is zero-padded up to
+ * Fp = ceil(F/tf)*tf (likewise Hp, Wp).  A block is one tile of
+ * bs = tf*th*tw tokens; tiles are numbered in raster tile order and the
+ * tokens inside a tile in raster order.  nb = Npad/bs blocks per head;
+ * every block holds at least one real token.
+ */
+#ifndef FVATTN_H
+#define FVATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Opaque stream handle: pass a cudaStream_t. */
+typedef struct CUstream_st *fvattn_stream_t;
+
+enum {
+    FVATTN_OK = 0,
+    FVATTN_ERR_INVALID = 1,     /* null / misaligned pointer, bad p or k, workspace too small */
+    FVATTN_ERR_UNSUPPORTED = 2, /* geometry outside the supported range */
+    FVATTN_ERR_CUDA = 3,        /* a CUDA runtime or driver call failed */
+    FVATTN_ERR_TIMEOUT = 4,     /* a bounded device wait ran out (kernel returned early) */
+    FVATTN_ERR_BOUNDS = 5       /* a kv_idx / kv_cnt entry was out of range */
+};
+
+typedef struct {
+    /* set by the caller */
+    int B, H, D;          /* batch, heads, head dim (64 or 128) */
+    int F, Hs, Ws;        /* latent frames, rows, cols */
+    int tf, th, tw;       /* tile extent; bs = tf*th*tw in {16, 32, 64, 128} */
+    /* filled by fvattn_geom_init */
+    int Fp, Hp, Wp;       /* padded extents */
+    int nbf, nby, nbx;    /* tiles along frame, row, col */
+    int bs, nb;           /* tokens per block, blocks per head (nb <= 2560) */
+    long long N, Npad;    /* raster tokens, padded tokens (= nb*bs) */
+} fvattn_geom;
+
+/* Validate the caller-set fields and fill the derived ones.
+ * Returns FVATTN_ERR_INVALID for non-positive sizes, FVATTN_ERR_UNSUPPORTED
+ * for D not in {64, 128}, bs not in {16, 32, 64, 128} or nb > 2560. */
+int fvattn_geom_init(fvattn_geom *g);
+
+/* Video-aware block organisation (paperlayer.ai summary, section 3,
+ * "Sparse-routing frontend": spatially adjacent tokens share a block).
+ *   x       [B, N, H, D] bf16, raster token order (the DiT's layout)
+ *   x_tiled [B, H, Npad, D] bf16; token (f, y, x) of head h goes to row
+ *           block*bs + offset, block = ((f/tf)*nby + y/th)*nbx + x/tw,
+ *           offset = ((f%tf)*th + y%th)*tw + x%tw; padding rows are zero.
+ * Bit copy.  x and x_tiled must not overlap. */
+int fvattn_reorder(const fvattn_geom *g, const void *x, void *x_tiled, fvattn_stream_t stream);
+
+/* Restoration of the original layout (paperlayer.ai summary, section 3,
+ * "Pipeline", last step): the exact inverse of fvattn_reorder on real
+ * tokens; padding rows are dropped.
+ *   o_tiled [B, H, Npad, D] bf16  ->  o [B, N, H, D] bf16.  Bit copy. */
+int fvattn_inverse_reorder(const fvattn_geom *g, const void *o_tiled, void *o,
+                           fvattn_stream_t stream);
+
+/* Bytes of device workspace fvattn_route needs (pooled Q and K, fp32). */
+size_t fvattn_route_workspace_size(const fvattn_geom *g);
+
+/* Sparse-routing frontend (paperlayer.ai summary, section 3,
+ * "Sparse-routing frontend": Top-p CDF thresholding and a Top-k floor;
+ * section 2: Top-p keeps the smallest cumulative-importance set, the Top-k
+ * safety floor a minimum budget).  Per (b, h):
+ *   Qp[i] = mean of the real tokens of query block i (fp32), Kp likewise;
+ *   L[i][j] = scale * Qp[i] . Kp[j]                      (fp32)
+ *   order blocks of row i by L descending, equal L by lower j;
+ *   P = softmax(L[i]); m_p = smallest prefix whose mass reaches p
+ *   (m_p = nb when p >= 1); m = max(m_p, min(k_floor, nb));
+ *   kv_idx[b,h,i,0..m) = the first m blocks of that order, ascending;
+ *   kv_cnt[b,h,i] = m.
+ * Arguments:
+ *   q_tiled, k_tiled  [B, H, Npad, D] bf16 from fvattn_reorder
+ *   p                 in (0, 1]
+ *   k_floor           >= 1
+ *   scale             softmax scale (normally 1/sqrt(D)); must be finite
+ *   kv_idx            [B, H, nb, nb] int32; entries at and after kv_cnt are
+ *                     left unwritten
+ *   kv_cnt            [B, H, nb] int32
+ *   q_pool, k_pool    optional [B, H, nb, D] fp32 outputs (may be NULL)
+ *   logits            optional [B, H, nb, nb] fp32 output of L (may be NULL)
+ *   workspace         device scratch of >= fvattn_route_workspace_size bytes,
+ *                     256-byte aligned
+ * Logits must be finite (NaN inputs give an unspecified mask). */
+int fvattn_route(const fvattn_geom *g, const void *q_tiled, const void *k_tiled,
+                 double p, int k_floor, float scale,
+                 int32_t *kv_idx, int32_t *kv_cnt,
+                 float *q_pool, float *k_pool, float *logits,
+                 void *workspace, size_t ws_bytes, fvattn_stream_t stream);
+
+/* Bytes of device workspace fvattn_sparse_attn needs (work list, head
+ * order, per-block validity masks, work counter). */
+size_t fvattn_attn_workspace_size(const fvattn_geom *g);
+
+/* Number of CTAs (one per SM) the persistent attention kernel launches on
+ * the current device; the length of each half of sm_stats. */
+int fvattn_num_sms(void);
+
+/* Dynamic block-sparse attention (paperlayer.ai summary, section 2,
+ * "Sparse Attention": dynamic block-sparse attention; section 3,
+ * "Pipeline": it runs on the materialised mask).  For each (b, h, query
+ * block i) and each real or padding query row t of block i:
+ *   O_t = softmax_u(scale * q_t . k_u) v_u  over the real tokens u of the
+ *         kv_cnt[b,h,i] blocks kv_idx[b,h,i,0..cnt)
+ * computed with bf16 tensor-core products, fp32 online softmax and fp32
+ * accumulation, written as bf16.  Work items are taken longest-first by a
+ * persistent kernel with one CTA per SM.
+ *   q_t, k_t, v_t  [B, H, Npad, D] bf16 from fvattn_reorder (padding zero)
+ *   kv_idx, kv_cnt as written by fvattn_route (each row: cnt in [1, nb],
+ *                  distinct indices in [0, nb)); out-of-range entries set
+ *                  FVATTN_ERR_BOUNDS in the status word and are skipped
+ *   o_t            [B, H, Npad, D] bf16 output (all rows written)
+ *   sm_stats       optional (may be NULL) uint64[2 * fvattn_num_sms()]:
+ *                  [0, n) busy nanoseconds of each CTA, [n, 2n) kv blocks
+ *                  each CTA attended to
+ *   workspace      >= fvattn_attn_workspace_size bytes, 256-byte aligned */
+int fvattn_sparse_attn(const fvattn_geom *g, const void *q_t, const void *k_t, const void *v_t,
+                       const int32_t *kv_idx, const int32_t *kv_cnt, float scale,
+                       void *o_t, unsigned long long *sm_stats,
+                       void *workspace, size_t ws_bytes, fvattn_stream_t stream);
+
+/* Synchronise `stream`, read and clear the device status word, and return
+ * it (FVATTN_OK, FVATTN_ERR_TIMEOUT or FVATTN_ERR_BOUNDS), or
+ * FVATTN_ERR_CUDA if the synchronisation itself failed. */
+int fvattn_get_status(fvattn_stream_t stream);
+
+/* Static string naming a status code. */
+const char *fvattn_status_string(int code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FVATTN_H */

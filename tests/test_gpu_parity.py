@@ -1,0 +1,288 @@
+"""CUDA path vs CPU oracle, element by element, on the same seeded inputs.
+
+Bars (stated where they are used):
+  - reorder / inverse reorder: bit-exact;
+  - pooled Q/K: |gpu - oracle| <= 1e-5 * rms(oracle) + 1e-6 (fp32 sums of
+    at most 128 bf16 values against fp64);
+  - logits: |gpu - oracle| <= 2e-5 * scale * |Qp| |Kp| + 1e-6;
+  - masks: the oracle's selection run on the GPU's own fp32 logits must equal
+    the GPU's kv lists exactly, except in rows the oracle flags as near ties
+    (cumulative mass within 1e-5 of p), which are counted;
+  - attention on the GPU's mask: max-abs <= 2e-2 and mean-abs <= 2e-3 over
+    real query rows (bf16 inputs, bf16 P, fp32 accumulation, bf16 output).
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from block_sparse_attention_aware_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+MAX_ABS = 2e-2
+MEAN_ABS = 2e-3
+
+
+@pytest.fixture(scope="module")
+def fv():
+    from block_sparse_attention_aware_b200 import build, fvattn
+    build.build()
+    assert torch.cuda.is_available(), "the CUDA path needs a GPU"
+    fvattn.load()
+    return fvattn
+
+
+def _bits(t):
+    return synth.bf16_bits(t)
+
+
+def _gpu_inputs(w, device="cuda", layer=0):
+    q, k, v, _ = synth.make_qkv(w, layer=layer, device=device)
+    return q.contiguous(), k.contiguous(), v.contiguous()
+
+
+def _check_mask(orc, logits_gpu, kv_idx, kv_cnt, p, k):
+    """Oracle select on the GPU logits; returns (mismatched rows, near-tie rows)."""
+    L = logits_gpu.cpu().numpy()
+    nb = L.shape[-1]
+    idx_o, cnt_o, _, tie = orc.select(L.reshape(-1, nb), p, k)
+    cnt_g = kv_cnt.cpu().numpy().reshape(-1)
+    idx_g = kv_idx.cpu().numpy().reshape(-1, nb)
+    bad = []
+    for r in np.nonzero(cnt_g != cnt_o)[0].tolist():
+        bad.append(r)
+    same_cnt = np.nonzero(cnt_g == cnt_o)[0]
+    for r in same_cnt:
+        c = cnt_g[r]
+        if not np.array_equal(idx_g[r, :c], idx_o[r, :c]):
+            bad.append(int(r))
+    bad = sorted(set(bad))
+    unexcused = [r for r in bad if not tie[r]]
+    return bad, unexcused, int(tie.sum())
+
+
+def _attn_check(orc, w, g, qt, kt, vt, ot, kv_idx, kv_cnt, items, scale):
+    """Compare GPU tiled output with the oracle on `items` (real rows only)."""
+    qb, kb, vb = _bits(qt), _bits(kt), _bits(vt)
+    ref = orc.attention(qb, kb, vb, kv_idx.cpu().numpy(), kv_cnt.cpu().numpy(), items, w, scale)
+    counts = orc.block_valid_counts(w)
+    got_all = ot.view(-1, g.bs, g.D)
+    errs = []
+    for n, it in enumerate(items):
+        blk = it % g.nb
+        real = _real_rows(w, g, blk)
+        got = got_all[it].float().cpu().numpy()[real]
+        want = ref[n][real]
+        assert len(real) == counts[blk]
+        errs.append(np.abs(got - want))
+    e = np.concatenate([x.ravel() for x in errs])
+    return float(e.max()), float(e.mean())
+
+
+_real_cache = {}
+
+
+def _real_rows(w, g, blk):
+    key = (w.F, w.Hs, w.Ws, w.tf, w.th, w.tw, blk)
+    if key not in _real_cache:
+        bx = blk % g.nbx
+        by = (blk // g.nbx) % g.nby
+        bf = blk // (g.nbx * g.nby)
+        rows = []
+        for o in range(g.bs):
+            ox, oy, of = o % w.tw, (o // w.tw) % w.th, o // (w.tw * w.th)
+            if bf * w.tf + of < w.F and by * w.th + oy < w.Hs and bx * w.tw + ox < w.Ws:
+                rows.append(o)
+        _real_cache[key] = np.array(rows)
+    return _real_cache[key]
+
+
+SMALL = [
+    ("tiny", synth.WORKLOADS["tiny"]),
+    ("pad-bs16-d64", synth.custom_workload(B=2, H=3, D=64, F=3, Hs=5, Ws=7, tf=2, th=2, tw=4, seed=5,
+                                           p=0.8, k=2, qscale="fixed", qscale_values=(0.3, 2.0, 6.0))),
+    ("pad-bs128-d128", synth.custom_workload(B=1, H=2, D=128, F=5, Hs=19, Ws=21, tf=2, th=8, tw=8, seed=6,
+                                             p=0.9, k=3, qscale="fixed", qscale_values=(1.0, 8.0))),
+    ("bs64-d128", synth.custom_workload(B=2, H=2, D=128, F=3, Hs=16, Ws=24, tf=1, th=8, tw=8, seed=7,
+                                        p=0.95, k=4, qscale="fixed", qscale_values=(0.5, 4.0))),
+    ("bs32-d64", synth.custom_workload(B=1, H=2, D=64, F=2, Hs=12, Ws=16, tf=2, th=4, tw=4, seed=8,
+                                       p=0.7, k=2, qscale="fixed", qscale_values=(1.0, 10.0))),
+    ("lowrank-bs128", synth.custom_workload(B=1, H=3, D=128, F=6, Hs=24, Ws=32, tf=2, th=8, tw=8, seed=9,
+                                            p=0.9, k=2, lowrank=True)),
+]
+
+
+@pytest.mark.parametrize("name,w", SMALL, ids=[s[0] for s in SMALL])
+def test_reorder_roundtrip_bit_exact(fv, orc, name, w):
+    g = fv.geom_of(w)
+    q, _, _ = _gpu_inputs(w)
+    qt = fv.reorder(g, q)
+    want = orc.reorder(_bits(q), w)
+    assert np.array_equal(_bits(qt), want)
+    back = fv.inverse_reorder(g, qt)
+    assert np.array_equal(_bits(back), _bits(q))
+    assert fv.get_status() == 0
+
+
+@pytest.mark.parametrize("name,w", SMALL, ids=[s[0] for s in SMALL])
+def test_route_parity(fv, orc, name, w):
+    g = fv.geom_of(w)
+    q, k, _ = _gpu_inputs(w)
+    qt, kt = fv.reorder(g, q), fv.reorder(g, k)
+    scale = 1.0 / math.sqrt(w.D)
+    r = fv.route(g, qt, kt, w.p, w.k, scale, debug=True)
+    torch.cuda.synchronize()
+    qp_o = orc.pool(_bits(qt), w)
+    kp_o = orc.pool(_bits(kt), w)
+    for got, want in ((r.q_pool, qp_o), (r.k_pool, kp_o)):
+        got = got.cpu().numpy().astype(np.float64)
+        tol = 1e-5 * np.sqrt(np.mean(want ** 2)) + 1e-6
+        assert np.max(np.abs(got - want)) <= tol
+    L_o = orc.logits(qp_o, kp_o, scale)
+    nq = np.linalg.norm(qp_o, axis=-1)[..., :, None]
+    nk = np.linalg.norm(kp_o, axis=-1)[..., None, :]
+    L_g = r.logits.cpu().numpy().astype(np.float64)
+    assert np.all(np.abs(L_g - L_o) <= 2e-5 * scale * nq * nk + 1e-6)
+    bad, unexcused, ties = _check_mask(orc, r.logits, r.kv_idx, r.kv_cnt, w.p, w.k)
+    assert unexcused == [], f"mask mismatch outside the near-tie band in rows {unexcused[:10]}"
+    cnt = r.kv_cnt.cpu().numpy()
+    assert cnt.min() >= min(w.k, g.nb) and cnt.max() <= g.nb
+    assert fv.get_status() == 0
+
+
+@pytest.mark.parametrize("name,w", SMALL, ids=[s[0] for s in SMALL])
+def test_sparse_attention_parity(fv, orc, name, w):
+    g = fv.geom_of(w)
+    q, k, v = _gpu_inputs(w)
+    layer = fv.Layer(g, w.p, w.k)
+    out = layer(q, k, v, stats=True)
+    torch.cuda.synchronize()
+    assert fv.get_status() == 0
+    items = list(range(w.B * w.H * g.nb))
+    mx, mean = _attn_check(orc, w, g, layer.qt, layer.kt, layer.vt, layer.ot, layer.routed.kv_idx,
+                           layer.routed.kv_cnt, items, layer.scale)
+    assert mx <= MAX_ABS and mean <= MEAN_ABS, (mx, mean)
+    # the raster output is the inverse reorder of the tiled one
+    assert np.array_equal(_bits(out), orc.inverse_reorder(_bits(layer.ot), w))
+    # every kept block was attended exactly once
+    st = layer.sm_stats.cpu().numpy()
+    n = fv.num_sms()
+    assert st[n:2 * n].sum() == int(layer.routed.kv_cnt.sum())
+
+
+@pytest.mark.parametrize("p,k", [(1.0, 1), (0.3, 1), (0.9, 10_000), (0.5, 3)])
+def test_attention_edge_routing(fv, orc, p, k):
+    """p = 1 (dense), a single-block Top-p, a Top-k floor above nb, mixed."""
+    w = synth.custom_workload(B=1, H=2, D=128, F=3, Hs=9, Ws=17, tf=1, th=8, tw=8, seed=21, p=p, k=k,
+                              qscale="fixed", qscale_values=(12.0, 0.2))
+    g = fv.geom_of(w)
+    q, kk, v = _gpu_inputs(w)
+    layer = fv.Layer(g, p, k, debug=True)
+    layer(q, kk, v)
+    torch.cuda.synchronize()
+    assert fv.get_status() == 0
+    cnt = layer.routed.kv_cnt.cpu().numpy()
+    if p >= 1.0 or k >= g.nb:
+        assert np.all(cnt == g.nb)
+    bad, unexcused, _ = _check_mask(orc, layer.routed.logits, layer.routed.kv_idx, layer.routed.kv_cnt, p, k)
+    assert unexcused == []
+    items = list(range(w.B * w.H * g.nb))
+    mx, mean = _attn_check(orc, w, g, layer.qt, layer.kt, layer.vt, layer.ot, layer.routed.kv_idx,
+                           layer.routed.kv_cnt, items, layer.scale)
+    assert mx <= MAX_ABS and mean <= MEAN_ABS, (mx, mean)
+
+
+def test_single_block_video(fv, orc):
+    """nb = 1: one partial block per head (a 1 x 3 x 5 latent in a 2 x 8 x 8 tile)."""
+    w = synth.custom_workload(B=1, H=2, D=128, F=1, Hs=3, Ws=5, tf=2, th=8, tw=8, seed=3, p=0.9, k=1)
+    g = fv.geom_of(w)
+    assert g.nb == 1
+    q, k, v = _gpu_inputs(w)
+    layer = fv.Layer(g, w.p, w.k)
+    out = layer(q, k, v)
+    torch.cuda.synchronize()
+    assert fv.get_status() == 0
+    qd, kd, vd = (t.double().cpu() for t in (q, k, v))
+    want = torch.nn.functional.scaled_dot_product_attention(
+        qd.permute(0, 2, 1, 3), kd.permute(0, 2, 1, 3), vd.permute(0, 2, 1, 3)).permute(0, 2, 1, 3)
+    err = (out.double().cpu() - want).abs()
+    assert err.max() <= MAX_ABS and err.mean() <= MEAN_ABS
+
+
+def test_custom_mask_through_attention(fv, orc):
+    """kv lists written by hand (not by routing), including a reversed order."""
+    w = synth.custom_workload(B=1, H=1, D=64, F=2, Hs=8, Ws=8, tf=2, th=2, tw=4, seed=2)
+    g = fv.geom_of(w)
+    q, k, v = _gpu_inputs(w)
+    qt, kt, vt = fv.reorder(g, q), fv.reorder(g, k), fv.reorder(g, v)
+    nb = g.nb
+    kv_idx = torch.zeros((1, 1, nb, nb), dtype=torch.int32)
+    kv_cnt = torch.zeros((1, 1, nb), dtype=torch.int32)
+    rng = np.random.default_rng(0)
+    for i in range(nb):
+        c = int(rng.integers(1, nb + 1))
+        sel = rng.choice(nb, size=c, replace=False)
+        if i % 2:
+            sel = sel[::-1].copy()
+        kv_idx[0, 0, i, :c] = torch.from_numpy(sel.astype(np.int32))
+        kv_cnt[0, 0, i] = c
+    kv_idx, kv_cnt = kv_idx.cuda(), kv_cnt.cuda()
+    ot = fv.sparse_attn(g, qt, kt, vt, kv_idx, kv_cnt)
+    torch.cuda.synchronize()
+    assert fv.get_status() == 0
+    mx, mean = _attn_check(orc, w, g, qt, kt, vt, ot, kv_idx, kv_cnt, list(range(nb)), 1.0 / math.sqrt(w.D))
+    assert mx <= MAX_ABS and mean <= MEAN_ABS
+
+
+def test_out_of_range_kv_is_reported_not_faulted(fv):
+    """Malformed lists (index >= nb, count 0 or > nb) are caught by the kernel's
+    own checks: status FVATTN_ERR_BOUNDS, no memory access out of range."""
+    w = synth.custom_workload(B=1, H=1, D=64, F=2, Hs=8, Ws=8, tf=2, th=2, tw=4, seed=2)
+    g = fv.geom_of(w)
+    q, k, v = _gpu_inputs(w)
+    qt, kt, vt = fv.reorder(g, q), fv.reorder(g, k), fv.reorder(g, v)
+    nb = g.nb
+    kv_idx = torch.zeros((1, 1, nb, nb), dtype=torch.int32, device="cuda")
+    kv_cnt = torch.ones((1, 1, nb), dtype=torch.int32, device="cuda")
+    kv_idx[0, 0, 1, 0] = nb + 5
+    kv_cnt[0, 0, 2] = 0
+    kv_cnt[0, 0, 3] = nb + 1
+    assert fv.get_status() == 0
+    fv.sparse_attn(g, qt, kt, vt, kv_idx, kv_cnt)
+    assert fv.get_status() == fv.ERR_BOUNDS
+    assert fv.get_status() == 0  # reading clears it
+
+
+# ---------------------------------------------------------------- full-size configurations
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name", ["480p", "720p", "cfg720p"])
+def test_full_size_sampled_parity(fv, orc, name):
+    """Full-size layer in the launch configuration the benchmark times:
+    reorder bit-exact on Q, masks exact outside near ties on every row, and
+    attention within the bar on a seeded sample of items (plus the heaviest
+    and lightest item)."""
+    w = synth.WORKLOADS[name]
+    g = fv.geom_of(w)
+    q, k, v = _gpu_inputs(w)
+    layer = fv.Layer(g, w.p, w.k, debug=True)
+    layer(q, k, v, stats=True)
+    torch.cuda.synchronize()
+    assert fv.get_status() == 0
+    qb = _bits(q)
+    assert np.array_equal(_bits(layer.qt), orc.reorder(qb, w))
+    del qb
+    bad, unexcused, ties = _check_mask(orc, layer.routed.logits, layer.routed.kv_idx, layer.routed.kv_cnt,
+                                       w.p, w.k)
+    assert unexcused == [], unexcused[:10]
+    cnt = layer.routed.kv_cnt.cpu().numpy().reshape(-1)
+    items = synth.sample_items(len(cnt), 6, seed=123)
+    items = sorted(set(items) | {int(np.argmax(cnt)), int(np.argmin(cnt))})
+    mx, mean = _attn_check(orc, w, g, layer.qt, layer.kt, layer.vt, layer.ot, layer.routed.kv_idx,
+                           layer.routed.kv_cnt, items, layer.scale)
+    assert mx <= MAX_ABS and mean <= MEAN_ABS, (mx, mean)
+    st = layer.sm_stats.cpu().numpy()
+    n = fv.num_sms()
+    assert st[n:2 * n].sum() == int(cnt.sum())
