@@ -111,7 +111,7 @@ class ClockSampler:
 
 # ---------------------------------------------------------------- CPU oracle (baseline / reference arm)
 
-def oracle_sample_time(w, qt, kt, vt, q_raster, kv_idx_full, kv_cnt_full, heads=2, items_per_head=2):
+def oracle_sample_time(w, qt, kt, vt, q_raster, kv_idx_full, kv_cnt_full, heads=4, items_per_head=12):
     """Time the oracle, as it stands, on a bounded sample of one layer and
     extrapolate to the whole layer.
 
@@ -140,7 +140,7 @@ def oracle_sample_time(w, qt, kt, vt, q_raster, kv_idx_full, kv_cnt_full, heads=
     items = []
     for h in range(heads):
         order = np.argsort(-cnt[0, h], kind="stable")
-        picks = [int(order[0]), int(order[len(order) // 2])][:items_per_head]
+        picks = [int(order[(i * len(order)) // items_per_head]) for i in range(items_per_head)]
         items += [h * nb + i for i in picks]
     t0 = time.perf_counter()
     orc.attention(qb, kb, vb, idx, cnt, items, sub, 1.0 / math.sqrt(w.D))
@@ -212,7 +212,9 @@ def run_fvattn(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
     fvattn.load()
-    w = synth.WORKLOADS[WORKLOAD]
+    w = synth.WORKLOADS[args.workload]
+    if args.heads:
+        w = synth.custom_workload(**{**w.as_dict(), "H": args.heads, "name": f"{w.name}-h{args.heads}"})
     g = fvattn.geom_of(w)
     dev = torch.device("cuda", local)
     # each rank: its own seeded replica layer
@@ -371,6 +373,9 @@ def main():
     ap.add_argument("--impl", default="fvattn", choices=["fvattn", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", default=WORKLOAD, help="named workload of synth.WORKLOADS")
+    ap.add_argument("--heads", type=int, default=0,
+                    help="profiling-size variant: the same layer with fewer heads (0 = all)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
