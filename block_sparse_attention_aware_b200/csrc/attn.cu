@@ -13,17 +13,20 @@
 // items dynamically in that order is a longest-processing-time greedy, and
 // keeping concurrent items inside one head keeps that head's K/V in L2.
 //
-// Kernel per CTA (192 threads, one CTA per SM):
-//   warp 0      producer: takes items, TMA-loads the Q tile and, per chunk of
-//               128 keys, the selected K and V blocks into a 2-stage ring,
-//               and writes the chunk's key-validity mask (padding tokens)
+// Kernel per CTA (224 threads, one CTA per SM):
+//   warp 0      K producer: takes items, TMA-loads the Q tile and, per chunk
+//               of 128 keys, the selected K blocks into a 3-stage ring, and
+//               writes the chunk's key-validity mask (padding tokens)
+//   warp 2      V producer: the same chunks' V blocks into a 2-stage ring
 //   warp 1      one lane issues tcgen05.mma: S = Q K^T into one of two TMEM
-//               S buffers, then O += P V into the TMEM O accumulator
-//   warps 2..5  softmax: one query row per thread (TMEM lane), online softmax
-//               in fp32 (exp2 on the MUFU), P rounded to bf16 into shared
-//               memory in the 128-byte-swizzled K-major layout, O rescaled
-//               in TMEM when the row maximum grows, and the epilogue
-//               (O / l -> bf16 -> global)
+//               S buffers, then O += P V into the TMEM O accumulator; a K
+//               stage is released when its S is done, a V stage when its PV is
+//   warps 3..6  softmax: one query row per thread (TMEM lane), online softmax
+//               in fp32 (exp2 on the MUFU, eight independent max and sum
+//               chains), P rounded to bf16 into shared memory in the
+//               128-byte-swizzled K-major layout, O rescaled in TMEM only
+//               when the row maximum grows by more than 2^8, and the
+//               epilogue (O / l -> bf16 -> global)
 // Every wait is bounded; a wait that runs out records FVATTN_ERR_TIMEOUT,
 // raises a CTA-wide abort flag and all roles leave their loops, so the CTA
 // always reaches the TMEM release.
@@ -34,11 +37,16 @@
 
 namespace fv {
 
-constexpr int ATT_THREADS = 192;
-constexpr int STAGES = 2;
+constexpr int ATT_THREADS = 224;        // 7 warps, see the role map above
+constexpr int K_STAGES = 3;             // K ring: a stage is free once its S = Q K^T is done
+constexpr int V_STAGES = 2;             // V ring: a stage is free once its O += P V is done
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t O_COL = 256;          // S buffers at columns 0 and 128
 constexpr unsigned long long WAIT_LIMIT_NS = 4000000000ull;
+// Lazy rescaling: the running row maximum (log2 units) is only moved, and O
+// rescaled, when a new score exceeds it by more than this; until then
+// probabilities may reach 2^8, which bf16 P and fp32 sums hold exactly enough.
+constexpr float RESCALE_THRESHOLD = 8.0f;
 
 struct AttnArgs {
     Geo g;
@@ -49,18 +57,19 @@ struct AttnArgs {
     int* counter;                // next item to hand out
     __nv_bfloat16* o;            // [B, H, Npad, D]
     unsigned long long* sm_stats;
-    float scale_log2;            // scale * log2(e)
+    float scale_log2;            // scale * log2(e), > 0
     int total_items;
 };
 
 struct __align__(8) Ctrl {
     unsigned long long q_full, q_empty;
-    unsigned long long k_full[STAGES], v_full[STAGES], kv_empty[STAGES];
+    unsigned long long k_full[K_STAGES], k_empty[K_STAGES];
+    unsigned long long v_full[V_STAGES], v_empty[V_STAGES];
     unsigned long long s_full[2], s_free[2];
     unsigned long long p_full, pv_done, o_free;
     unsigned long long item_full[2], item_empty[2];
     int item[2][4];              // bh, qb, cnt, valid
-    uint32_t mask[STAGES][4];
+    uint32_t mask[K_STAGES][4];  // key-validity bits of the chunk held by a K stage
     uint32_t tmem_base;
     int abort_flag;
     unsigned long long blocks_done;
@@ -73,8 +82,8 @@ struct Smem {
     static constexpr uint32_t P_BYTES = 128u * 128u * 2u;
     static constexpr uint32_t Q_OFF = 0;
     static constexpr uint32_t K_OFF = Q_OFF + Q_BYTES;
-    static constexpr uint32_t V_OFF = K_OFF + STAGES * KV_BYTES;
-    static constexpr uint32_t P_OFF = V_OFF + STAGES * KV_BYTES;
+    static constexpr uint32_t V_OFF = K_OFF + K_STAGES * KV_BYTES;
+    static constexpr uint32_t P_OFF = V_OFF + V_STAGES * KV_BYTES;
     static constexpr uint32_t CTRL_OFF = P_OFF + P_BYTES;
     static constexpr uint32_t TOTAL = CTRL_OFF + static_cast<uint32_t>(sizeof(Ctrl));
     // 1024 bytes of slack for the 1024-byte alignment; at least 120 KB so two
@@ -123,6 +132,19 @@ __device__ __forceinline__ bool token_real(const Geo& g, int block, int off) {
     return bf * g.tf + of < g.F && by * g.th + oy < g.Hs && bx * g.tw + ox < g.Ws;
 }
 
+// Block id of slot `s` of chunk `cl` of a kv list (lanes < nblk), range-checked.
+__device__ __forceinline__ int chunk_block(const int32_t* list, int cl, int bpc, int nblk, int lane, int nb) {
+    int j = 0;
+    if (lane < nblk) {
+        j = __ldg(list + cl * bpc + lane);
+        if (j < 0 || j >= nb) {
+            record_status(FVATTN_ERR_BOUNDS);
+            j = 0;
+        }
+    }
+    return j;
+}
+
 template <int D>
 __global__ void __launch_bounds__(ATT_THREADS, 1)
     sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -155,16 +177,19 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     if (threadIdx.x == 0) {
         mbar_init(smem_u32(&ctl.q_full), 1);
         mbar_init(smem_u32(&ctl.q_empty), 1);
-        for (int s = 0; s < STAGES; ++s) {
+        for (int s = 0; s < K_STAGES; ++s) {
             mbar_init(smem_u32(&ctl.k_full[s]), 1);
+            mbar_init(smem_u32(&ctl.k_empty[s]), 1 + 4);   // QK^T commit + 4 softmax warps (mask read)
+        }
+        for (int s = 0; s < V_STAGES; ++s) {
             mbar_init(smem_u32(&ctl.v_full[s]), 1);
-            mbar_init(smem_u32(&ctl.kv_empty[s]), 1);
+            mbar_init(smem_u32(&ctl.v_empty[s]), 1);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(smem_u32(&ctl.s_full[b]), 1);
             mbar_init(smem_u32(&ctl.s_free[b]), 4);
             mbar_init(smem_u32(&ctl.item_full[b]), 1);
-            mbar_init(smem_u32(&ctl.item_empty[b]), 5);
+            mbar_init(smem_u32(&ctl.item_empty[b]), 6);    // MMA, V producer, 4 softmax warps
         }
         mbar_init(smem_u32(&ctl.p_full), 4);
         mbar_init(smem_u32(&ctl.pv_done), 1);
@@ -188,7 +213,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     const uint32_t tmem = ctl.tmem_base;
 
     if (warp == 0) {
-        // =========================== producer
+        // =========================== K producer: items, Q tile, K blocks, masks
         int item_seq = 0;
         uint32_t c_seq = 0;
         bool ok = true;
@@ -221,7 +246,6 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                 ctl.item[slot][3] = 1;
                 mbar_arrive(smem_u32(&ctl.item_full[slot]));
             }
-            // Q tile
             if (!wait_warp(smem_u32(&ctl.q_empty), (item_seq & 1) ^ 1, abort_flag)) break;
             const int row_base = bh * static_cast<int>(g.Npad);
             if (lane == 0) {
@@ -233,54 +257,71 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
             const int32_t* list = a.kv_idx + (static_cast<long long>(bh) * g.nb + qb) * g.nb;
             const int nc = (cnt + bpc - 1) / bpc;
             for (int cl = 0; cl < nc; ++cl, ++c_seq) {
-                const int stage = c_seq % STAGES;
-                if (!wait_warp(smem_u32(&ctl.kv_empty[stage]), ((c_seq / STAGES) & 1) ^ 1, abort_flag)) {
+                const int stage = c_seq % K_STAGES;
+                if (!wait_warp(smem_u32(&ctl.k_empty[stage]), ((c_seq / K_STAGES) & 1) ^ 1, abort_flag)) {
                     ok = false;
                     break;
                 }
                 const int nblk = min(bpc, cnt - cl * bpc);
-                int j = 0;
-                if (lane < nblk) {
-                    j = __ldg(list + cl * bpc + lane);
-                    if (j < 0 || j >= g.nb) {
-                        record_status(FVATTN_ERR_BOUNDS);
-                        j = 0;
-                    }
-                }
+                const int j = chunk_block(list, cl, bpc, nblk, lane, g.nb);
                 uint32_t words[4];
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
                     const int col = q * 32 + lane;
                     const int s = col / bs;
                     const int off = col - s * bs;
-                    const int jj = __shfl_sync(0xffffffffu, j, s < 8 ? s : 0);
+                    const int jj = __shfl_sync(0xffffffffu, j, s);
                     const bool valid = (s < nblk) && token_real(g, jj, off);
                     words[q] = __ballot_sync(0xffffffffu, valid);
                 }
+                const uint32_t bar = smem_u32(&ctl.k_full[stage]);
                 if (lane == 0) {
 #pragma unroll
                     for (int q = 0; q < 4; ++q) ctl.mask[stage][q] = words[q];
+                    mbar_arrive_expect_tx(bar, static_cast<uint32_t>(nblk * bs * D * 2));
                 }
-                const uint32_t kb = sK + stage * L::KV_BYTES;
-                const uint32_t vb = sV + stage * L::KV_BYTES;
-                const uint32_t bytes = static_cast<uint32_t>(nblk * bs * D * 2);
-                // every lane < nblk holds one block id; lane 0 issues the copies
-                int jl[8];
+                __syncwarp();
+                if (lane < nblk) {
+                    const uint32_t kb = sK + stage * L::KV_BYTES + lane * bs * 128u;
 #pragma unroll
-                for (int s = 0; s < 8; ++s) jl[s] = __shfl_sync(0xffffffffu, j, s);
-                if (lane == 0) {
-                    mbar_arrive_expect_tx(smem_u32(&ctl.k_full[stage]), bytes);
-                    for (int s = 0; s < nblk; ++s)
+                    for (int h = 0; h < D / 64; ++h) tma_load_2d(kb + h * 16384u, &tmK, h * 64, row_base + j * bs, bar);
+                }
+            }
+            ++item_seq;
+        }
+    } else if (warp == 2) {
+        // =========================== V producer
+        int item_seq = 0;
+        uint32_t c_seq = 0;
+        bool ok = true;
+        while (ok) {
+            const int slot = item_seq & 1;
+            if (!wait_warp(smem_u32(&ctl.item_full[slot]), (item_seq >> 1) & 1, abort_flag)) break;
+            const int bh = ctl.item[slot][0];
+            const int qb = ctl.item[slot][1];
+            const int cnt = ctl.item[slot][2];
+            const int valid = ctl.item[slot][3];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&ctl.item_empty[slot]));
+            if (!valid) break;
+            const int row_base = bh * static_cast<int>(g.Npad);
+            const int32_t* list = a.kv_idx + (static_cast<long long>(bh) * g.nb + qb) * g.nb;
+            const int nc = (cnt + bpc - 1) / bpc;
+            for (int cl = 0; cl < nc; ++cl, ++c_seq) {
+                const int stage = c_seq % V_STAGES;
+                if (!wait_warp(smem_u32(&ctl.v_empty[stage]), ((c_seq / V_STAGES) & 1) ^ 1, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                const int nblk = min(bpc, cnt - cl * bpc);
+                const int j = chunk_block(list, cl, bpc, nblk, lane, g.nb);
+                const uint32_t bar = smem_u32(&ctl.v_full[stage]);
+                if (lane == 0) mbar_arrive_expect_tx(bar, static_cast<uint32_t>(nblk * bs * D * 2));
+                __syncwarp();
+                if (lane < nblk) {
+                    const uint32_t vb = sV + stage * L::KV_BYTES + lane * bs * 128u;
 #pragma unroll
-                        for (int h = 0; h < D / 64; ++h)
-                            tma_load_2d(kb + h * 16384u + s * bs * 128u, &tmK, h * 64, row_base + jl[s] * bs,
-                                        smem_u32(&ctl.k_full[stage]));
-                    mbar_arrive_expect_tx(smem_u32(&ctl.v_full[stage]), bytes);
-                    for (int s = 0; s < nblk; ++s)
-#pragma unroll
-                        for (int h = 0; h < D / 64; ++h)
-                            tma_load_2d(vb + h * 16384u + s * bs * 128u, &tmV, h * 64, row_base + jl[s] * bs,
-                                        smem_u32(&ctl.v_full[stage]));
+                    for (int h = 0; h < D / 64; ++h) tma_load_2d(vb + h * 16384u, &tmV, h * 64, row_base + j * bs, bar);
                 }
             }
             ++item_seq;
@@ -296,9 +337,9 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
             bool ok = true;
             // O += P V for global chunk c; `first` starts a new accumulation
             auto issue_pv = [&](uint32_t c, bool first) -> bool {
-                const int stage = c % STAGES;
+                const int stage = c % V_STAGES;
                 if (!wait_bar(smem_u32(&ctl.p_full), c & 1, abort_flag)) return false;
-                if (!wait_bar(smem_u32(&ctl.v_full[stage]), (c / STAGES) & 1, abort_flag)) return false;
+                if (!wait_bar(smem_u32(&ctl.v_full[stage]), (c / V_STAGES) & 1, abort_flag)) return false;
                 if (first && !wait_bar(smem_u32(&ctl.o_free), (item_seq & 1) ^ 1, abort_flag)) return false;
                 tc_fence_after();
                 const uint32_t vb = sV + stage * L::KV_BYTES;
@@ -308,7 +349,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                     const uint64_t bd = sw128_desc(vb + kk * 2048u, 16384u, 1024u);
                     mma_bf16_ss(tmem + O_COL, ad, bd, IDESC_PV, (first && kk == 0) ? 0u : 1u);
                 }
-                mma_commit(smem_u32(&ctl.kv_empty[stage]));
+                mma_commit(smem_u32(&ctl.v_empty[stage]));
                 mma_commit(smem_u32(&ctl.pv_done));
                 return true;
             };
@@ -325,9 +366,9 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                 tc_fence_after();
                 for (int cl = 0; cl < nc && ok; ++cl) {
                     const uint32_t c = c_seq + cl;
-                    const int stage = c % STAGES;
+                    const int stage = c % K_STAGES;
                     const int b = c & 1;
-                    if (!wait_bar(smem_u32(&ctl.k_full[stage]), (c / STAGES) & 1, abort_flag) ||
+                    if (!wait_bar(smem_u32(&ctl.k_full[stage]), (c / K_STAGES) & 1, abort_flag) ||
                         !wait_bar(smem_u32(&ctl.s_free[b]), ((c >> 1) & 1) ^ 1, abort_flag)) {
                         ok = false;
                         break;
@@ -342,6 +383,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                         mma_bf16_ss(tmem + b * 128u, ad, bd, IDESC_QK, kk > 0 ? 1u : 0u);
                     }
                     mma_commit(smem_u32(&ctl.s_full[b]));
+                    mma_commit(smem_u32(&ctl.k_empty[stage]));
                     if (cl == nc - 1) mma_commit(smem_u32(&ctl.q_empty));
                     if (cl > 0 && !issue_pv(c - 1, cl == 1)) ok = false;
                 }
@@ -353,8 +395,8 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
             ctl.blocks_done = blocks;
         }
         __syncwarp();
-    } else {
-        // =========================== softmax / correction / epilogue
+    } else if (warp >= 3) {
+        // =========================== softmax / correction / epilogue (warps 3..6)
         const int quad = warp & 3;                 // TMEM lanes 32*quad ..
         const int row = quad * 32 + lane;          // query row in the 128-row tile
         const uint32_t trow = tmem + (static_cast<uint32_t>(quad * 32) << 16);
@@ -373,51 +415,53 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
             if (lane == 0) mbar_arrive(smem_u32(&ctl.item_empty[slot]));
             if (!valid) break;
             const int nc = (cnt + bpc - 1) / bpc;
-            float m = -INFINITY, l = 0.f;
+            float m_ref = -INFINITY;   // reference maximum, log2 units
+            float l = 0.f;
             for (int cl = 0; cl < nc; ++cl) {
                 const uint32_t c = c_seq + cl;
-                const int stage = c % STAGES;
+                const int kst = c % K_STAGES;
                 const int b = c & 1;
-                if (!wait_warp(smem_u32(&ctl.k_full[stage]), (c / STAGES) & 1, abort_flag) ||
+                if (!wait_warp(smem_u32(&ctl.k_full[kst]), (c / K_STAGES) & 1, abort_flag) ||
                     !wait_warp(smem_u32(&ctl.s_full[b]), (c >> 1) & 1, abort_flag)) {
                     ok = false;
                     break;
                 }
-                uint32_t mw[4];
-#pragma unroll
-                for (int q = 0; q < 4; ++q) mw[q] = ctl.mask[stage][q];
+                const uint32_t* mrow = ctl.mask[kst];
+                const uint32_t mw0 = mrow[0], mw1 = mrow[1], mw2 = mrow[2], mw3 = mrow[3];
+                const bool partial = (mw0 & mw1 & mw2 & mw3) != 0xFFFFFFFFu;   // chunk holds padding keys
+                const uint32_t sb = trow + b * 128u;
                 tc_fence_after();
-                uint32_t sr[4][32];
+                // pass 1: row maximum of the raw scores, eight independent chains
+                float mx[8];
+                {
+                    uint32_t sr[4][32];
 #pragma unroll
-                for (int q = 0; q < 4; ++q) tmem_ld32(trow + b * 128u + q * 32u, sr[q]);
-                tmem_wait_ld();
-                tc_fence_before();
+                    for (int q = 0; q < 4; ++q) tmem_ld32(sb + q * 32u, sr[q]);
+                    tmem_wait_ld();
+                    if (partial) {
+                        const uint32_t mwq[4] = {mw0, mw1, mw2, mw3};
+#pragma unroll
+                        for (int q = 0; q < 4; ++q)
+#pragma unroll
+                            for (int i = 0; i < 32; ++i)
+                                if (!((mwq[q] >> i) & 1u)) sr[q][i] = 0xFF800000u;
+                    }
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) mx[i] = -INFINITY;
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) mx[i & 7] = fmaxf(mx[i & 7], __uint_as_float(sr[q][i]));
+                }
                 __syncwarp();
-                if (lane == 0) mbar_arrive(smem_u32(&ctl.s_free[b]));
-                // scale into log2 units, mask padding keys, row max
-                float mx = -INFINITY;
-#pragma unroll
-                for (int q = 0; q < 4; ++q)
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        float v = __uint_as_float(sr[q][i]) * sl2;
-                        v = ((mw[q] >> i) & 1u) ? v : -INFINITY;
-                        sr[q][i] = __float_as_uint(v);
-                        mx = fmaxf(mx, v);
-                    }
-                const float m_new = fmaxf(m, mx);
-                const float alpha = ex2_approx(m - m_new);
-                float sum = 0.f;
-#pragma unroll
-                for (int q = 0; q < 4; ++q)
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        float pv = ex2_approx(__uint_as_float(sr[q][i]) - m_new);
-                        sr[q][i] = __float_as_uint(pv);
-                        sum += pv;
-                    }
-                l = l * alpha + sum;
-                m = m_new;
+                if (lane == 0) mbar_arrive(smem_u32(&ctl.k_empty[kst]));   // mask consumed
+                const float mxs = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                                        fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * sl2;
+                const bool grow = mxs > m_ref + RESCALE_THRESHOLD;
+                const float m_new = grow ? mxs : m_ref;
+                const float alpha = ex2_approx(m_ref - m_new);
+                const float neg = -m_new;
+                m_ref = m_new;
                 if (cl > 0) {
                     // O and the P buffer are free once the previous PV finished
                     if (!wait_warp(smem_u32(&ctl.pv_done), (c - 1) & 1, abort_flag)) {
@@ -425,8 +469,8 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                         break;
                     }
                     tc_fence_after();
-                    if (__any_sync(0xffffffffu, alpha != 1.0f)) {
-#pragma unroll
+                    if (__any_sync(0xffffffffu, grow)) {
+#pragma unroll 1
                         for (int q = 0; q < D / 32; ++q) {
                             uint32_t o[32];
                             tmem_ld32(trow + O_COL + q * 32u, o);
@@ -438,23 +482,46 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                         tmem_wait_st();
                     }
                 }
-                // P row -> shared memory, bf16, 128-byte swizzle (K-major operand)
-                const uint32_t prow = sP + static_cast<uint32_t>(row) * 128u;
+                // pass 2, 32 columns at a time: P = 2^(s*scale*log2e - m), row sum,
+                // bf16 P row into shared memory (128-byte swizzle, K-major operand)
+                float sm[8];
 #pragma unroll
-                for (int kc = 0; kc < 16; ++kc) {
-                    const int q = kc >> 2;
-                    const int i0 = (kc & 3) * 8;
-                    uint32_t w0 = pack_bf16x2(__uint_as_float(sr[q][i0 + 0]), __uint_as_float(sr[q][i0 + 1]));
-                    uint32_t w1 = pack_bf16x2(__uint_as_float(sr[q][i0 + 2]), __uint_as_float(sr[q][i0 + 3]));
-                    uint32_t w2 = pack_bf16x2(__uint_as_float(sr[q][i0 + 4]), __uint_as_float(sr[q][i0 + 5]));
-                    uint32_t w3 = pack_bf16x2(__uint_as_float(sr[q][i0 + 6]), __uint_as_float(sr[q][i0 + 7]));
-                    const int half = kc >> 3;
-                    const int chunk = (kc & 7) ^ (row & 7);
-                    const uint32_t addr = prow + half * 16384u + chunk * 16u;
-                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(w0), "r"(w1),
-                                 "r"(w2), "r"(w3)
-                                 : "memory");
+                for (int i = 0; i < 8; ++i) sm[i] = 0.f;
+                const uint32_t prow = sP + static_cast<uint32_t>(row) * 128u;
+#pragma unroll 1
+                for (int q = 0; q < 4; ++q) {
+                    uint32_t v[32];
+                    tmem_ld32(sb + q * 32u, v);
+                    tmem_wait_ld();
+                    const uint32_t mword = q == 0 ? mw0 : (q == 1 ? mw1 : (q == 2 ? mw2 : mw3));
+                    uint32_t w[16];
+#pragma unroll
+                    for (int i = 0; i < 32; i += 2) {
+                        float p0 = ex2_approx(fmaf(__uint_as_float(v[i]), sl2, neg));
+                        float p1 = ex2_approx(fmaf(__uint_as_float(v[i + 1]), sl2, neg));
+                        if (partial) {
+                            p0 = ((mword >> i) & 1u) ? p0 : 0.f;
+                            p1 = ((mword >> (i + 1)) & 1u) ? p1 : 0.f;
+                        }
+                        sm[i & 7] += p0;
+                        sm[(i + 1) & 7] += p1;
+                        w[i >> 1] = pack_bf16x2(p0, p1);
+                    }
+                    const int half = q >> 1;
+#pragma unroll
+                    for (int k4 = 0; k4 < 4; ++k4) {
+                        const int chunk = (((q & 1) << 2) | k4) ^ (row & 7);
+                        const uint32_t addr = prow + half * 16384u + chunk * 16u;
+                        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(w[4 * k4]),
+                                     "r"(w[4 * k4 + 1]), "r"(w[4 * k4 + 2]), "r"(w[4 * k4 + 3])
+                                     : "memory");
+                    }
                 }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(&ctl.s_free[b]));   // S buffer consumed
+                const float sum = ((sm[0] + sm[1]) + (sm[2] + sm[3])) + ((sm[4] + sm[5]) + (sm[6] + sm[7]));
+                l = l * alpha + sum;
                 fence_proxy_async_smem();
                 tc_fence_before();
                 __syncwarp();
@@ -657,7 +724,7 @@ extern "C" int fvattn_sparse_attn(const fvattn_geom* gp, const void* q_t, const 
     if (!aligned16(q_t) || !aligned16(k_t) || !aligned16(v_t) || !aligned16(o_t) || !aligned16(kv_idx) ||
         !aligned16(kv_cnt) || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
         return FVATTN_ERR_INVALID;
-    if (!isfinite(scale)) return FVATTN_ERR_INVALID;
+    if (!isfinite(scale) || !(scale > 0.f)) return FVATTN_ERR_INVALID;
     if (gp->D != 64 && gp->D != 128) return FVATTN_ERR_UNSUPPORTED;
     if (gp->bs != 16 && gp->bs != 32 && gp->bs != 64 && gp->bs != 128) return FVATTN_ERR_UNSUPPORTED;
     if (gp->nb <= 0 || gp->nb > 2560) return FVATTN_ERR_UNSUPPORTED;

@@ -141,8 +141,8 @@ int fvattn_num_sms(void);
  *   O_t = softmax_u(scale * q_t . k_u) v_u  over the real tokens u of the
  *         kv_cnt[b,h,i] blocks kv_idx[b,h,i,0..cnt)
  * computed with bf16 tensor-core products, fp32 online softmax and fp32
- * accumulation, written as bf16.  Work items are taken longest-first by a
- * persistent kernel with one CTA per SM.
+ * accumulation, written as bf16.  scale must be finite and > 0.  Work items
+ * are taken longest-first by a persistent kernel with one CTA per SM.
  *   q_t, k_t, v_t  [B, H, Npad, D] bf16 from fvattn_reorder (padding zero)
  *   kv_idx, kv_cnt as written by fvattn_route (each row: cnt in [1, nb],
  *                  distinct indices in [0, nb)); out-of-range entries set
