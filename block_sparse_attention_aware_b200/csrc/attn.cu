@@ -20,11 +20,13 @@
 //   warp 2      V producer: the same chunks' V blocks into a 2-stage ring
 //   warp 1      one lane issues tcgen05.mma: S = Q K^T into one of two TMEM
 //               S buffers, then O += P V into the TMEM O accumulator; a K
-//               stage is released when its S is done, a V stage when its PV is
+//               stage is released when its S is done, a V stage and a P
+//               buffer when their PV is
 //   warps 3..6  softmax: one query row per thread (TMEM lane), online softmax
 //               in fp32 (exp2 on the MUFU, eight independent max and sum
-//               chains), P rounded to bf16 into shared memory in the
-//               128-byte-swizzled K-major layout, O rescaled in TMEM only
+//               chains), P rounded to bf16 into one of two shared-memory P
+//               tiles (128-byte-swizzled K-major layout), so the exp pass of
+//               chunk c+1 overlaps the PV of chunk c; O rescaled in TMEM only
 //               when the row maximum grows by more than 2^8, and the
 //               epilogue (O / l -> bf16 -> global)
 // Every wait is bounded; a wait that runs out records FVATTN_ERR_TIMEOUT,
@@ -38,8 +40,9 @@
 namespace fv {
 
 constexpr int ATT_THREADS = 224;        // 7 warps, see the role map above
-constexpr int K_STAGES = 3;             // K ring: a stage is free once its S = Q K^T is done
+constexpr int MAX_K_STAGES = 3;         // K ring: a stage is free once its S = Q K^T is done
 constexpr int V_STAGES = 2;             // V ring: a stage is free once its O += P V is done
+constexpr uint32_t MAX_DYN_SMEM = 232448;   // sm_100 opt-in shared memory per block
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t O_COL = 256;          // S buffers at columns 0 and 128
 constexpr unsigned long long WAIT_LIMIT_NS = 4000000000ull;
@@ -63,13 +66,14 @@ struct AttnArgs {
 
 struct __align__(8) Ctrl {
     unsigned long long q_full, q_empty;
-    unsigned long long k_full[K_STAGES], k_empty[K_STAGES];
+    unsigned long long k_full[MAX_K_STAGES], k_empty[MAX_K_STAGES];
     unsigned long long v_full[V_STAGES], v_empty[V_STAGES];
     unsigned long long s_full[2], s_free[2];
-    unsigned long long p_full, pv_done, o_free;
+    unsigned long long p_full, o_free;
+    unsigned long long p_free[2];        // P buffer b: the PV that read it is done
     unsigned long long item_full[2], item_empty[2];
     int item[2][4];              // bh, qb, cnt, valid
-    uint32_t mask[K_STAGES][4];  // key-validity bits of the chunk held by a K stage
+    uint32_t mask[MAX_K_STAGES][4];  // key-validity bits of the chunk held by a K stage
     uint32_t tmem_base;
     int abort_flag;
     unsigned long long blocks_done;
@@ -79,16 +83,23 @@ template <int D>
 struct Smem {
     static constexpr uint32_t Q_BYTES = 128u * D * 2u;   // D/64 halves of 16 KB
     static constexpr uint32_t KV_BYTES = 128u * D * 2u;
-    static constexpr uint32_t P_BYTES = 128u * 128u * 2u;
+    static constexpr uint32_t P_BYTES = 128u * 128u * 2u; // one P tile; two are kept
+    static constexpr uint32_t base_total(int ks) {
+        return Q_BYTES + (ks + V_STAGES) * KV_BYTES + 2 * P_BYTES + static_cast<uint32_t>(sizeof(Ctrl));
+    }
+    // K ring depth: 3 stages when they fit, else 2.
+    static constexpr int KS = base_total(3) <= MAX_DYN_SMEM ? 3 : 2;
     static constexpr uint32_t Q_OFF = 0;
     static constexpr uint32_t K_OFF = Q_OFF + Q_BYTES;
-    static constexpr uint32_t V_OFF = K_OFF + K_STAGES * KV_BYTES;
+    static constexpr uint32_t V_OFF = K_OFF + KS * KV_BYTES;
     static constexpr uint32_t P_OFF = V_OFF + V_STAGES * KV_BYTES;
-    static constexpr uint32_t CTRL_OFF = P_OFF + P_BYTES;
+    static constexpr uint32_t CTRL_OFF = P_OFF + 2 * P_BYTES;
     static constexpr uint32_t TOTAL = CTRL_OFF + static_cast<uint32_t>(sizeof(Ctrl));
-    // 1024 bytes of slack for the 1024-byte alignment; at least 120 KB so two
-    // CTAs never share an SM (each holds all 512 TMEM columns).
-    static constexpr uint32_t ALLOC = TOTAL + 1024 > 120u * 1024u ? TOTAL + 1024 : 120u * 1024u;
+    // Dynamic shared memory starts 1024-byte aligned on sm_100 (the kernel
+    // checks); at least 120 KB so two CTAs never share an SM (each holds all
+    // 512 TMEM columns).
+    static constexpr uint32_t ALLOC = TOTAL > 120u * 1024u ? TOTAL : 120u * 1024u;
+    static_assert(ALLOC <= MAX_DYN_SMEM, "shared-memory layout too large");
 };
 
 // Bounded mbarrier wait.  Returns false if the CTA aborted or the wait ran
@@ -120,19 +131,20 @@ __device__ __forceinline__ bool wait_warp(uint32_t bar, uint32_t parity, volatil
     return __all_sync(0xffffffffu, ok);
 }
 
-__device__ __forceinline__ bool token_real(const Geo& g, int block, int off) {
-    int bx = block % g.nbx;
-    int rest = block / g.nbx;
-    int by = rest % g.nby;
-    int bf = rest / g.nby;
-    int ox = off % g.tw;
-    int r2 = off / g.tw;
-    int oy = r2 % g.th;
-    int of = r2 / g.th;
-    return bf * g.tf + of < g.F && by * g.th + oy < g.Hs && bx * g.tw + ox < g.Ws;
+// Real extent of a tile: frames, rows and cols that hold tokens, packed as
+// nf | ny << 8 | nx << 16 (each <= 128).
+__device__ __forceinline__ int block_extent(const Geo& g, int block) {
+    const int bx = block % g.nbx;
+    const int rest = block / g.nbx;
+    const int by = rest % g.nby;
+    const int bf = rest / g.nby;
+    const int nf = min(g.tf, g.F - bf * g.tf);
+    const int ny = min(g.th, g.Hs - by * g.th);
+    const int nx = min(g.tw, g.Ws - bx * g.tw);
+    return nf | (ny << 8) | (nx << 16);
 }
 
-// Block id of slot `s` of chunk `cl` of a kv list (lanes < nblk), range-checked.
+// Block id of slot `lane` of chunk `cl` of a kv list (lanes < nblk), range-checked.
 __device__ __forceinline__ int chunk_block(const int32_t* list, int cl, int bpc, int nblk, int lane, int nb) {
     int j = 0;
     if (lane < nblk) {
@@ -150,9 +162,14 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const AttnArgs a) {
     using L = Smem<D>;
-    extern __shared__ unsigned char att_smem_raw[];
-    unsigned char* smem = reinterpret_cast<unsigned char*>(
-        (reinterpret_cast<uintptr_t>(att_smem_raw) + 1023u) & ~static_cast<uintptr_t>(1023u));
+    constexpr int KS = L::KS;
+    extern __shared__ __align__(1024) unsigned char smem[];
+    // The 128-byte swizzle of TMA and of the tcgen05 operand descriptors
+    // needs 1024-byte aligned tiles.
+    if (smem_u32(smem) & 1023u) {
+        if (threadIdx.x == 0) record_status(FVATTN_ERR_UNSUPPORTED);
+        return;
+    }
     Ctrl& ctl = *reinterpret_cast<Ctrl*>(smem + L::CTRL_OFF);
     const uint32_t sbase = smem_u32(smem);
     const uint32_t sQ = sbase + L::Q_OFF;
@@ -177,7 +194,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     if (threadIdx.x == 0) {
         mbar_init(smem_u32(&ctl.q_full), 1);
         mbar_init(smem_u32(&ctl.q_empty), 1);
-        for (int s = 0; s < K_STAGES; ++s) {
+        for (int s = 0; s < KS; ++s) {
             mbar_init(smem_u32(&ctl.k_full[s]), 1);
             mbar_init(smem_u32(&ctl.k_empty[s]), 1 + 4);   // QK^T commit + 4 softmax warps (mask read)
         }
@@ -192,7 +209,8 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
             mbar_init(smem_u32(&ctl.item_empty[b]), 6);    // MMA, V producer, 4 softmax warps
         }
         mbar_init(smem_u32(&ctl.p_full), 4);
-        mbar_init(smem_u32(&ctl.pv_done), 1);
+        mbar_init(smem_u32(&ctl.p_free[0]), 1);
+        mbar_init(smem_u32(&ctl.p_free[1]), 1);
         mbar_init(smem_u32(&ctl.o_free), 4);
         ctl.abort_flag = 0;
         ctl.blocks_done = 0ull;
@@ -214,6 +232,18 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
 
     if (warp == 0) {
         // =========================== K producer: items, Q tile, K blocks, masks
+        // Column col = q*32 + lane of a chunk is token `off` of slot `slot`;
+        // its frame / row / col offsets inside the tile never change.
+        int c_slot[4], c_of[4], c_oy[4], c_ox[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int col = q * 32 + lane;
+            c_slot[q] = col / bs;
+            const int off = col - c_slot[q] * bs;
+            c_ox[q] = off % g.tw;
+            c_oy[q] = (off / g.tw) % g.th;
+            c_of[q] = off / (g.tw * g.th);
+        }
         int item_seq = 0;
         uint32_t c_seq = 0;
         bool ok = true;
@@ -256,22 +286,22 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
             }
             const int32_t* list = a.kv_idx + (static_cast<long long>(bh) * g.nb + qb) * g.nb;
             const int nc = (cnt + bpc - 1) / bpc;
+            int j_next = chunk_block(list, 0, bpc, min(bpc, cnt), lane, g.nb);
             for (int cl = 0; cl < nc; ++cl, ++c_seq) {
-                const int stage = c_seq % K_STAGES;
-                if (!wait_warp(smem_u32(&ctl.k_empty[stage]), ((c_seq / K_STAGES) & 1) ^ 1, abort_flag)) {
+                const int stage = c_seq % KS;
+                const int nblk = min(bpc, cnt - cl * bpc);
+                const int j = j_next;
+                if (cl + 1 < nc) j_next = chunk_block(list, cl + 1, bpc, min(bpc, cnt - (cl + 1) * bpc), lane, g.nb);
+                const int ext = lane < nblk ? block_extent(g, j) : 0;
+                if (!wait_warp(smem_u32(&ctl.k_empty[stage]), ((c_seq / KS) & 1) ^ 1, abort_flag)) {
                     ok = false;
                     break;
                 }
-                const int nblk = min(bpc, cnt - cl * bpc);
-                const int j = chunk_block(list, cl, bpc, nblk, lane, g.nb);
                 uint32_t words[4];
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
-                    const int col = q * 32 + lane;
-                    const int s = col / bs;
-                    const int off = col - s * bs;
-                    const int jj = __shfl_sync(0xffffffffu, j, s);
-                    const bool valid = (s < nblk) && token_real(g, jj, off);
+                    const int e = __shfl_sync(0xffffffffu, ext, c_slot[q]);
+                    const bool valid = (c_of[q] < (e & 255)) && (c_oy[q] < ((e >> 8) & 255)) && (c_ox[q] < (e >> 16));
                     words[q] = __ballot_sync(0xffffffffu, valid);
                 }
                 const uint32_t bar = smem_u32(&ctl.k_full[stage]);
@@ -307,14 +337,16 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
             const int row_base = bh * static_cast<int>(g.Npad);
             const int32_t* list = a.kv_idx + (static_cast<long long>(bh) * g.nb + qb) * g.nb;
             const int nc = (cnt + bpc - 1) / bpc;
+            int j_next = chunk_block(list, 0, bpc, min(bpc, cnt), lane, g.nb);
             for (int cl = 0; cl < nc; ++cl, ++c_seq) {
                 const int stage = c_seq % V_STAGES;
+                const int nblk = min(bpc, cnt - cl * bpc);
+                const int j = j_next;
+                if (cl + 1 < nc) j_next = chunk_block(list, cl + 1, bpc, min(bpc, cnt - (cl + 1) * bpc), lane, g.nb);
                 if (!wait_warp(smem_u32(&ctl.v_empty[stage]), ((c_seq / V_STAGES) & 1) ^ 1, abort_flag)) {
                     ok = false;
                     break;
                 }
-                const int nblk = min(bpc, cnt - cl * bpc);
-                const int j = chunk_block(list, cl, bpc, nblk, lane, g.nb);
                 const uint32_t bar = smem_u32(&ctl.v_full[stage]);
                 if (lane == 0) mbar_arrive_expect_tx(bar, static_cast<uint32_t>(nblk * bs * D * 2));
                 __syncwarp();
@@ -343,14 +375,15 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                 if (first && !wait_bar(smem_u32(&ctl.o_free), (item_seq & 1) ^ 1, abort_flag)) return false;
                 tc_fence_after();
                 const uint32_t vb = sV + stage * L::KV_BYTES;
+                const uint32_t pb = sP + (c & 1) * L::P_BYTES;
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
-                    const uint64_t ad = sw128_desc(sP + (kk >> 2) * 16384u + (kk & 3) * 32u, 16u, 1024u);
+                    const uint64_t ad = sw128_desc(pb + (kk >> 2) * 16384u + (kk & 3) * 32u, 16u, 1024u);
                     const uint64_t bd = sw128_desc(vb + kk * 2048u, 16384u, 1024u);
                     mma_bf16_ss(tmem + O_COL, ad, bd, IDESC_PV, (first && kk == 0) ? 0u : 1u);
                 }
                 mma_commit(smem_u32(&ctl.v_empty[stage]));
-                mma_commit(smem_u32(&ctl.pv_done));
+                mma_commit(smem_u32(&ctl.p_free[c & 1]));
                 return true;
             };
             while (ok) {
@@ -366,9 +399,9 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                 tc_fence_after();
                 for (int cl = 0; cl < nc && ok; ++cl) {
                     const uint32_t c = c_seq + cl;
-                    const int stage = c % K_STAGES;
+                    const int stage = c % KS;
                     const int b = c & 1;
-                    if (!wait_bar(smem_u32(&ctl.k_full[stage]), (c / K_STAGES) & 1, abort_flag) ||
+                    if (!wait_bar(smem_u32(&ctl.k_full[stage]), (c / KS) & 1, abort_flag) ||
                         !wait_bar(smem_u32(&ctl.s_free[b]), ((c >> 1) & 1) ^ 1, abort_flag)) {
                         ok = false;
                         break;
@@ -419,9 +452,9 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
             float l = 0.f;
             for (int cl = 0; cl < nc; ++cl) {
                 const uint32_t c = c_seq + cl;
-                const int kst = c % K_STAGES;
+                const int kst = c % KS;
                 const int b = c & 1;
-                if (!wait_warp(smem_u32(&ctl.k_full[kst]), (c / K_STAGES) & 1, abort_flag) ||
+                if (!wait_warp(smem_u32(&ctl.k_full[kst]), (c / KS) & 1, abort_flag) ||
                     !wait_warp(smem_u32(&ctl.s_full[b]), (c >> 1) & 1, abort_flag)) {
                     ok = false;
                     break;
@@ -462,59 +495,51 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                 const float alpha = ex2_approx(m_ref - m_new);
                 const float neg = -m_new;
                 m_ref = m_new;
-                if (cl > 0) {
-                    // O and the P buffer are free once the previous PV finished
-                    if (!wait_warp(smem_u32(&ctl.pv_done), (c - 1) & 1, abort_flag)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    if (__any_sync(0xffffffffu, grow)) {
-#pragma unroll 1
-                        for (int q = 0; q < D / 32; ++q) {
-                            uint32_t o[32];
-                            tmem_ld32(trow + O_COL + q * 32u, o);
-                            tmem_wait_ld();
-#pragma unroll
-                            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-                            tmem_st32(trow + O_COL + q * 32u, o);
-                        }
-                        tmem_wait_st();
-                    }
+                // P buffer b was last read by the PV of chunk c-2
+                if (!wait_warp(smem_u32(&ctl.p_free[b]), ((c >> 1) & 1) ^ 1, abort_flag)) {
+                    ok = false;
+                    break;
                 }
                 // pass 2, 32 columns at a time: P = 2^(s*scale*log2e - m), row sum,
                 // bf16 P row into shared memory (128-byte swizzle, K-major operand)
                 float sm[8];
 #pragma unroll
                 for (int i = 0; i < 8; ++i) sm[i] = 0.f;
-                const uint32_t prow = sP + static_cast<uint32_t>(row) * 128u;
+                const uint32_t prow = sP + b * L::P_BYTES + static_cast<uint32_t>(row) * 128u;
+                // two 32-column groups per step: both TMEM loads are in
+                // flight together
 #pragma unroll 1
-                for (int q = 0; q < 4; ++q) {
-                    uint32_t v[32];
-                    tmem_ld32(sb + q * 32u, v);
+                for (int q2 = 0; q2 < 4; q2 += 2) {
+                    uint32_t v[2][32];
+                    tmem_ld32(sb + q2 * 32u, v[0]);
+                    tmem_ld32(sb + q2 * 32u + 32u, v[1]);
                     tmem_wait_ld();
-                    const uint32_t mword = q == 0 ? mw0 : (q == 1 ? mw1 : (q == 2 ? mw2 : mw3));
-                    uint32_t w[16];
 #pragma unroll
-                    for (int i = 0; i < 32; i += 2) {
-                        float p0 = ex2_approx(fmaf(__uint_as_float(v[i]), sl2, neg));
-                        float p1 = ex2_approx(fmaf(__uint_as_float(v[i + 1]), sl2, neg));
-                        if (partial) {
-                            p0 = ((mword >> i) & 1u) ? p0 : 0.f;
-                            p1 = ((mword >> (i + 1)) & 1u) ? p1 : 0.f;
+                    for (int hq = 0; hq < 2; ++hq) {
+                        const int q = q2 + hq;
+                        const uint32_t mword = q == 0 ? mw0 : (q == 1 ? mw1 : (q == 2 ? mw2 : mw3));
+                        uint32_t w[16];
+#pragma unroll
+                        for (int i = 0; i < 32; i += 2) {
+                            float p0 = ex2_approx(fmaf(__uint_as_float(v[hq][i]), sl2, neg));
+                            float p1 = ex2_approx(fmaf(__uint_as_float(v[hq][i + 1]), sl2, neg));
+                            if (partial) {
+                                p0 = ((mword >> i) & 1u) ? p0 : 0.f;
+                                p1 = ((mword >> (i + 1)) & 1u) ? p1 : 0.f;
+                            }
+                            sm[i & 7] += p0;
+                            sm[(i + 1) & 7] += p1;
+                            w[i >> 1] = pack_bf16x2(p0, p1);
                         }
-                        sm[i & 7] += p0;
-                        sm[(i + 1) & 7] += p1;
-                        w[i >> 1] = pack_bf16x2(p0, p1);
-                    }
-                    const int half = q >> 1;
+                        const int half = q >> 1;
 #pragma unroll
-                    for (int k4 = 0; k4 < 4; ++k4) {
-                        const int chunk = (((q & 1) << 2) | k4) ^ (row & 7);
-                        const uint32_t addr = prow + half * 16384u + chunk * 16u;
-                        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(w[4 * k4]),
-                                     "r"(w[4 * k4 + 1]), "r"(w[4 * k4 + 2]), "r"(w[4 * k4 + 3])
-                                     : "memory");
+                        for (int k4 = 0; k4 < 4; ++k4) {
+                            const int chunk = (((q & 1) << 2) | k4) ^ (row & 7);
+                            const uint32_t addr = prow + half * 16384u + chunk * 16u;
+                            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(w[4 * k4]),
+                                         "r"(w[4 * k4 + 1]), "r"(w[4 * k4 + 2]), "r"(w[4 * k4 + 3])
+                                         : "memory");
+                        }
                     }
                 }
                 tc_fence_before();
@@ -522,6 +547,26 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                 if (lane == 0) mbar_arrive(smem_u32(&ctl.s_free[b]));   // S buffer consumed
                 const float sum = ((sm[0] + sm[1]) + (sm[2] + sm[3])) + ((sm[4] + sm[5]) + (sm[6] + sm[7]));
                 l = l * alpha + sum;
+                if (cl > 0 && __any_sync(0xffffffffu, grow)) {
+                    // the row maximum moved: O must be rescaled before PV(c)
+                    // adds to it, i.e. after PV(c-1) is done
+                    const uint32_t cp = c - 1;
+                    if (!wait_warp(smem_u32(&ctl.p_free[cp & 1]), (cp >> 1) & 1, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+#pragma unroll 1
+                    for (int q = 0; q < D / 32; ++q) {
+                        uint32_t o[32];
+                        tmem_ld32(trow + O_COL + q * 32u, o);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+                        tmem_st32(trow + O_COL + q * 32u, o);
+                    }
+                    tmem_wait_st();
+                }
                 fence_proxy_async_smem();
                 tc_fence_before();
                 __syncwarp();
@@ -530,7 +575,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
             if (!ok) break;
             // epilogue: wait for the last PV, normalise, store bf16
             const uint32_t c_last = c_seq + nc - 1;
-            if (!wait_warp(smem_u32(&ctl.pv_done), c_last & 1, abort_flag)) break;
+            if (!wait_warp(smem_u32(&ctl.p_free[c_last & 1]), (c_last >> 1) & 1, abort_flag)) break;
             tc_fence_after();
             const float inv_l = 1.0f / l;
             __nv_bfloat16* orow = a.o + ((static_cast<long long>(bh) * g.Npad) + static_cast<long long>(qb) * bs + row) * D;
