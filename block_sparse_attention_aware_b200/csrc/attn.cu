@@ -39,12 +39,13 @@
 
 namespace fv {
 
-constexpr int ATT_THREADS = 224;        // 7 warps, see the role map above
+constexpr int SOFTMAX_WARPS = 8;        // two groups of four warps
+constexpr int ATT_THREADS = 32 * (3 + SOFTMAX_WARPS);
 constexpr int MAX_K_STAGES = 3;         // K ring: a stage is free once its S = Q K^T is done
 constexpr int V_STAGES = 2;             // V ring: a stage is free once its O += P V is done
 constexpr uint32_t MAX_DYN_SMEM = 232448;   // sm_100 opt-in shared memory per block
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t O_COL = 256;          // S buffers at columns 0 and 128
+constexpr uint32_t O_COL = 256;          // S_w at columns 128*w, O_w at 256 + 128*w
 constexpr unsigned long long WAIT_LIMIT_NS = 4000000000ull;
 // Lazy rescaling: the running row maximum (log2 units) is only moved, and O
 // rescaled, when a new score exceeds it by more than this; until then
@@ -64,26 +65,29 @@ struct AttnArgs {
     int total_items;
 };
 
-struct __align__(8) Ctrl {
+struct __align__(16) Ctrl {
     unsigned long long q_full, q_empty;
     unsigned long long k_full[MAX_K_STAGES], k_empty[MAX_K_STAGES];
     unsigned long long v_full[V_STAGES], v_empty[V_STAGES];
-    unsigned long long s_full[2], s_free[2];
-    unsigned long long p_full, o_free;
-    unsigned long long p_free[2];        // P buffer b: the PV that read it is done
+    unsigned long long s_full[2], s_free[2];   // per softmax group w: S_w written / read
+    unsigned long long p_full[2], p_free[2];   // per group: P_w written / its PV done
+    unsigned long long o_free;                 // both O accumulators read by the epilogue
+    unsigned long long mrg_full, mrg_empty;    // end-of-item exchange of (m, l)
     unsigned long long item_full[2], item_empty[2];
+    unsigned long long blocks_done;
     int item[2][4];              // bh, qb, cnt, valid
     uint32_t mask[MAX_K_STAGES][4];  // key-validity bits of the chunk held by a K stage
     uint32_t tmem_base;
     int abort_flag;
-    unsigned long long blocks_done;
+    float mrg_m[2][128];         // [group][row] running maximum (log2 units)
+    float mrg_l[2][128];         // [group][row] running sum
 };
 
 template <int D>
 struct Smem {
     static constexpr uint32_t Q_BYTES = 128u * D * 2u;   // D/64 halves of 16 KB
     static constexpr uint32_t KV_BYTES = 128u * D * 2u;
-    static constexpr uint32_t P_BYTES = 128u * 128u * 2u; // one P tile; two are kept
+    static constexpr uint32_t P_BYTES = 128u * 128u * 2u; // one P tile per softmax group
     static constexpr uint32_t base_total(int ks) {
         return Q_BYTES + (ks + V_STAGES) * KV_BYTES + 2 * P_BYTES + static_cast<uint32_t>(sizeof(Ctrl));
     }
@@ -196,22 +200,23 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         mbar_init(smem_u32(&ctl.q_empty), 1);
         for (int s = 0; s < KS; ++s) {
             mbar_init(smem_u32(&ctl.k_full[s]), 1);
-            mbar_init(smem_u32(&ctl.k_empty[s]), 1 + 4);   // QK^T commit + 4 softmax warps (mask read)
+            mbar_init(smem_u32(&ctl.k_empty[s]), 1 + 4);   // QK^T commit + the owning group's mask read
         }
         for (int s = 0; s < V_STAGES; ++s) {
             mbar_init(smem_u32(&ctl.v_full[s]), 1);
             mbar_init(smem_u32(&ctl.v_empty[s]), 1);
         }
-        for (int b = 0; b < 2; ++b) {
-            mbar_init(smem_u32(&ctl.s_full[b]), 1);
-            mbar_init(smem_u32(&ctl.s_free[b]), 4);
-            mbar_init(smem_u32(&ctl.item_full[b]), 1);
-            mbar_init(smem_u32(&ctl.item_empty[b]), 6);    // MMA, V producer, 4 softmax warps
+        for (int w = 0; w < 2; ++w) {
+            mbar_init(smem_u32(&ctl.s_full[w]), 1);
+            mbar_init(smem_u32(&ctl.s_free[w]), 4);
+            mbar_init(smem_u32(&ctl.p_full[w]), 4);
+            mbar_init(smem_u32(&ctl.p_free[w]), 1);
+            mbar_init(smem_u32(&ctl.item_full[w]), 1);
+            mbar_init(smem_u32(&ctl.item_empty[w]), 2 + SOFTMAX_WARPS);  // MMA, V producer, softmax
         }
-        mbar_init(smem_u32(&ctl.p_full), 4);
-        mbar_init(smem_u32(&ctl.p_free[0]), 1);
-        mbar_init(smem_u32(&ctl.p_free[1]), 1);
-        mbar_init(smem_u32(&ctl.o_free), 4);
+        mbar_init(smem_u32(&ctl.o_free), SOFTMAX_WARPS);
+        mbar_init(smem_u32(&ctl.mrg_full), SOFTMAX_WARPS);
+        mbar_init(smem_u32(&ctl.mrg_empty), SOFTMAX_WARPS);
         ctl.abort_flag = 0;
         ctl.blocks_done = 0ull;
         fence_mbar_init();
@@ -360,30 +365,36 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         }
     } else if (warp == 1) {
         // =========================== MMA issuer (one lane)
+        // Chunk c of the CTA's stream goes to softmax group w = c & 1: S_w,
+        // P_w and O_w.  n[w] counts the chunks group w has been given.
         if (lane == 0) {
             constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, 128, false);
             constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, D, true);
             int item_seq = 0;
             uint32_t c_seq = 0;
+            uint32_t nq0 = 0u, nq1 = 0u;   // QKs issued per group
+            uint32_t np0 = 0u, np1 = 0u;   // PVs issued per group
             unsigned long long blocks = 0;
             bool ok = true;
-            // O += P V for global chunk c; `first` starts a new accumulation
+            // O_w += P_w V for chunk c; `first` starts group w's accumulation
             auto issue_pv = [&](uint32_t c, bool first) -> bool {
+                const int w = c & 1;
                 const int stage = c % V_STAGES;
-                if (!wait_bar(smem_u32(&ctl.p_full), c & 1, abort_flag)) return false;
+                if (!wait_bar(smem_u32(&ctl.p_full[w]), (w ? np1 : np0) & 1, abort_flag)) return false;
                 if (!wait_bar(smem_u32(&ctl.v_full[stage]), (c / V_STAGES) & 1, abort_flag)) return false;
-                if (first && !wait_bar(smem_u32(&ctl.o_free), (item_seq & 1) ^ 1, abort_flag)) return false;
                 tc_fence_after();
                 const uint32_t vb = sV + stage * L::KV_BYTES;
-                const uint32_t pb = sP + (c & 1) * L::P_BYTES;
+                const uint32_t pb = sP + w * L::P_BYTES;
+                const uint32_t od = tmem + O_COL + static_cast<uint32_t>(w) * 128u;
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
                     const uint64_t ad = sw128_desc(pb + (kk >> 2) * 16384u + (kk & 3) * 32u, 16u, 1024u);
                     const uint64_t bd = sw128_desc(vb + kk * 2048u, 16384u, 1024u);
-                    mma_bf16_ss(tmem + O_COL, ad, bd, IDESC_PV, (first && kk == 0) ? 0u : 1u);
+                    mma_bf16_ss(od, ad, bd, IDESC_PV, (first && kk == 0) ? 0u : 1u);
                 }
                 mma_commit(smem_u32(&ctl.v_empty[stage]));
-                mma_commit(smem_u32(&ctl.p_free[c & 1]));
+                mma_commit(smem_u32(&ctl.p_free[w]));
+                if (w) ++np1; else ++np0;
                 return true;
             };
             while (ok) {
@@ -400,9 +411,9 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                 for (int cl = 0; cl < nc && ok; ++cl) {
                     const uint32_t c = c_seq + cl;
                     const int stage = c % KS;
-                    const int b = c & 1;
+                    const int w = c & 1;
                     if (!wait_bar(smem_u32(&ctl.k_full[stage]), (c / KS) & 1, abort_flag) ||
-                        !wait_bar(smem_u32(&ctl.s_free[b]), ((c >> 1) & 1) ^ 1, abort_flag)) {
+                        !wait_bar(smem_u32(&ctl.s_free[w]), ((w ? nq1 : nq0) & 1) ^ 1, abort_flag)) {
                         ok = false;
                         break;
                     }
@@ -413,29 +424,48 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                         const uint32_t off = (kk >> 2) * 16384u + (kk & 3) * 32u;
                         const uint64_t ad = sw128_desc(sQ + off, 16u, 1024u);
                         const uint64_t bd = sw128_desc(kb + off, 16u, 1024u);
-                        mma_bf16_ss(tmem + b * 128u, ad, bd, IDESC_QK, kk > 0 ? 1u : 0u);
+                        mma_bf16_ss(tmem + static_cast<uint32_t>(w) * 128u, ad, bd, IDESC_QK, kk > 0 ? 1u : 0u);
                     }
-                    mma_commit(smem_u32(&ctl.s_full[b]));
+                    mma_commit(smem_u32(&ctl.s_full[w]));
                     mma_commit(smem_u32(&ctl.k_empty[stage]));
+                    if (w) ++nq1; else ++nq0;
                     if (cl == nc - 1) mma_commit(smem_u32(&ctl.q_empty));
-                    if (cl > 0 && !issue_pv(c - 1, cl == 1)) ok = false;
+                    if (cl > 0) {
+                        // the item's first PV waits until the previous item's
+                        // epilogue has read both accumulators
+                        if (cl == 1 && !wait_bar(smem_u32(&ctl.o_free), (item_seq & 1) ^ 1, abort_flag)) {
+                            ok = false;
+                            break;
+                        }
+                        if (!issue_pv(c - 1, cl - 1 < 2)) ok = false;
+                    }
                 }
                 if (!ok) break;
-                if (!issue_pv(c_seq + nc - 1, nc == 1)) break;
+                if (nc == 1 && !wait_bar(smem_u32(&ctl.o_free), (item_seq & 1) ^ 1, abort_flag)) break;
+                if (!issue_pv(c_seq + nc - 1, nc - 1 < 2)) break;
                 c_seq += nc;
                 ++item_seq;
             }
             ctl.blocks_done = blocks;
         }
         __syncwarp();
-    } else if (warp >= 3) {
-        // =========================== softmax / correction / epilogue (warps 3..6)
+    } else {
+        // =========================== softmax groups (warps 3..6: w = 0, 7..10: w = 1)
+        // Group w takes the chunks c with c & 1 == w: its own S_w, P_w and
+        // O_w, running maximum m and sum l.  At the end of an item the two
+        // groups exchange (m, l) per row and each writes half of the output
+        // columns: O = (O_0 2^(m_0-M) + O_1 2^(m_1-M)) / (l_0 2^(m_0-M) + l_1 2^(m_1-M)).
+        const int w = (warp - 3) >> 2;
         const int quad = warp & 3;                 // TMEM lanes 32*quad ..
         const int row = quad * 32 + lane;          // query row in the 128-row tile
         const uint32_t trow = tmem + (static_cast<uint32_t>(quad * 32) << 16);
+        const uint32_t sb = trow + static_cast<uint32_t>(w) * 128u;
+        const uint32_t ob = trow + O_COL + static_cast<uint32_t>(w) * 128u;
+        const uint32_t pbase = sP + static_cast<uint32_t>(w) * L::P_BYTES + static_cast<uint32_t>(row) * 128u;
         const float sl2 = a.scale_log2;
         int item_seq = 0;
         uint32_t c_seq = 0;
+        uint32_t n = 0;   // chunks this group has processed
         bool ok = true;
         while (ok) {
             const int slot = item_seq & 1;
@@ -450,41 +480,42 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
             const int nc = (cnt + bpc - 1) / bpc;
             float m_ref = -INFINITY;   // reference maximum, log2 units
             float l = 0.f;
-            for (int cl = 0; cl < nc; ++cl) {
+            bool mine_any = false;
+            for (int cl = (static_cast<int>((c_seq + w) & 1u)); cl < nc; cl += 2) {
+                // chunk c = c_seq + cl has c & 1 == w
                 const uint32_t c = c_seq + cl;
                 const int kst = c % KS;
-                const int b = c & 1;
                 if (!wait_warp(smem_u32(&ctl.k_full[kst]), (c / KS) & 1, abort_flag) ||
-                    !wait_warp(smem_u32(&ctl.s_full[b]), (c >> 1) & 1, abort_flag)) {
+                    !wait_warp(smem_u32(&ctl.s_full[w]), n & 1, abort_flag)) {
                     ok = false;
                     break;
                 }
                 const uint32_t* mrow = ctl.mask[kst];
                 const uint32_t mw0 = mrow[0], mw1 = mrow[1], mw2 = mrow[2], mw3 = mrow[3];
                 const bool partial = (mw0 & mw1 & mw2 & mw3) != 0xFFFFFFFFu;   // chunk holds padding keys
-                const uint32_t sb = trow + b * 128u;
                 tc_fence_after();
                 // pass 1: row maximum of the raw scores, eight independent chains
                 float mx[8];
-                {
-                    uint32_t sr[4][32];
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) tmem_ld32(sb + q * 32u, sr[q]);
+                for (int i = 0; i < 8; ++i) mx[i] = -INFINITY;
+#pragma unroll
+                for (int q2 = 0; q2 < 4; q2 += 2) {
+                    uint32_t sr[2][32];
+                    tmem_ld32(sb + q2 * 32u, sr[0]);
+                    tmem_ld32(sb + q2 * 32u + 32u, sr[1]);
                     tmem_wait_ld();
                     if (partial) {
-                        const uint32_t mwq[4] = {mw0, mw1, mw2, mw3};
+                        const uint32_t mwa = q2 == 0 ? mw0 : mw2, mwb = q2 == 0 ? mw1 : mw3;
 #pragma unroll
-                        for (int q = 0; q < 4; ++q)
-#pragma unroll
-                            for (int i = 0; i < 32; ++i)
-                                if (!((mwq[q] >> i) & 1u)) sr[q][i] = 0xFF800000u;
+                        for (int i = 0; i < 32; ++i) {
+                            if (!((mwa >> i) & 1u)) sr[0][i] = 0xFF800000u;
+                            if (!((mwb >> i) & 1u)) sr[1][i] = 0xFF800000u;
+                        }
                     }
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) mx[i] = -INFINITY;
+                    for (int hq = 0; hq < 2; ++hq)
 #pragma unroll
-                    for (int q = 0; q < 4; ++q)
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) mx[i & 7] = fmaxf(mx[i & 7], __uint_as_float(sr[q][i]));
+                        for (int i = 0; i < 32; ++i) mx[i & 7] = fmaxf(mx[i & 7], __uint_as_float(sr[hq][i]));
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(smem_u32(&ctl.k_empty[kst]));   // mask consumed
@@ -495,19 +526,29 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                 const float alpha = ex2_approx(m_ref - m_new);
                 const float neg = -m_new;
                 m_ref = m_new;
-                // P buffer b was last read by the PV of chunk c-2
-                if (!wait_warp(smem_u32(&ctl.p_free[b]), ((c >> 1) & 1) ^ 1, abort_flag)) {
+                // P_w and O_w were last used by this group's previous PV
+                if (!wait_warp(smem_u32(&ctl.p_free[w]), (n & 1) ^ 1, abort_flag)) {
                     ok = false;
                     break;
                 }
-                // pass 2, 32 columns at a time: P = 2^(s*scale*log2e - m), row sum,
-                // bf16 P row into shared memory (128-byte swizzle, K-major operand)
+                if (mine_any && __any_sync(0xffffffffu, grow)) {
+                    tc_fence_after();
+#pragma unroll 1
+                    for (int q = 0; q < D / 32; ++q) {
+                        uint32_t o[32];
+                        tmem_ld32(ob + q * 32u, o);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+                        tmem_st32(ob + q * 32u, o);
+                    }
+                    tmem_wait_st();
+                }
+                // pass 2: P = 2^(s*scale*log2e - m), row sum, bf16 P row into
+                // P_w (128-byte swizzle, K-major operand); two TMEM loads in flight
                 float sm[8];
 #pragma unroll
                 for (int i = 0; i < 8; ++i) sm[i] = 0.f;
-                const uint32_t prow = sP + b * L::P_BYTES + static_cast<uint32_t>(row) * 128u;
-                // two 32-column groups per step: both TMEM loads are in
-                // flight together
 #pragma unroll 1
                 for (int q2 = 0; q2 < 4; q2 += 2) {
                     uint32_t v[2][32];
@@ -518,7 +559,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                     for (int hq = 0; hq < 2; ++hq) {
                         const int q = q2 + hq;
                         const uint32_t mword = q == 0 ? mw0 : (q == 1 ? mw1 : (q == 2 ? mw2 : mw3));
-                        uint32_t w[16];
+                        uint32_t wv[16];
 #pragma unroll
                         for (int i = 0; i < 32; i += 2) {
                             float p0 = ex2_approx(fmaf(__uint_as_float(v[hq][i]), sl2, neg));
@@ -529,71 +570,88 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                             }
                             sm[i & 7] += p0;
                             sm[(i + 1) & 7] += p1;
-                            w[i >> 1] = pack_bf16x2(p0, p1);
+                            wv[i >> 1] = pack_bf16x2(p0, p1);
                         }
                         const int half = q >> 1;
 #pragma unroll
                         for (int k4 = 0; k4 < 4; ++k4) {
                             const int chunk = (((q & 1) << 2) | k4) ^ (row & 7);
-                            const uint32_t addr = prow + half * 16384u + chunk * 16u;
-                            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(w[4 * k4]),
-                                         "r"(w[4 * k4 + 1]), "r"(w[4 * k4 + 2]), "r"(w[4 * k4 + 3])
+                            const uint32_t addr = pbase + half * 16384u + chunk * 16u;
+                            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(wv[4 * k4]),
+                                         "r"(wv[4 * k4 + 1]), "r"(wv[4 * k4 + 2]), "r"(wv[4 * k4 + 3])
                                          : "memory");
                         }
                     }
                 }
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(smem_u32(&ctl.s_free[b]));   // S buffer consumed
+                if (lane == 0) mbar_arrive(smem_u32(&ctl.s_free[w]));   // S_w consumed
                 const float sum = ((sm[0] + sm[1]) + (sm[2] + sm[3])) + ((sm[4] + sm[5]) + (sm[6] + sm[7]));
                 l = l * alpha + sum;
-                if (cl > 0 && __any_sync(0xffffffffu, grow)) {
-                    // the row maximum moved: O must be rescaled before PV(c)
-                    // adds to it, i.e. after PV(c-1) is done
-                    const uint32_t cp = c - 1;
-                    if (!wait_warp(smem_u32(&ctl.p_free[cp & 1]), (cp >> 1) & 1, abort_flag)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-#pragma unroll 1
-                    for (int q = 0; q < D / 32; ++q) {
-                        uint32_t o[32];
-                        tmem_ld32(trow + O_COL + q * 32u, o);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-                        tmem_st32(trow + O_COL + q * 32u, o);
-                    }
-                    tmem_wait_st();
-                }
                 fence_proxy_async_smem();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(smem_u32(&ctl.p_full));
+                if (lane == 0) mbar_arrive(smem_u32(&ctl.p_full[w]));
+                mine_any = true;
+                ++n;
             }
             if (!ok) break;
-            // epilogue: wait for the last PV, normalise, store bf16
-            const uint32_t c_last = c_seq + nc - 1;
-            if (!wait_warp(smem_u32(&ctl.p_free[c_last & 1]), (c_last >> 1) & 1, abort_flag)) break;
+            // ---- epilogue: wait for this group's last PV, swap (m, l), merge
+            if (mine_any && !wait_warp(smem_u32(&ctl.p_free[w]), (n & 1) ^ 1, abort_flag)) break;
+            if (!wait_warp(smem_u32(&ctl.mrg_empty), (item_seq & 1) ^ 1, abort_flag)) break;
+            ctl.mrg_m[w][row] = m_ref;
+            ctl.mrg_l[w][row] = l;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&ctl.mrg_full));
+            if (!wait_warp(smem_u32(&ctl.mrg_full), item_seq & 1, abort_flag)) break;
+            const float m0 = ctl.mrg_m[0][row], m1 = ctl.mrg_m[1][row];
+            const float l0 = ctl.mrg_l[0][row], l1 = ctl.mrg_l[1][row];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&ctl.mrg_empty));
+            const float mm = fmaxf(m0, m1);
+            // a group with no chunk in this item has l = 0 and m = -inf: weight 0
+            const float a0 = l0 > 0.f ? ex2_approx(m0 - mm) : 0.f;
+            const float a1 = l1 > 0.f ? ex2_approx(m1 - mm) : 0.f;
+            const float inv = 1.0f / (l0 * a0 + l1 * a1);
+            const float f0 = a0 * inv, f1 = a1 * inv;
+            const bool use0 = __any_sync(0xffffffffu, l0 > 0.f), use1 = __any_sync(0xffffffffu, l1 > 0.f);
             tc_fence_after();
-            const float inv_l = 1.0f / l;
             __nv_bfloat16* orow = a.o + ((static_cast<long long>(bh) * g.Npad) + static_cast<long long>(qb) * bs + row) * D;
             const bool store = row < bs;
+            // this group writes output columns [w*D/2, w*D/2 + D/2)
+#pragma unroll 1
+            for (int q = 0; q < D / 64; ++q) {
+                const uint32_t col = static_cast<uint32_t>(w * (D / 2) + q * 32);
+                float r[32];
 #pragma unroll
-            for (int q = 0; q < D / 32; ++q) {
-                uint32_t o[32];
-                tmem_ld32(trow + O_COL + q * 32u, o);
-                tmem_wait_ld();
+                for (int i = 0; i < 32; ++i) r[i] = 0.f;
+                if (use0) {
+                    uint32_t o0[32];
+                    tmem_ld32(trow + O_COL + col, o0);
+                    tmem_wait_ld();
+                    if (l0 > 0.f) {
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) r[i] = __uint_as_float(o0[i]) * f0;
+                    }
+                }
+                if (use1) {
+                    uint32_t o1[32];
+                    tmem_ld32(trow + O_COL + 128u + col, o1);
+                    tmem_wait_ld();
+                    if (l1 > 0.f) {
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) r[i] = fmaf(__uint_as_float(o1[i]), f1, r[i]);
+                    }
+                }
                 if (store) {
 #pragma unroll
-                    for (int v = 0; v < 4; ++v) {
-                        uint4 w;
-                        w.x = pack_bf16x2(__uint_as_float(o[v * 8 + 0]) * inv_l, __uint_as_float(o[v * 8 + 1]) * inv_l);
-                        w.y = pack_bf16x2(__uint_as_float(o[v * 8 + 2]) * inv_l, __uint_as_float(o[v * 8 + 3]) * inv_l);
-                        w.z = pack_bf16x2(__uint_as_float(o[v * 8 + 4]) * inv_l, __uint_as_float(o[v * 8 + 5]) * inv_l);
-                        w.w = pack_bf16x2(__uint_as_float(o[v * 8 + 6]) * inv_l, __uint_as_float(o[v * 8 + 7]) * inv_l);
-                        *reinterpret_cast<uint4*>(orow + q * 32 + v * 8) = w;
+                    for (int v8 = 0; v8 < 4; ++v8) {
+                        uint4 wq;
+                        wq.x = pack_bf16x2(r[v8 * 8 + 0], r[v8 * 8 + 1]);
+                        wq.y = pack_bf16x2(r[v8 * 8 + 2], r[v8 * 8 + 3]);
+                        wq.z = pack_bf16x2(r[v8 * 8 + 4], r[v8 * 8 + 5]);
+                        wq.w = pack_bf16x2(r[v8 * 8 + 6], r[v8 * 8 + 7]);
+                        *reinterpret_cast<uint4*>(orow + col + v8 * 8) = wq;
                     }
                 }
             }
