@@ -376,12 +376,11 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
             uint32_t np0 = 0u, np1 = 0u;   // PVs issued per group
             unsigned long long blocks = 0;
             bool ok = true;
-            // O_w += P_w V for chunk c; `first` starts group w's accumulation
-            auto issue_pv = [&](uint32_t c, bool first) -> bool {
+            // O_w += P_w V for chunk c (its P and V are ready); `first` starts
+            // group w's accumulation
+            auto issue_pv = [&](uint32_t c, bool first) {
                 const int w = c & 1;
                 const int stage = c % V_STAGES;
-                if (!wait_bar(smem_u32(&ctl.p_full[w]), (w ? np1 : np0) & 1, abort_flag)) return false;
-                if (!wait_bar(smem_u32(&ctl.v_full[stage]), (c / V_STAGES) & 1, abort_flag)) return false;
                 tc_fence_after();
                 const uint32_t vb = sV + stage * L::KV_BYTES;
                 const uint32_t pb = sP + w * L::P_BYTES;
@@ -395,8 +394,31 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                 mma_commit(smem_u32(&ctl.v_empty[stage]));
                 mma_commit(smem_u32(&ctl.p_free[w]));
                 if (w) ++np1; else ++np0;
-                return true;
             };
+            // S_w = Q K^T for chunk c (its K and S_w are ready); `last`
+            // releases the Q tile afterwards
+            auto issue_qk = [&](uint32_t c, bool last) {
+                const int stage = c % KS;
+                const int w = c & 1;
+                tc_fence_after();
+                const uint32_t kb = sK + stage * L::KV_BYTES;
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * 16384u + (kk & 3) * 32u;
+                    const uint64_t ad = sw128_desc(sQ + off, 16u, 1024u);
+                    const uint64_t bd = sw128_desc(kb + off, 16u, 1024u);
+                    mma_bf16_ss(tmem + static_cast<uint32_t>(w) * 128u, ad, bd, IDESC_QK, kk > 0 ? 1u : 0u);
+                }
+                mma_commit(smem_u32(&ctl.s_full[w]));
+                mma_commit(smem_u32(&ctl.k_empty[stage]));
+                if (last) mma_commit(smem_u32(&ctl.q_empty));
+                if (w) ++nq1; else ++nq0;
+            };
+            // Within an item the two groups progress independently: the issuer
+            // polls both groups' next QK and next PV and issues whichever has
+            // its inputs ready, so the tensor pipe serves one group while the
+            // other runs its softmax.  Per group, QKs and PVs stay in chunk
+            // order; K and V stages are consumed in stream order per ring.
             while (ok) {
                 const int slot = item_seq & 1;
                 if (!wait_bar(smem_u32(&ctl.item_full[slot]), (item_seq >> 1) & 1, abort_flag)) break;
@@ -407,42 +429,55 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                 const int nc = (cnt + bpc - 1) / bpc;
                 blocks += static_cast<unsigned long long>(cnt);
                 if (!wait_bar(smem_u32(&ctl.q_full), item_seq & 1, abort_flag)) break;
-                tc_fence_after();
-                for (int cl = 0; cl < nc && ok; ++cl) {
-                    const uint32_t c = c_seq + cl;
-                    const int stage = c % KS;
-                    const int w = c & 1;
-                    if (!wait_bar(smem_u32(&ctl.k_full[stage]), (c / KS) & 1, abort_flag) ||
-                        !wait_bar(smem_u32(&ctl.s_free[w]), ((w ? nq1 : nq0) & 1) ^ 1, abort_flag)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    const uint32_t kb = sK + stage * L::KV_BYTES;
+                // next chunk (index within the item) to QK / PV for each group
+                const int first0 = static_cast<int>(c_seq & 1u);   // group 0's first chunk index
+                int qk_i[2] = {first0, first0 ^ 1};
+                int pv_i[2] = {first0, first0 ^ 1};
+                bool o_ok = false;
+                int qks_left = nc;
+                unsigned long long t_stall = 0;
+                while (pv_i[0] < nc || pv_i[1] < nc) {
+                    bool progress = false;
 #pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
-                        const uint32_t off = (kk >> 2) * 16384u + (kk & 3) * 32u;
-                        const uint64_t ad = sw128_desc(sQ + off, 16u, 1024u);
-                        const uint64_t bd = sw128_desc(kb + off, 16u, 1024u);
-                        mma_bf16_ss(tmem + static_cast<uint32_t>(w) * 128u, ad, bd, IDESC_QK, kk > 0 ? 1u : 0u);
+                    for (int w = 0; w < 2; ++w) {
+                        const int iq = w ? qk_i[1] : qk_i[0];
+                        if (iq < nc) {
+                            const uint32_t c = c_seq + iq;
+                            if (mbar_test(smem_u32(&ctl.k_full[c % KS]), (c / KS) & 1) &&
+                                mbar_test(smem_u32(&ctl.s_free[w]), ((w ? nq1 : nq0) & 1) ^ 1)) {
+                                issue_qk(c, --qks_left == 0);
+                                if (w) qk_i[1] += 2; else qk_i[0] += 2;
+                                progress = true;
+                            }
+                        }
+                        const int ip = w ? pv_i[1] : pv_i[0];
+                        if (ip < nc && ip < (w ? qk_i[1] : qk_i[0])) {
+                            const uint32_t c = c_seq + ip;
+                            if (!o_ok) o_ok = mbar_test(smem_u32(&ctl.o_free), (item_seq & 1) ^ 1);
+                            if (o_ok && mbar_test(smem_u32(&ctl.p_full[w]), (w ? np1 : np0) & 1) &&
+                                mbar_test(smem_u32(&ctl.v_full[c % V_STAGES]), (c / V_STAGES) & 1)) {
+                                issue_pv(c, ip < 2);
+                                if (w) pv_i[1] += 2; else pv_i[0] += 2;
+                                progress = true;
+                            }
+                        }
                     }
-                    mma_commit(smem_u32(&ctl.s_full[w]));
-                    mma_commit(smem_u32(&ctl.k_empty[stage]));
-                    if (w) ++nq1; else ++nq0;
-                    if (cl == nc - 1) mma_commit(smem_u32(&ctl.q_empty));
-                    if (cl > 0) {
-                        // the item's first PV waits until the previous item's
-                        // epilogue has read both accumulators
-                        if (cl == 1 && !wait_bar(smem_u32(&ctl.o_free), (item_seq & 1) ^ 1, abort_flag)) {
+                    if (progress) {
+                        t_stall = 0;
+                    } else {
+                        __nanosleep(20);   // leave issue slots to the softmax warps of this SMSP
+                        const unsigned long long now = global_timer_ns();
+                        if (t_stall == 0) {
+                            t_stall = now;
+                        } else if (now - t_stall > WAIT_LIMIT_NS || *abort_flag) {
+                            if (!*abort_flag) record_status(FVATTN_ERR_TIMEOUT);
+                            *abort_flag = 1;
                             ok = false;
                             break;
                         }
-                        if (!issue_pv(c - 1, cl - 1 < 2)) ok = false;
                     }
                 }
                 if (!ok) break;
-                if (nc == 1 && !wait_bar(smem_u32(&ctl.o_free), (item_seq & 1) ^ 1, abort_flag)) break;
-                if (!issue_pv(c_seq + nc - 1, nc - 1 < 2)) break;
                 c_seq += nc;
                 ++item_seq;
             }
