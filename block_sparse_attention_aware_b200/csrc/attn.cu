@@ -13,22 +13,22 @@
 // items dynamically in that order is a longest-processing-time greedy, and
 // keeping concurrent items inside one head keeps that head's K/V in L2.
 //
-// Kernel per CTA (224 threads, one CTA per SM):
+// Kernel per CTA (384 threads, one CTA per SM):
 //   warp 0      K producer: takes items, TMA-loads the Q tile and, per chunk
-//               of 128 keys, the selected K blocks into a 3-stage ring, and
-//               writes the chunk's key-validity mask (padding tokens)
+//               of 128 keys, the selected K blocks into a 2- or 3-stage ring,
+//               and writes the chunk's key-validity mask (padding tokens)
 //   warp 2      V producer: the same chunks' V blocks into a 2-stage ring
-//   warp 1      one lane issues tcgen05.mma: S = Q K^T into one of two TMEM
-//               S buffers, then O += P V into the TMEM O accumulator; a K
-//               stage is released when its S is done, a V stage and a P
-//               buffer when their PV is
-//   warps 3..6  softmax: one query row per thread (TMEM lane), online softmax
-//               in fp32 (exp2 on the MUFU, eight independent max and sum
-//               chains), P rounded to bf16 into one of two shared-memory P
-//               tiles (128-byte-swizzled K-major layout), so the exp pass of
-//               chunk c+1 overlaps the PV of chunk c; O rescaled in TMEM only
-//               when the row maximum grows by more than 2^8, and the
-//               epilogue (O / l -> bf16 -> global)
+//   warp 1      one lane issues S = Q K^T (tcgen05.mma, bf16 -> fp32 TMEM)
+//   warp 3      one lane issues O += P V; two issuing threads keep the tensor
+//               pipe busy while either waits on a barrier
+//   warps 4..11 softmax, two groups of four warps: chunk c goes to group
+//               c & 1, which owns S_(c&1) and O_(c&1) in TMEM and a P tile in
+//               shared memory.  One query row per thread (its TMEM lane);
+//               online softmax in fp32 (exp2 on the MUFU, eight independent
+//               max and sum chains); P rounded to bf16 in the 128-byte-swizzled
+//               K-major layout; O rescaled only when the row maximum grows by
+//               more than 2^8.  At the end of an item the groups swap (m, l)
+//               per row and each writes half of the output columns.
 // Every wait is bounded; a wait that runs out records FVATTN_ERR_TIMEOUT,
 // raises a CTA-wide abort flag and all roles leave their loops, so the CTA
 // always reaches the TMEM release.
@@ -40,7 +40,8 @@
 namespace fv {
 
 constexpr int SOFTMAX_WARPS = 8;        // two groups of four warps
-constexpr int ATT_THREADS = 32 * (3 + SOFTMAX_WARPS);
+constexpr int FIRST_SOFTMAX_WARP = 4;   // warps 0..3: K producer, QK issuer, V producer, PV issuer
+constexpr int ATT_THREADS = 32 * (FIRST_SOFTMAX_WARP + SOFTMAX_WARPS);
 constexpr int MAX_K_STAGES = 3;         // K ring: a stage is free once its S = Q K^T is done
 constexpr int V_STAGES = 2;             // V ring: a stage is free once its O += P V is done
 constexpr uint32_t MAX_DYN_SMEM = 232448;   // sm_100 opt-in shared memory per block
@@ -212,7 +213,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
             mbar_init(smem_u32(&ctl.p_full[w]), 4);
             mbar_init(smem_u32(&ctl.p_free[w]), 1);
             mbar_init(smem_u32(&ctl.item_full[w]), 1);
-            mbar_init(smem_u32(&ctl.item_empty[w]), 2 + SOFTMAX_WARPS);  // MMA, V producer, softmax
+            mbar_init(smem_u32(&ctl.item_empty[w]), 3 + SOFTMAX_WARPS);  // two issuers, V producer, softmax
         }
         mbar_init(smem_u32(&ctl.o_free), SOFTMAX_WARPS);
         mbar_init(smem_u32(&ctl.mrg_full), SOFTMAX_WARPS);
@@ -363,62 +364,22 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
             }
             ++item_seq;
         }
-    } else if (warp == 1) {
-        // =========================== MMA issuer (one lane)
-        // Chunk c of the CTA's stream goes to softmax group w = c & 1: S_w,
-        // P_w and O_w.  n[w] counts the chunks group w has been given.
+    } else if (warp == 1 || warp == 3) {
+        // =========================== tensor-core issuers (one lane each)
+        // Chunk c of the CTA's stream goes to softmax group w = c & 1 (S_w,
+        // P_w, O_w).  Warp 1 issues S_w = Q K^T for every chunk, warp 3
+        // issues O_w += P_w V.  Two issuing threads keep the tensor pipe fed:
+        // while one waits on its barriers (a memory operation by the issuing
+        // thread stalls until its own MMAs drain) the other's MMAs run.
         if (lane == 0) {
+            const bool qk_role = warp == 1;
             constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, 128, false);
             constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, D, true);
             int item_seq = 0;
             uint32_t c_seq = 0;
-            uint32_t nq0 = 0u, nq1 = 0u;   // QKs issued per group
-            uint32_t np0 = 0u, np1 = 0u;   // PVs issued per group
+            uint32_t n0 = 0u, n1 = 0u;   // chunks handled per group
             unsigned long long blocks = 0;
             bool ok = true;
-            // O_w += P_w V for chunk c (its P and V are ready); `first` starts
-            // group w's accumulation
-            auto issue_pv = [&](uint32_t c, bool first) {
-                const int w = c & 1;
-                const int stage = c % V_STAGES;
-                tc_fence_after();
-                const uint32_t vb = sV + stage * L::KV_BYTES;
-                const uint32_t pb = sP + w * L::P_BYTES;
-                const uint32_t od = tmem + O_COL + static_cast<uint32_t>(w) * 128u;
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint64_t ad = sw128_desc(pb + (kk >> 2) * 16384u + (kk & 3) * 32u, 16u, 1024u);
-                    const uint64_t bd = sw128_desc(vb + kk * 2048u, 16384u, 1024u);
-                    mma_bf16_ss(od, ad, bd, IDESC_PV, (first && kk == 0) ? 0u : 1u);
-                }
-                mma_commit(smem_u32(&ctl.v_empty[stage]));
-                mma_commit(smem_u32(&ctl.p_free[w]));
-                if (w) ++np1; else ++np0;
-            };
-            // S_w = Q K^T for chunk c (its K and S_w are ready); `last`
-            // releases the Q tile afterwards
-            auto issue_qk = [&](uint32_t c, bool last) {
-                const int stage = c % KS;
-                const int w = c & 1;
-                tc_fence_after();
-                const uint32_t kb = sK + stage * L::KV_BYTES;
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * 16384u + (kk & 3) * 32u;
-                    const uint64_t ad = sw128_desc(sQ + off, 16u, 1024u);
-                    const uint64_t bd = sw128_desc(kb + off, 16u, 1024u);
-                    mma_bf16_ss(tmem + static_cast<uint32_t>(w) * 128u, ad, bd, IDESC_QK, kk > 0 ? 1u : 0u);
-                }
-                mma_commit(smem_u32(&ctl.s_full[w]));
-                mma_commit(smem_u32(&ctl.k_empty[stage]));
-                if (last) mma_commit(smem_u32(&ctl.q_empty));
-                if (w) ++nq1; else ++nq0;
-            };
-            // Within an item the two groups progress independently: the issuer
-            // polls both groups' next QK and next PV and issues whichever has
-            // its inputs ready, so the tensor pipe serves one group while the
-            // other runs its softmax.  Per group, QKs and PVs stay in chunk
-            // order; K and V stages are consumed in stream order per ring.
             while (ok) {
                 const int slot = item_seq & 1;
                 if (!wait_bar(smem_u32(&ctl.item_full[slot]), (item_seq >> 1) & 1, abort_flag)) break;
@@ -427,70 +388,74 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                 mbar_arrive(smem_u32(&ctl.item_empty[slot]));
                 if (!valid) break;
                 const int nc = (cnt + bpc - 1) / bpc;
-                blocks += static_cast<unsigned long long>(cnt);
-                if (!wait_bar(smem_u32(&ctl.q_full), item_seq & 1, abort_flag)) break;
-                // next chunk (index within the item) to QK / PV for each group
-                const int first0 = static_cast<int>(c_seq & 1u);   // group 0's first chunk index
-                int qk_i[2] = {first0, first0 ^ 1};
-                int pv_i[2] = {first0, first0 ^ 1};
-                bool o_ok = false;
-                int qks_left = nc;
-                unsigned long long t_stall = 0;
-                while (pv_i[0] < nc || pv_i[1] < nc) {
-                    bool progress = false;
-#pragma unroll
-                    for (int w = 0; w < 2; ++w) {
-                        const int iq = w ? qk_i[1] : qk_i[0];
-                        if (iq < nc) {
-                            const uint32_t c = c_seq + iq;
-                            if (mbar_test(smem_u32(&ctl.k_full[c % KS]), (c / KS) & 1) &&
-                                mbar_test(smem_u32(&ctl.s_free[w]), ((w ? nq1 : nq0) & 1) ^ 1)) {
-                                issue_qk(c, --qks_left == 0);
-                                if (w) qk_i[1] += 2; else qk_i[0] += 2;
-                                progress = true;
-                            }
-                        }
-                        const int ip = w ? pv_i[1] : pv_i[0];
-                        if (ip < nc && ip < (w ? qk_i[1] : qk_i[0])) {
-                            const uint32_t c = c_seq + ip;
-                            if (!o_ok) o_ok = mbar_test(smem_u32(&ctl.o_free), (item_seq & 1) ^ 1);
-                            if (o_ok && mbar_test(smem_u32(&ctl.p_full[w]), (w ? np1 : np0) & 1) &&
-                                mbar_test(smem_u32(&ctl.v_full[c % V_STAGES]), (c / V_STAGES) & 1)) {
-                                issue_pv(c, ip < 2);
-                                if (w) pv_i[1] += 2; else pv_i[0] += 2;
-                                progress = true;
-                            }
-                        }
-                    }
-                    if (progress) {
-                        t_stall = 0;
-                    } else {
-                        __nanosleep(20);   // leave issue slots to the softmax warps of this SMSP
-                        const unsigned long long now = global_timer_ns();
-                        if (t_stall == 0) {
-                            t_stall = now;
-                        } else if (now - t_stall > WAIT_LIMIT_NS || *abort_flag) {
-                            if (!*abort_flag) record_status(FVATTN_ERR_TIMEOUT);
-                            *abort_flag = 1;
+                if (qk_role) {
+                    blocks += static_cast<unsigned long long>(cnt);
+                    if (!wait_bar(smem_u32(&ctl.q_full), item_seq & 1, abort_flag)) break;
+                } else {
+                    // the item's first PV waits until the previous item's
+                    // epilogue has read both accumulators
+                    if (!wait_bar(smem_u32(&ctl.o_free), (item_seq & 1) ^ 1, abort_flag)) break;
+                }
+                for (int cl = 0; cl < nc; ++cl) {
+                    const uint32_t c = c_seq + cl;
+                    const int w = c & 1;
+                    const uint32_t n = w ? n1 : n0;
+                    if (qk_role) {
+                        const int stage = c % KS;
+                        if (!wait_bar(smem_u32(&ctl.k_full[stage]), (c / KS) & 1, abort_flag) ||
+                            !wait_bar(smem_u32(&ctl.s_free[w]), (n & 1) ^ 1, abort_flag)) {
                             ok = false;
                             break;
                         }
+                        tc_fence_after();
+                        const uint32_t kb = sK + stage * L::KV_BYTES;
+#pragma unroll
+                        for (int kk = 0; kk < D / 16; ++kk) {
+                            const uint32_t off = (kk >> 2) * 16384u + (kk & 3) * 32u;
+                            const uint64_t ad = sw128_desc(sQ + off, 16u, 1024u);
+                            const uint64_t bd = sw128_desc(kb + off, 16u, 1024u);
+                            mma_bf16_ss(tmem + static_cast<uint32_t>(w) * 128u, ad, bd, IDESC_QK, kk > 0 ? 1u : 0u);
+                        }
+                        mma_commit(smem_u32(&ctl.s_full[w]));
+                        mma_commit(smem_u32(&ctl.k_empty[stage]));
+                        if (cl == nc - 1) mma_commit(smem_u32(&ctl.q_empty));
+                    } else {
+                        const int stage = c % V_STAGES;
+                        if (!wait_bar(smem_u32(&ctl.p_full[w]), n & 1, abort_flag) ||
+                            !wait_bar(smem_u32(&ctl.v_full[stage]), (c / V_STAGES) & 1, abort_flag)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        const uint32_t vb = sV + stage * L::KV_BYTES;
+                        const uint32_t pb = sP + w * L::P_BYTES;
+                        const uint32_t od = tmem + O_COL + static_cast<uint32_t>(w) * 128u;
+                        const bool first = cl < 2;   // group w's first chunk of the item
+#pragma unroll
+                        for (int kk = 0; kk < 8; ++kk) {
+                            const uint64_t ad = sw128_desc(pb + (kk >> 2) * 16384u + (kk & 3) * 32u, 16u, 1024u);
+                            const uint64_t bd = sw128_desc(vb + kk * 2048u, 16384u, 1024u);
+                            mma_bf16_ss(od, ad, bd, IDESC_PV, (first && kk == 0) ? 0u : 1u);
+                        }
+                        mma_commit(smem_u32(&ctl.v_empty[stage]));
+                        mma_commit(smem_u32(&ctl.p_free[w]));
                     }
+                    if (w) ++n1; else ++n0;
                 }
                 if (!ok) break;
                 c_seq += nc;
                 ++item_seq;
             }
-            ctl.blocks_done = blocks;
+            if (qk_role) ctl.blocks_done = blocks;
         }
         __syncwarp();
     } else {
-        // =========================== softmax groups (warps 3..6: w = 0, 7..10: w = 1)
+        // =========================== softmax groups (warps 4..7: w = 0, 8..11: w = 1)
         // Group w takes the chunks c with c & 1 == w: its own S_w, P_w and
         // O_w, running maximum m and sum l.  At the end of an item the two
         // groups exchange (m, l) per row and each writes half of the output
         // columns: O = (O_0 2^(m_0-M) + O_1 2^(m_1-M)) / (l_0 2^(m_0-M) + l_1 2^(m_1-M)).
-        const int w = (warp - 3) >> 2;
+        const int w = (warp - FIRST_SOFTMAX_WARP) >> 2;
         const int quad = warp & 3;                 // TMEM lanes 32*quad ..
         const int row = quad * 32 + lane;          // query row in the 128-row tile
         const uint32_t trow = tmem + (static_cast<uint32_t>(quad * 32) << 16);
