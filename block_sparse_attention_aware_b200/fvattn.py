@@ -22,7 +22,8 @@ _lib = None
 OK, ERR_INVALID, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_BOUNDS = range(6)
 EXPORTED = ("fvattn_geom_init", "fvattn_reorder", "fvattn_inverse_reorder",
             "fvattn_route_workspace_size", "fvattn_route", "fvattn_attn_workspace_size",
-            "fvattn_num_sms", "fvattn_sparse_attn", "fvattn_get_status", "fvattn_status_string")
+            "fvattn_num_sms", "fvattn_sparse_attn", "fvattn_sparse_attn_noalloc", "fvattn_get_status",
+            "fvattn_status_string")
 
 
 class FVAttnError(RuntimeError):
@@ -66,6 +67,8 @@ def load(path: str = LIB_PATH):
     L.fvattn_num_sms.restype = I
     L.fvattn_sparse_attn.argtypes = [G, P, P, P, P, P, ctypes.c_float, P, P, P, S, P]
     L.fvattn_sparse_attn.restype = I
+    L.fvattn_sparse_attn_noalloc.argtypes = [G, P, P, P, P, P, ctypes.c_float, P, P, P]
+    L.fvattn_sparse_attn_noalloc.restype = I
     L.fvattn_get_status.argtypes = [P]
     L.fvattn_get_status.restype = I
     L.fvattn_status_string.argtypes = [I]
@@ -199,6 +202,29 @@ def sparse_attn(g: Geom, qt, kt, vt, kv_idx, kv_cnt, scale: Optional[float] = No
                                    _ptr(kv_cnt), float(scale), _ptr(out), _ptr(sm_stats),
                                    _ptr(workspace), workspace.numel(), _stream(stream))
     _check("fvattn_sparse_attn", rc)
+    return out
+
+
+# Scratch bytes available to sparse_attn_noalloc (FVATTN_NOALLOC_SCRATCH_BYTES).
+NOALLOC_SCRATCH_BYTES = 2 * 1024 * 1024
+
+
+def sparse_attn_noalloc(g: Geom, qt, kt, vt, kv_idx, kv_cnt, scale: Optional[float] = None,
+                        out: Optional[torch.Tensor] = None, sm_stats: Optional[torch.Tensor] = None,
+                        stream=None) -> torch.Tensor:
+    """fvattn_sparse_attn_noalloc: the same attention with the library's own
+    scratch array instead of a caller workspace (for callers that cannot
+    allocate device memory).  Calls that overlap on the GPU share that
+    scratch and must be serialised by the caller."""
+    _need_cuda(qt, kt, vt, kv_idx, kv_cnt, out, sm_stats)
+    if scale is None:
+        scale = 1.0 / math.sqrt(g.D)
+    if out is None:
+        out = tiled_empty(g, qt.device)
+    rc = load().fvattn_sparse_attn_noalloc(ctypes.byref(g), _ptr(qt), _ptr(kt), _ptr(vt), _ptr(kv_idx),
+                                           _ptr(kv_cnt), float(scale), _ptr(out), _ptr(sm_stats),
+                                           _stream(stream))
+    _check("fvattn_sparse_attn_noalloc", rc)
     return out
 
 

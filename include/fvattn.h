@@ -157,6 +157,34 @@ int fvattn_sparse_attn(const fvattn_geom *g, const void *q_t, const void *k_t, c
                        void *o_t, unsigned long long *sm_stats,
                        void *workspace, size_t ws_bytes, fvattn_stream_t stream);
 
+/* Maximum scratch, in bytes, of fvattn_sparse_attn_noalloc (2 MiB): enough
+ * for fvattn_attn_workspace_size(g) of up to about 500 000 work items
+ * (B*H*nb), e.g. a 40-head layer with nb = 12 000 or B = 2 and nb = 6 000. */
+#define FVATTN_NOALLOC_SCRATCH_BYTES (2u * 1024u * 1024u)
+
+/* fvattn_sparse_attn without a workspace argument, for callers that cannot
+ * allocate device memory (a plugin whose host framework owns all device
+ * memory, a C caller with no device allocator, code that must not call
+ * cudaMalloc once running).  The pages have no counterpart: this is a
+ * packaging variant of the same computation and kernels.
+ *   - Scratch: a device array of FVATTN_NOALLOC_SCRATCH_BYTES inside the
+ *     library, held by every GPU that loads it until the process exits.  The
+ *     call allocates nothing (no cudaMalloc, cudaFree or allocating library
+ *     routine).
+ *   - The first call on a device looks the array's device address up with
+ *     cudaGetSymbolAddress (with that device current); make that first call
+ *     before any stream capture.
+ *   - Every call on a device shares the one array and fully rewrites what it
+ *     reads, resetting its item counter to zero.  Calls that overlap on the
+ *     GPU (different streams, or different host threads) race on it and must
+ *     be serialised by the caller.
+ *   - Returns FVATTN_ERR_UNSUPPORTED, before launching anything, when
+ *     fvattn_attn_workspace_size(g) exceeds FVATTN_NOALLOC_SCRATCH_BYTES;
+ *     otherwise the arguments and results are those of fvattn_sparse_attn. */
+int fvattn_sparse_attn_noalloc(const fvattn_geom *g, const void *q_t, const void *k_t, const void *v_t,
+                               const int32_t *kv_idx, const int32_t *kv_cnt, float scale,
+                               void *o_t, unsigned long long *sm_stats, fvattn_stream_t stream);
+
 /* Synchronise `stream`, read and clear the device status word, and return
  * it (FVATTN_OK, FVATTN_ERR_TIMEOUT or FVATTN_ERR_BOUNDS), or
  * FVATTN_ERR_CUDA if the synchronisation itself failed. */
