@@ -4,24 +4,25 @@
 // Top-p keeps the smallest cumulative-importance set, the Top-k safety floor
 // a minimum budget; dynamic masks come from the current attention features).
 //
-// Two kernels:
-//   pool_kernel          HBM-bound.  One CTA per (tensor, b, h, block) sums the
-//                        block's real rows with 16-byte loads (padding rows are
-//                        never read) and writes the fp32 mean.
-//   score_select_kernel  One CTA per (b, h, 32 query blocks).  Scores
-//                        L = scale * Qp Kp^T for its 32 rows against every key
-//                        block into shared memory (fp32 FMA, register-tiled),
-//                        then one warp per row selects the kept set:
-//                          - masses e_j = exp(L_j - max L) as 48-bit fixed
-//                            point, so partial sums are exact integers and do
-//                            not depend on summation order;
-//                          - a most-significant-digit radix select over the
-//                            order key (logit descending, index ascending)
-//                            finds the first prefix whose mass reaches
-//                            p * total (Top-p), and a second, count-based one
-//                            the min(k, nb)-th entry (Top-k floor) when needed;
-//                          - the kept indices are written in ascending order
-//                            with ballots.
+// Three kernels:
+//   pool_kernel    HBM-bound.  One CTA per (tensor, b, h, block) sums the
+//                  block's real rows with 16-byte loads, all issued before the
+//                  first add (padding rows are never read), and writes the fp32
+//                  mean.
+//   score_kernel   L = scale * Qp Kp^T per (b, h): an fp32 register-tiled
+//                  product, 64 x 64 logits per CTA, 4 x 4 per thread, operands
+//                  staged in shared memory k-major.
+//   select_kernel  One warp per (b, h, query block) row, the row's logits in
+//                  registers.  Probability masses e_j = exp(L_j - max L) are
+//                  48-bit fixed point, so every partial sum is an exact integer
+//                  independent of summation order.  The first prefix (logit
+//                  descending, index ascending) whose mass reaches p * total
+//                  (Top-p) and the min(k, nb)-th entry (Top-k floor) are found
+//                  by linear bucketing of the logit range into 256 buckets with
+//                  a mass/count histogram, refined inside the boundary bucket
+//                  until at most 32 candidates remain, which one warp sorts
+//                  (bitonic) and scans.  Equal logits go by ascending index.
+//                  The kept indices are written in ascending order with ballots.
 #include "common.cuh"
 #include "ptx.cuh"
 
@@ -29,133 +30,320 @@ namespace fv {
 
 // ------------------------------------------------------------------ pooling
 
+// One warp per (tensor, b, h, block); 8 warps per CTA.  A lane owns one
+// 16-byte column slice (D/8 slices per row) of every (32 / (D/8))-th row, so
+// one warp instruction reads 512 contiguous bytes; full tiles issue all their
+// loads before the first add.
 template <int D>
-__global__ void __launch_bounds__(256) pool_kernel(Geo g, const __nv_bfloat16* __restrict__ qt,
+__global__ void __launch_bounds__(256, 3) pool_kernel(Geo g, const __nv_bfloat16* __restrict__ qt,
                                                    const __nv_bfloat16* __restrict__ kt,
                                                    float* __restrict__ qp, float* __restrict__ kp) {
-    constexpr int VPR = D / 8;            // 16-byte vectors per row
-    constexpr int RG = 256 / VPR;         // rows handled per pass
-    __shared__ float red[RG][D + 1];
-    const int blk = blockIdx.x;
-    const long long bh = blockIdx.y;
-    const bool is_k = blockIdx.z != 0;
-    const __nv_bfloat16* src = (is_k ? kt : qt) + (bh * g.Npad + static_cast<long long>(blk) * g.bs) * D;
+    constexpr int VPR = D / 8;             // 16-byte vectors per row
+    constexpr int RPI = 32 / VPR;          // rows per warp instruction
+    constexpr int UNR = 8;                 // loads in flight per lane
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const long long unit = static_cast<long long>(blockIdx.x) * 8 + warp;   // (tensor, bh, blk) flattened
+    const long long per_tensor = static_cast<long long>(g.B) * g.H * g.nb;
+    if (unit >= 2 * per_tensor) return;
+    const bool is_k = unit >= per_tensor;
+    const long long ub = is_k ? unit - per_tensor : unit;
+    const long long bh = ub / g.nb;
+    const int blk = static_cast<int>(ub - bh * g.nb);
+    const uint4* src = reinterpret_cast<const uint4*>((is_k ? kt : qt) +
+                                                      (bh * g.Npad + static_cast<long long>(blk) * g.bs) * D);
     float* dst = (is_k ? kp : qp) + (bh * g.nb + blk) * D;
-
-    const int vec = threadIdx.x % VPR;
-    const int rg = threadIdx.x / VPR;
-    // extents of this tile that hold real tokens
+    const int vec = lane % VPR;
+    const int r0 = lane / VPR;
     const int bx = blk % g.nbx, by = (blk / g.nbx) % g.nby, bf = blk / (g.nbx * g.nby);
     const int nf = min(g.tf, g.F - bf * g.tf);
     const int ny = min(g.th, g.Hs - by * g.th);
     const int nx = min(g.tw, g.Ws - bx * g.tw);
-
+    const bool full = nf == g.tf && ny == g.th && nx == g.tw;
     float acc[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-    for (int r = rg; r < g.bs; r += RG) {
-        const int ox = r % g.tw, oy = (r / g.tw) % g.th, of = r / (g.tw * g.th);
-        if (of >= nf || oy >= ny || ox >= nx) continue;
-        uint4 u = __ldg(reinterpret_cast<const uint4*>(src + static_cast<long long>(r) * D) + vec);
-        const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&u);
+    for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+    const int steps = g.bs / RPI;          // warp instructions per tile
+    for (int s0 = 0; s0 < steps; s0 += UNR) {
+        uint4 u[UNR];
+        if (full && s0 + UNR <= steps) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            float2 f = __bfloat1622float2(p2[i]);
-            acc[2 * i] += f.x;
-            acc[2 * i + 1] += f.y;
+            for (int i = 0; i < UNR; ++i) u[i] = __ldg(src + static_cast<long long>(r0 + (s0 + i) * RPI) * VPR + vec);
+        } else {
+#pragma unroll
+            for (int i = 0; i < UNR; ++i) {
+                const int r = r0 + (s0 + i) * RPI;
+                bool take = s0 + i < steps;
+                if (take && !full) {
+                    const int ox = r % g.tw, oy = (r / g.tw) % g.th, of = r / (g.tw * g.th);
+                    take = of < nf && oy < ny && ox < nx;
+                }
+                u[i] = take ? __ldg(src + static_cast<long long>(r) * VPR + vec) : make_uint4(0, 0, 0, 0);
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < UNR; ++i) {
+            const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&u[i]);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 f = __bfloat1622float2(p2[e]);
+                acc[2 * e] += f.x;
+                acc[2 * e + 1] += f.y;
+            }
         }
     }
+    // lanes with the same column slice hold partial sums of different rows
 #pragma unroll
-    for (int i = 0; i < 8; ++i) red[rg][vec * 8 + i] = acc[i];
-    __syncthreads();
-    if (threadIdx.x < D) {
-        float s = 0.f;
-        for (int i = 0; i < RG; ++i) s += red[i][threadIdx.x];
-        dst[threadIdx.x] = s / static_cast<float>(nf * ny * nx);
+    for (int o = VPR; o < 32; o <<= 1)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], o);
+    if (lane < VPR) {
+        const float inv = 1.0f / static_cast<float>(nf * ny * nx);
+        float4* d4 = reinterpret_cast<float4*>(dst + lane * 8);
+        d4[0] = make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
+        d4[1] = make_float4(acc[4] * inv, acc[5] * inv, acc[6] * inv, acc[7] * inv);
     }
 }
 
-// ------------------------------------------------------------------ score + select
+// ------------------------------------------------------------------ scores
 
-constexpr int SS_KCH = 64;       // key blocks per staged chunk
-constexpr int SS_THREADS = 256;
-constexpr int SS_WARPS = SS_THREADS / 32;
+constexpr int SC_TILE = 64;   // logits per CTA side
+constexpr int SC_KC = 32;     // head-dim slice staged per step
 
-// Order key: ascending key = descending logit.  -0 is folded into +0 so that
-// equal logits always get equal keys.
-__device__ __forceinline__ uint32_t desc_key(float v) {
-    uint32_t b = __float_as_uint(v + 0.0f);
-    uint32_t asc = (b & 0x80000000u) ? ~b : (b | 0x80000000u);
-    return ~asc;
+// L[bh][i][j] = scale * <Qp[bh][i], Kp[bh][j]>; grid (tiles_j, tiles_i, B*H).
+__global__ void __launch_bounds__(256) score_kernel(Geo g, const float* __restrict__ qp, const float* __restrict__ kp,
+                                                    float scale, float* __restrict__ L) {
+    __shared__ __align__(16) float As[SC_KC][SC_TILE + 4];
+    __shared__ __align__(16) float Bs[SC_KC][SC_TILE + 4];
+    const int nb = g.nb, D = g.D;
+    const long long bh = blockIdx.z;
+    const int i0 = blockIdx.y * SC_TILE, j0 = blockIdx.x * SC_TILE;
+    const float* A = qp + bh * nb * D;
+    const float* Bm = kp + bh * nb * D;
+    const int tid = threadIdx.x;
+    const int ty = tid / 16, tx = tid % 16;
+    float acc[4][4];
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) acc[a][b] = 0.f;
+    for (int k0 = 0; k0 < D; k0 += SC_KC) {
+        // 64 rows x 32 floats of each operand: 512 float4, two per thread,
+        // stored transposed (k-major)
+#pragma unroll
+        for (int rep = 0; rep < 2; ++rep) {
+            const int idx = tid + rep * 256;
+            const int r = idx / (SC_KC / 4), c4 = idx % (SC_KC / 4);
+            float4 va = make_float4(0.f, 0.f, 0.f, 0.f), vb = va;
+            if (i0 + r < nb) va = __ldg(reinterpret_cast<const float4*>(A + static_cast<long long>(i0 + r) * D + k0) + c4);
+            if (j0 + r < nb) vb = __ldg(reinterpret_cast<const float4*>(Bm + static_cast<long long>(j0 + r) * D + k0) + c4);
+            As[c4 * 4 + 0][r] = va.x; As[c4 * 4 + 1][r] = va.y; As[c4 * 4 + 2][r] = va.z; As[c4 * 4 + 3][r] = va.w;
+            Bs[c4 * 4 + 0][r] = vb.x; Bs[c4 * 4 + 1][r] = vb.y; Bs[c4 * 4 + 2][r] = vb.z; Bs[c4 * 4 + 3][r] = vb.w;
+        }
+        __syncthreads();
+#pragma unroll 8
+        for (int k = 0; k < SC_KC; ++k) {
+            const float4 a = *reinterpret_cast<const float4*>(&As[k][ty * 4]);
+            const float4 b = *reinterpret_cast<const float4*>(&Bs[k][tx * 4]);
+            const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+            for (int x = 0; x < 4; ++x)
+#pragma unroll
+                for (int y = 0; y < 4; ++y) acc[x][y] = fmaf(av[x], bv[y], acc[x][y]);
+        }
+        __syncthreads();
+    }
+#pragma unroll
+    for (int x = 0; x < 4; ++x) {
+        const int i = i0 + ty * 4 + x;
+        if (i >= nb) continue;
+        float* row = L + (bh * nb + i) * nb;
+#pragma unroll
+        for (int y = 0; y < 4; ++y) {
+            const int j = j0 + tx * 4 + y;
+            if (j < nb) row[j] = acc[x][y] * scale;
+        }
+    }
 }
 
+// ------------------------------------------------------------------ selection
+
+constexpr int SEL_WARPS = 8;
+constexpr int SEL_MAX_LEVELS = 4;
+
+// Order key of (logit, index): ascending key = logit descending, then index
+// ascending.  -0 is folded into +0 so that equal logits get equal keys.
+__device__ __forceinline__ unsigned long long order_key(float v, int j) {
+    const uint32_t b = __float_as_uint(v + 0.0f);
+    const uint32_t asc = (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+    return (static_cast<unsigned long long>(~asc) << 32) | static_cast<uint32_t>(j);
+}
+
+// Probability mass exp(l - lmax) in (0, 1] as 48-bit fixed point; with at
+// most 2560 entries every sum stays below 2^60.
 __device__ __forceinline__ unsigned long long fixed_mass(float l, float lmax) {
-    // e in (0, 1]; 2^48 * e <= 2^48, and nb <= 2560 keeps sums below 2^60.
-    float e = __expf(l - lmax);
-    return static_cast<unsigned long long>(e * 281474976710656.0f);
+    return static_cast<unsigned long long>(__expf(l - lmax) * 281474976710656.0f);
 }
 
-struct SelWarpSmem {
+struct SelSmem {
     unsigned int cnt[256];
     unsigned long long mass[256];
+    unsigned long long ckey[32];
+    unsigned long long cmass[32];
 };
 
-// Most-significant-digit radix select over the 32-bit order key.  Finds
-// the key u* of the entry at which the running total (fixed-point mass or
-// count, taken in key order) first reaches `target`, and how many entries
-// with key exactly u* (equal logits, taken by ascending index) are needed.
-// The caller passes the smallest and largest key of the row; bits above the
-// highest bit in which they differ are shared by every entry and are fixed
-// from the start.  If the target is never reached every entry is kept
-// (u* = 0xFFFFFFFF, which no finite logit maps to).
-__device__ __forceinline__ void radix_select(const float* __restrict__ L, int nb, float lmax, bool use_mass,
-                             double target, uint32_t umin, uint32_t umax,
-                             unsigned long long total, SelWarpSmem& sm, uint32_t& u_star,
-                             int& take_ties, int& before_cnt) {
+// Refinement levels of the boundary search: the candidates are the entries
+// whose level-t bucket equals bsel[t] for every level t < n.
+struct Levels {
+    float hi[SEL_MAX_LEVELS];
+    float scl[SEL_MAX_LEVELS];
+    int bsel[SEL_MAX_LEVELS];
+    int n;
+};
+
+// Monotone bucket of a logit inside [lo, hi]: larger logits, lower buckets.
+__device__ __forceinline__ int lin_bucket(float v, float hi, float scl) {
+    const int b = static_cast<int>((hi - v) * scl);
+    return b < 255 ? b : 255;
+}
+
+__device__ __forceinline__ bool in_levels(float v, const Levels& lv) {
+    bool in = true;
+#pragma unroll
+    for (int t = 0; t < SEL_MAX_LEVELS; ++t)
+        if (t < lv.n) in = in && lin_bucket(v, lv.hi[t], lv.scl[t]) == lv.bsel[t];
+    return in;
+}
+
+// Boundary of the weighted prefix: the first entry, in (logit desc, index
+// asc) order, at which the running weight (fixed-point mass, or 1 per entry
+// when use_mass is false) reaches `target`.  Returns its order key; *rank is
+// its 1-based position.  If the target is never reached, returns ~0ull.
+// Slow path, taken only when a boundary bucket holds more than 32 entries:
+// the same search, refined level by level, re-reading the row from memory.
+__device__ __noinline__ unsigned long long find_boundary(const float* __restrict__ Lr, int nb, float lmax, float lmin,
+                                                         bool use_mass, double target, SelSmem& sm, int* rank) {
     const int lane = threadIdx.x & 31;
-    const uint32_t diff = umin ^ umax;
-    int hb = diff ? 31 - __clz(diff) : -1;            // highest undecided bit
-    uint32_t pmask = (hb >= 31) ? 0u : (0xFFFFFFFFu << (hb + 1));
-    uint32_t prefix = umin & pmask;
-    double before = 0.0;
+    Levels lv;
+    lv.n = 0;
+    double before = 0.0;        // weight of all entries ordered before the candidate set
     int before_c = 0;
-    unsigned int bucket_cnt = static_cast<unsigned int>(nb);
-    unsigned long long bucket_w = use_mass ? total : static_cast<unsigned long long>(nb);
-    while (hb >= 0) {
-        const int width = hb + 1 < 8 ? hb + 1 : 8;
-        const int shift = hb + 1 - width;
-        const uint32_t dmask = (1u << width) - 1u;
-        for (int i = lane; i < 256; i += 32) {
-            sm.cnt[i] = 0;
-            sm.mass[i] = 0ull;
+    float hi = lmax, lo = lmin;
+    unsigned int ccount = static_cast<unsigned int>(nb);
+#pragma unroll 1
+    for (int level = 0; level <= SEL_MAX_LEVELS; ++level) {
+        if (hi == lo) {
+            // every candidate carries the same logit: take them by index
+            const unsigned long long each = use_mass ? fixed_mass(hi, lmax) : 1ull;
+            const double need = target - before;
+            long long t = each ? static_cast<long long>(ceil(need / static_cast<double>(each))) : 1;
+            if (t < 1) t = 1;
+            if (t > static_cast<long long>(ccount)) t = ccount;
+            int seen = 0;
+            unsigned long long key = ~0ull;
+            for (int j0 = 0; j0 < nb; j0 += 32) {
+                const int j = j0 + lane;
+                const float x = j < nb ? Lr[j] + 0.0f : 0.f;
+                const bool c = j < nb && x == hi && in_levels(x, lv);
+                const unsigned int bal = __ballot_sync(0xffffffffu, c);
+                const int pos = seen + __popc(bal & ((1u << lane) - 1u));
+                if (c && pos + 1 == t) key = order_key(x, j);
+                seen += __popc(bal);
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) key = min(key, __shfl_xor_sync(0xffffffffu, key, o));
+            *rank = before_c + static_cast<int>(t);
+            return key;
+        }
+        if (ccount <= 32u || level == SEL_MAX_LEVELS) {
+            // at most 32 candidates: gather, sort by order key, scan
+            int seen = 0;
+            for (int j0 = 0; j0 < nb; j0 += 32) {
+                const int j = j0 + lane;
+                const float x = j < nb ? Lr[j] + 0.0f : 0.f;
+                const bool c = j < nb && in_levels(x, lv);
+                const unsigned int bal = __ballot_sync(0xffffffffu, c);
+                if (c) {
+                    const int pos = seen + __popc(bal & ((1u << lane) - 1u));
+                    if (pos < 32) {
+                        sm.ckey[pos] = order_key(x, j);
+                        sm.cmass[pos] = use_mass ? fixed_mass(x, lmax) : 1ull;
+                    }
+                }
+                seen += __popc(bal);
+            }
+            if (seen > 32) return ~0ull;   // cannot happen for finite logits
+            __syncwarp();
+            unsigned long long key = lane < seen ? sm.ckey[lane] : ~0ull;
+            unsigned long long w = lane < seen ? sm.cmass[lane] : 0ull;
+            __syncwarp();
+            // bitonic sort of (key, w) ascending by key across the warp
+#pragma unroll
+            for (int size = 2; size <= 32; size <<= 1) {
+#pragma unroll
+                for (int stride = size >> 1; stride > 0; stride >>= 1) {
+                    const unsigned long long ok = __shfl_xor_sync(0xffffffffu, key, stride);
+                    const unsigned long long ow = __shfl_xor_sync(0xffffffffu, w, stride);
+                    const bool ascending = (lane & size) == 0;
+                    const bool lower = (lane & stride) == 0;
+                    const bool swap = (ascending == lower) ? (ok < key) : (ok > key);
+                    if (swap) {
+                        key = ok;
+                        w = ow;
+                    }
+                }
+            }
+            // inclusive prefix of the weights in sorted order
+            unsigned long long pre = w;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const unsigned long long t = __shfl_up_sync(0xffffffffu, pre, o);
+                if (lane >= o) pre += t;
+            }
+            const bool hit = lane < seen && before + static_cast<double>(pre) >= target;
+            const unsigned int bal = __ballot_sync(0xffffffffu, hit);
+            if (bal == 0u) return ~0ull;
+            const int src = __ffs(bal) - 1;
+            *rank = before_c + src + 1;
+            return __shfl_sync(0xffffffffu, key, src);
+        }
+        // histogram of the candidates over 256 linear buckets of [lo, hi]
+        const float scl = 256.0f / (hi - lo);
+        for (int b = lane; b < 256; b += 32) {
+            sm.cnt[b] = 0u;
+            sm.mass[b] = 0ull;
         }
         __syncwarp();
         for (int j = lane; j < nb; j += 32) {
-            uint32_t u = desc_key(L[j]);
-            if ((u & pmask) != prefix) continue;
-            uint32_t dgt = (u >> shift) & dmask;
-            atomicAdd(&sm.cnt[dgt], 1u);
-            if (use_mass) atomicAdd(&sm.mass[dgt], fixed_mass(L[j], lmax));
+            const float x = Lr[j] + 0.0f;
+            if (in_levels(x, lv)) {
+                const int b = lin_bucket(x, hi, scl);
+                atomicAdd(&sm.cnt[b], 1u);
+                if (use_mass) atomicAdd(&sm.mass[b], fixed_mass(x, lmax));
+            }
         }
         __syncwarp();
-        unsigned long long w[8];
-        unsigned int c[8];
+        // first bucket at which the running weight reaches the target
+        unsigned long long wb[8];
+        unsigned int cb[8];
         unsigned long long wsum = 0;
         unsigned int csum = 0;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            c[i] = sm.cnt[lane * 8 + i];
-            w[i] = use_mass ? sm.mass[lane * 8 + i] : static_cast<unsigned long long>(c[i]);
-            wsum += w[i];
-            csum += c[i];
+        for (int e = 0; e < 8; ++e) {
+            cb[e] = sm.cnt[lane * 8 + e];
+            wb[e] = use_mass ? sm.mass[lane * 8 + e] : static_cast<unsigned long long>(cb[e]);
+            wsum += wb[e];
+            csum += cb[e];
         }
         unsigned long long wex = wsum;
         unsigned int cex = csum;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
-            unsigned long long tw = __shfl_up_sync(0xffffffffu, wex, o);
-            unsigned int tc = __shfl_up_sync(0xffffffffu, cex, o);
-            if (lane >= o) { wex += tw; cex += tc; }
+            const unsigned long long tw = __shfl_up_sync(0xffffffffu, wex, o);
+            const unsigned int tc = __shfl_up_sync(0xffffffffu, cex, o);
+            if (lane >= o) {
+                wex += tw;
+                cex += tc;
+            }
         }
         wex -= wsum;
         cex -= csum;
@@ -165,221 +353,287 @@ __device__ __forceinline__ void radix_select(const float* __restrict__ L, int nb
         double run_at = 0.0;
         int runc_at = 0;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            if (found < 0 && c[i] > 0 && run + static_cast<double>(w[i]) >= target) {
-                found = lane * 8 + i;
+        for (int e = 0; e < 8; ++e) {
+            if (found < 0 && cb[e] > 0u && run + static_cast<double>(wb[e]) >= target) {
+                found = lane * 8 + e;
                 run_at = run;
                 runc_at = runc;
             }
-            run += static_cast<double>(w[i]);
-            runc += static_cast<int>(c[i]);
+            run += static_cast<double>(wb[e]);
+            runc += static_cast<int>(cb[e]);
         }
-        const unsigned int ball = __ballot_sync(0xffffffffu, found >= 0);
-        if (ball == 0u) {
-            u_star = 0xFFFFFFFFu;
-            take_ties = nb;
-            before_cnt = 0;
-            return;
-        }
-        const int src = __ffs(ball) - 1;
-        const int dgt = __shfl_sync(0xffffffffu, found, src);
+        const unsigned int bal = __ballot_sync(0xffffffffu, found >= 0);
+        if (bal == 0u) return ~0ull;
+        const int src = __ffs(bal) - 1;
+        const int bsel = __shfl_sync(0xffffffffu, found, src);
         before = __shfl_sync(0xffffffffu, run_at, src);
         before_c = __shfl_sync(0xffffffffu, runc_at, src);
-        bucket_cnt = sm.cnt[dgt];
-        bucket_w = use_mass ? sm.mass[dgt] : static_cast<unsigned long long>(bucket_cnt);
+        ccount = sm.cnt[bsel];
         __syncwarp();
-        prefix |= static_cast<uint32_t>(dgt) << shift;
-        pmask |= dmask << shift;
-        hb = shift - 1;
-        if (bucket_cnt == 1u && hb >= 0) {
-            // the bucket's single entry fixes the remaining bits
-            uint32_t u_found = 0u;
-            for (int j = lane; j < nb; j += 32) {
-                uint32_t u = desc_key(L[j]);
-                if ((u & pmask) == prefix) u_found = u;
+#pragma unroll
+        for (int t = 0; t < SEL_MAX_LEVELS; ++t)
+            if (t == lv.n) {
+                lv.hi[t] = hi;
+                lv.scl[t] = scl;
+                lv.bsel[t] = bsel;
             }
-            prefix = __reduce_or_sync(0xffffffffu, u_found);
-            hb = -1;
+        ++lv.n;
+        // the candidate range for the next level
+        float nhi = -INFINITY, nlo = INFINITY;
+        for (int j = lane; j < nb; j += 32) {
+            const float x = Lr[j] + 0.0f;
+            if (in_levels(x, lv)) {
+                nhi = fmaxf(nhi, x);
+                nlo = fminf(nlo, x);
+            }
         }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            nhi = fmaxf(nhi, __shfl_xor_sync(0xffffffffu, nhi, o));
+            nlo = fminf(nlo, __shfl_xor_sync(0xffffffffu, nlo, o));
+        }
+        hi = nhi;
+        lo = nlo;
     }
-    if (diff == 0u && !use_mass) bucket_w = static_cast<unsigned long long>(nb);
-    // every entry with key == prefix has the same logit, hence the same weight
-    const unsigned long long each = bucket_w / bucket_cnt;
-    const double need = target - before;
-    long long t = (each > 0ull) ? static_cast<long long>(ceil(need / static_cast<double>(each)))
-                                : static_cast<long long>(bucket_cnt);
-    if (t < 1) t = 1;
-    if (t > static_cast<long long>(bucket_cnt)) t = bucket_cnt;
-    u_star = prefix;
-    take_ties = static_cast<int>(t);
-    before_cnt = before_c;
+    return ~0ull;
 }
 
-// ROWS query blocks per CTA (32, or 16 when a row of logits is long).
-template <int D, int ROWS>
-__global__ void __launch_bounds__(SS_THREADS) score_select_kernel(
-    Geo g, const float* __restrict__ qp, const float* __restrict__ kp, float scale, double p,
-    int kfloor, int32_t* __restrict__ kv_idx, int32_t* __restrict__ kv_cnt,
-    float* __restrict__ logits_out) {
-    extern __shared__ __align__(16) unsigned char ss_smem[];
-    constexpr int DP = D + 4;  // padded row (floats), keeps 16-byte alignment
-    const int nb = g.nb;
-    const long long bh = blockIdx.y;
-    constexpr int RPT = ROWS / 16;  // rows per thread
-    const int row0 = blockIdx.x * ROWS;
-    const int nrows = min(ROWS, nb - row0);
-    float* Ls = reinterpret_cast<float*>(ss_smem);                     // [ROWS][nb]
-    float* Qs = Ls + ROWS * nb;                                          // [ROWS][DP]
-    float* Ks = Qs + ROWS * DP;                                          // [SS_KCH][DP]
-    SelWarpSmem* sel = reinterpret_cast<SelWarpSmem*>(Qs);               // reuses Qs/Ks later
-
-    const int tid = threadIdx.x;
-    // stage the 32 query rows
-    for (int i = tid; i < ROWS * (D / 4); i += SS_THREADS) {
-        int r = i / (D / 4), c4 = i % (D / 4);
-        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (r < nrows) v = __ldg(reinterpret_cast<const float4*>(qp + (bh * nb + row0 + r) * D) + c4);
-        *reinterpret_cast<float4*>(Qs + r * DP + c4 * 4) = v;
-    }
-    const int ty = tid / 16;   // rows RPT*ty .. RPT*ty + RPT-1
-    const int tx = tid % 16;   // keys tx + 16c
-    for (int kc = 0; kc < nb; kc += SS_KCH) {
-        const int nk = min(SS_KCH, nb - kc);
-        __syncthreads();
-        for (int i = tid; i < SS_KCH * (D / 4); i += SS_THREADS) {
-            int r = i / (D / 4), c4 = i % (D / 4);
-            float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (r < nk) v = __ldg(reinterpret_cast<const float4*>(kp + (bh * nb + kc + r) * D) + c4);
-            *reinterpret_cast<float4*>(Ks + r * DP + c4 * 4) = v;
+// Gather the (at most 32) entries flagged by `pick`, sort them by order key
+// and return the first at which before + running weight reaches `target`
+// (key and 1-based rank within the sorted set).  ~0ull if never reached.
+template <int NPL, class Pick>
+__device__ __forceinline__ unsigned long long sort_scan_pick(const float (&v)[NPL], int nb, float lmax, bool use_mass,
+                                                             double before, double target, SelSmem& sm, Pick pick,
+                                                             int* rank) {
+    const int lane = threadIdx.x & 31;
+    int seen = 0;
+#pragma unroll
+    for (int i = 0; i < NPL; ++i) {
+        const int j = lane + 32 * i;
+        const bool c = j < nb && pick(i);
+        const unsigned int bal = __ballot_sync(0xffffffffu, c);
+        if (c) {
+            const int pos = seen + __popc(bal & ((1u << lane) - 1u));
+            sm.ckey[pos] = order_key(v[i], j);
+            sm.cmass[pos] = use_mass ? fixed_mass(v[i], lmax) : 1ull;
         }
-        __syncthreads();
-        float acc[RPT][4];
+        seen += __popc(bal);
+    }
+    __syncwarp();
+    unsigned long long key = lane < seen ? sm.ckey[lane] : ~0ull;
+    unsigned long long w = lane < seen ? sm.cmass[lane] : 0ull;
+    __syncwarp();
 #pragma unroll
-        for (int a = 0; a < RPT; ++a)
+    for (int size = 2; size <= 32; size <<= 1) {
 #pragma unroll
-            for (int b = 0; b < 4; ++b) acc[a][b] = 0.f;
-#pragma unroll 4
-        for (int d = 0; d < D; d += 4) {
-            float4 q[RPT];
+        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+            const unsigned long long ok = __shfl_xor_sync(0xffffffffu, key, stride);
+            const unsigned long long ow = __shfl_xor_sync(0xffffffffu, w, stride);
+            const bool ascending = (lane & size) == 0;
+            const bool lower = (lane & stride) == 0;
+            const bool swap = (ascending == lower) ? (ok < key) : (ok > key);
+            if (swap) {
+                key = ok;
+                w = ow;
+            }
+        }
+    }
+    unsigned long long pre = w;
 #pragma unroll
-            for (int a = 0; a < RPT; ++a)
-                q[a] = *reinterpret_cast<const float4*>(Qs + (RPT * ty + a) * DP + d);
+    for (int o = 1; o < 32; o <<= 1) {
+        const unsigned long long t = __shfl_up_sync(0xffffffffu, pre, o);
+        if (lane >= o) pre += t;
+    }
+    const unsigned int bal = __ballot_sync(0xffffffffu, lane < seen && before + static_cast<double>(pre) >= target);
+    if (bal == 0u) return ~0ull;
+    const int src = __ffs(bal) - 1;
+    *rank = src + 1;
+    return __shfl_sync(0xffffffffu, key, src);
+}
+
+// Shared first level: every entry's bucket among 256 linear buckets of
+// [lmin, lmax] (packed four per word), per-bucket counts and fixed-point
+// masses.  Then for each target (mass reaching p * total; count reaching
+// min(k, nb)) the boundary bucket is resolved directly when it holds at most
+// 32 entries; larger boundary buckets fall back to find_boundary.
+template <int NPL>
+__global__ void __launch_bounds__(32 * SEL_WARPS) select_kernel(int nb, long long rows, const float* __restrict__ L,
+                                                                double p, int kfloor, int32_t* __restrict__ kv_idx,
+                                                                int32_t* __restrict__ kv_cnt) {
+    __shared__ SelSmem sel[SEL_WARPS];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const long long row = static_cast<long long>(blockIdx.x) * SEL_WARPS + warp;
+    if (row >= rows) return;
+    SelSmem& sm = sel[warp];
+    const float* Lr = L + row * nb;
+    float v[NPL];
+    float lmax = -INFINITY, lmin = INFINITY;
 #pragma unroll
-            for (int b = 0; b < 4; ++b) {
-                float4 k4 = *reinterpret_cast<const float4*>(Ks + (tx + 16 * b) * DP + d);
+    for (int i = 0; i < NPL; ++i) {
+        const int j = lane + 32 * i;
+        v[i] = j < nb ? Lr[j] + 0.0f : 0.f;
+        if (j < nb) {
+            lmax = fmaxf(lmax, v[i]);
+            lmin = fminf(lmin, v[i]);
+        }
+    }
 #pragma unroll
-                for (int a = 0; a < RPT; ++a) {
-                    acc[a][b] = fmaf(q[a].x, k4.x, acc[a][b]);
-                    acc[a][b] = fmaf(q[a].y, k4.y, acc[a][b]);
-                    acc[a][b] = fmaf(q[a].z, k4.z, acc[a][b]);
-                    acc[a][b] = fmaf(q[a].w, k4.w, acc[a][b]);
+    for (int o = 16; o > 0; o >>= 1) {
+        lmax = fmaxf(lmax, __shfl_xor_sync(0xffffffffu, lmax, o));
+        lmin = fminf(lmin, __shfl_xor_sync(0xffffffffu, lmin, o));
+    }
+    const int kf = min(kfloor, nb);
+    unsigned long long thr = ~0ull;   // keep every entry whose order key is <= thr
+    if (p < 1.0) {
+        const float scl = lmax > lmin ? 256.0f / (lmax - lmin) : 0.f;
+        for (int b = lane; b < 256; b += 32) {
+            sm.cnt[b] = 0u;
+            sm.mass[b] = 0ull;
+        }
+        __syncwarp();
+        uint32_t bk[(NPL + 3) / 4];
+#pragma unroll
+        for (int q = 0; q < (NPL + 3) / 4; ++q) bk[q] = 0u;
+#pragma unroll
+        for (int i = 0; i < NPL; ++i) {
+            if (lane + 32 * i < nb) {
+                const int b = lin_bucket(v[i], lmax, scl);
+                bk[i >> 2] |= static_cast<uint32_t>(b) << (8 * (i & 3));
+                atomicAdd(&sm.cnt[b], 1u);
+                atomicAdd(&sm.mass[b], fixed_mass(v[i], lmax));
+            }
+        }
+        __syncwarp();
+        // per-lane bucket chunks (8 buckets a lane) and exclusive prefixes
+        unsigned long long wb[8];
+        unsigned int cb[8];
+        unsigned long long wsum = 0;
+        unsigned int csum = 0;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            cb[e] = sm.cnt[lane * 8 + e];
+            wb[e] = sm.mass[lane * 8 + e];
+            wsum += wb[e];
+            csum += cb[e];
+        }
+        unsigned long long wex = wsum, tot = wsum;
+        unsigned int cex = csum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const unsigned long long tw = __shfl_up_sync(0xffffffffu, wex, o);
+            const unsigned int tc = __shfl_up_sync(0xffffffffu, cex, o);
+            if (lane >= o) {
+                wex += tw;
+                cex += tc;
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, o);
+        wex -= wsum;
+        cex -= csum;
+        const double target = p * static_cast<double>(tot);
+        // boundary bucket of the mass target and of the count target
+        int fm = -1, fk = -1;
+        double bm = 0.0;
+        int bcm = 0, bck = 0;
+        {
+            double run = static_cast<double>(wex);
+            unsigned int runc = cex;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                if (fm < 0 && cb[e] > 0u && run + static_cast<double>(wb[e]) >= target) {
+                    fm = lane * 8 + e;
+                    bm = run;
+                    bcm = static_cast<int>(runc);
+                }
+                if (fk < 0 && cb[e] > 0u && static_cast<int>(runc + cb[e]) >= kf) {
+                    fk = lane * 8 + e;
+                    bck = static_cast<int>(runc);
+                }
+                run += static_cast<double>(wb[e]);
+                runc += cb[e];
+            }
+        }
+        const unsigned int balm = __ballot_sync(0xffffffffu, fm >= 0);
+        const unsigned int balk = __ballot_sync(0xffffffffu, fk >= 0);
+        if (balm != 0u) {
+            const int sm_ = __ffs(balm) - 1;
+            const int b_m = __shfl_sync(0xffffffffu, fm, sm_);
+            const double before_m = __shfl_sync(0xffffffffu, bm, sm_);
+            const int before_cm = __shfl_sync(0xffffffffu, bcm, sm_);
+            const unsigned int n_m = sm.cnt[b_m];
+            int rank = 0;
+            unsigned long long kp;
+            if (n_m <= 32u) {
+                kp = sort_scan_pick<NPL>(v, nb, lmax, true, before_m, target, sm,
+                                         [&](int i) { return static_cast<int>((bk[i >> 2] >> (8 * (i & 3))) & 255u) == b_m; },
+                                         &rank);
+                rank += before_cm;
+            } else {
+                kp = find_boundary(Lr, nb, lmax, lmin, true, target, sm, &rank);
+            }
+            if (kp != ~0ull) {
+                thr = kp;
+                if (rank < kf && balk != 0u) {
+                    const int sk = __ffs(balk) - 1;
+                    const int b_k = __shfl_sync(0xffffffffu, fk, sk);
+                    const int before_ck = __shfl_sync(0xffffffffu, bck, sk);
+                    const unsigned int n_k = sm.cnt[b_k];
+                    int rk = 0;
+                    if (n_k <= 32u) {
+                        thr = sort_scan_pick<NPL>(v, nb, lmax, false, static_cast<double>(before_ck), static_cast<double>(kf),
+                                                  sm,
+                                                  [&](int i) { return static_cast<int>((bk[i >> 2] >> (8 * (i & 3))) & 255u) == b_k; },
+                                                  &rk);
+                    } else {
+                        thr = find_boundary(Lr, nb, lmax, lmin, false, static_cast<double>(kf), sm, &rk);
+                    }
                 }
             }
         }
-#pragma unroll
-        for (int a = 0; a < RPT; ++a)
-#pragma unroll
-            for (int b = 0; b < 4; ++b) {
-                int key = tx + 16 * b;
-                if (key < nk) Ls[(RPT * ty + a) * nb + kc + key] = acc[a][b] * scale;
-            }
     }
-    __syncthreads();
-    if (logits_out) {
-        for (int i = tid; i < nrows * nb; i += SS_THREADS) {
-            int r = i / nb, j = i % nb;
-            logits_out[(bh * nb + row0 + r) * nb + j] = Ls[r * nb + j];
-        }
-    }
-    // ---- selection, one warp per row
-    const int warp = tid / 32, lane = tid % 32;
-    SelWarpSmem& sm = sel[warp];
-    const int kf = min(kfloor, nb);
-    for (int r = warp; r < nrows; r += SS_WARPS) {
-        const float* Lr = Ls + r * nb;
-        const long long row = bh * nb + row0 + r;
-        int32_t* out = kv_idx + row * nb;
-        uint32_t u_star = 0xFFFFFFFFu;
-        int take = nb, before = nb;
-        if (p < 1.0 || kf < nb) {
-            float lmax = -INFINITY;
-            uint32_t umin = 0xFFFFFFFFu, umax = 0u;
-            for (int j = lane; j < nb; j += 32) {
-                float v = Lr[j];
-                lmax = fmaxf(lmax, v);
-                uint32_t u = desc_key(v);
-                umin = min(umin, u);
-                umax = max(umax, u);
-            }
+    // emit the kept indices in ascending order
+    int32_t* out = kv_idx + row * nb;
+    int written = 0;
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) lmax = fmaxf(lmax, __shfl_xor_sync(0xffffffffu, lmax, o));
-            umin = __reduce_min_sync(0xffffffffu, umin);
-            umax = __reduce_max_sync(0xffffffffu, umax);
-            int mp = nb;
-            if (p < 1.0) {
-                unsigned long long tot = 0;
-                for (int j = lane; j < nb; j += 32) tot += fixed_mass(Lr[j], lmax);
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, o);
-                const double target = p * static_cast<double>(tot);
-                radix_select(Lr, nb, lmax, true, target, umin, umax, tot, sm, u_star, take, before);
-                mp = (u_star == 0xFFFFFFFFu) ? nb : before + take;
-            }
-            if (mp < kf) {
-                radix_select(Lr, nb, lmax, false, static_cast<double>(kf), umin, umax, 0ull, sm,
-                             u_star, take, before);
-            } else if (p >= 1.0) {
-                u_star = 0xFFFFFFFFu;
-            }
-        }
-        // emit ascending: keep u < u*, or u == u* among the first `take` ties
-        int written = 0, ties_seen = 0;
-        for (int j0 = 0; j0 < nb; j0 += 32) {
-            int j = j0 + lane;
-            bool in = j < nb;
-            uint32_t u = in ? desc_key(Lr[j]) : 0xFFFFFFFFu;
-            bool tie = in && (u == u_star);
-            unsigned int tb = __ballot_sync(0xffffffffu, tie);
-            int tie_rank = ties_seen + __popc(tb & ((1u << lane) - 1u));
-            bool keep = in && ((u < u_star) || (tie && tie_rank < take));
-            if (u_star == 0xFFFFFFFFu && in) keep = true;
-            unsigned int kb = __ballot_sync(0xffffffffu, keep);
-            if (keep) out[written + __popc(kb & ((1u << lane) - 1u))] = j;
-            written += __popc(kb);
-            ties_seen += __popc(tb);
-        }
-        if (lane == 0) kv_cnt[row] = written;
-        __syncwarp();
+    for (int i = 0; i < NPL; ++i) {
+        const int j = lane + 32 * i;
+        const bool keep = j < nb && order_key(v[i], j) <= thr;
+        const unsigned int bal = __ballot_sync(0xffffffffu, keep);
+        if (keep) out[written + __popc(bal & ((1u << lane) - 1u))] = j;
+        written += __popc(bal);
     }
+    if (lane == 0) kv_cnt[row] = written;
 }
 
-static size_t ss_smem_bytes(int nb, int D, int rows) {
-    size_t ls = sizeof(float) * rows * static_cast<size_t>(nb);
-    size_t qk = sizeof(float) * (rows + SS_KCH) * static_cast<size_t>(D + 4);
-    size_t sel = sizeof(SelWarpSmem) * SS_WARPS;
-    return ls + (qk > sel ? qk : sel);
-}
-
-template <int D, int ROWS>
-static int launch_score_select(const Geo& g, const float* qp, const float* kp, float scale,
-                               double p, int kfloor, int32_t* kv_idx, int32_t* kv_cnt,
-                               float* logits, cudaStream_t s) {
-    size_t smem = ss_smem_bytes(g.nb, D, ROWS);
-    if (cudaFuncSetAttribute(score_select_kernel<D, ROWS>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem)) != cudaSuccess)
-        return FVATTN_ERR_CUDA;
-    dim3 grid((g.nb + ROWS - 1) / ROWS, g.B * g.H);
-    score_select_kernel<D, ROWS><<<grid, SS_THREADS, smem, s>>>(g, qp, kp, scale, p, kfloor,
-                                                                kv_idx, kv_cnt, logits);
+template <int NPL>
+static int launch_select(long long rows, int nb, const float* L, double p, int kfloor, int32_t* kv_idx,
+                         int32_t* kv_cnt, cudaStream_t s) {
+    const long long blocks = (rows + SEL_WARPS - 1) / SEL_WARPS;
+    select_kernel<NPL><<<static_cast<unsigned>(blocks), 32 * SEL_WARPS, 0, s>>>(nb, rows, L, p, kfloor, kv_idx,
+                                                                              kv_cnt);
     FV_CHECK_LAUNCH();
     return FVATTN_OK;
 }
 
-// Largest shared-memory footprint the score/select kernel may use.
-constexpr size_t SS_SMEM_LIMIT = 220 * 1024;
-
 static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+struct RouteWs {
+    size_t qp, kp, logits, total;
+};
+
+static size_t al256(size_t x) { return (x + 255) / 256 * 256; }
+
+static RouteWs route_ws(const fvattn_geom& g) {
+    RouteWs w;
+    const size_t BH = static_cast<size_t>(g.B) * g.H;
+    const size_t pooled = al256(sizeof(float) * BH * g.nb * g.D);
+    w.qp = 0;
+    w.kp = pooled;
+    w.logits = 2 * pooled;
+    w.total = w.logits + al256(sizeof(float) * BH * g.nb * g.nb);
+    return w;
+}
 
 }  // namespace fv
 
@@ -387,49 +641,43 @@ using namespace fv;
 
 extern "C" size_t fvattn_route_workspace_size(const fvattn_geom* gp) {
     if (!gp) return 0;
-    size_t pooled = sizeof(float) * static_cast<size_t>(gp->B) * gp->H * gp->nb * gp->D;
-    return 2 * ((pooled + 255) / 256) * 256;
+    return route_ws(*gp).total;
 }
 
-extern "C" int fvattn_route(const fvattn_geom* gp, const void* q_tiled, const void* k_tiled,
-                            double p, int k_floor, float scale, int32_t* kv_idx, int32_t* kv_cnt,
-                            float* q_pool, float* k_pool, float* logits, void* workspace,
-                            size_t ws_bytes, fvattn_stream_t stream) {
+extern "C" int fvattn_route(const fvattn_geom* gp, const void* q_tiled, const void* k_tiled, double p, int k_floor,
+                            float scale, int32_t* kv_idx, int32_t* kv_cnt, float* q_pool, float* k_pool,
+                            float* logits, void* workspace, size_t ws_bytes, fvattn_stream_t stream) {
     if (!gp || !q_tiled || !k_tiled || !kv_idx || !kv_cnt) return FVATTN_ERR_INVALID;
     if (!aligned16(q_tiled) || !aligned16(k_tiled) || !aligned16(kv_idx) || !aligned16(kv_cnt))
         return FVATTN_ERR_INVALID;
     if (!(p > 0.0 && p <= 1.0) || k_floor < 1 || !isfinite(scale)) return FVATTN_ERR_INVALID;
     if (gp->nb <= 0 || gp->nb > 2560) return FVATTN_ERR_UNSUPPORTED;
     if (gp->D != 64 && gp->D != 128) return FVATTN_ERR_UNSUPPORTED;
-    Geo g = to_geo(*gp);
-    size_t pooled = sizeof(float) * static_cast<size_t>(g.B) * g.H * g.nb * g.D;
-    size_t pooled_al = (pooled + 255) / 256 * 256;
-    float* qp = q_pool;
-    float* kp = k_pool;
-    if (!qp || !kp) {
-        if (!workspace || ws_bytes < 2 * pooled_al ||
-            (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
-            return FVATTN_ERR_INVALID;
-        if (!qp) qp = reinterpret_cast<float*>(workspace);
-        if (!kp) kp = reinterpret_cast<float*>(static_cast<char*>(workspace) + pooled_al);
-    }
-    if (!aligned16(qp) || !aligned16(kp)) return FVATTN_ERR_INVALID;
+    const Geo g = to_geo(*gp);
+    const RouteWs wl = route_ws(*gp);
+    char* ws = static_cast<char*>(workspace);
+    const bool need_ws = !q_pool || !k_pool || !logits;
+    if (need_ws && (!workspace || ws_bytes < wl.total || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0))
+        return FVATTN_ERR_INVALID;
+    float* qp = q_pool ? q_pool : reinterpret_cast<float*>(ws + wl.qp);
+    float* kp = k_pool ? k_pool : reinterpret_cast<float*>(ws + wl.kp);
+    float* L = logits ? logits : reinterpret_cast<float*>(ws + wl.logits);
+    if (!aligned16(qp) || !aligned16(kp) || !aligned16(L)) return FVATTN_ERR_INVALID;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    const bool rows32 = ss_smem_bytes(g.nb, g.D, 32) <= SS_SMEM_LIMIT;
-    dim3 pg(g.nb, g.B * g.H, 2);
-    int rc;
-    if (g.D == 128) {
-        pool_kernel<128><<<pg, 256, 0, s>>>(g, static_cast<const __nv_bfloat16*>(q_tiled),
-                                            static_cast<const __nv_bfloat16*>(k_tiled), qp, kp);
-        FV_CHECK_LAUNCH();
-        rc = rows32 ? launch_score_select<128, 32>(g, qp, kp, scale, p, k_floor, kv_idx, kv_cnt, logits, s)
-                    : launch_score_select<128, 16>(g, qp, kp, scale, p, k_floor, kv_idx, kv_cnt, logits, s);
-    } else {
-        pool_kernel<64><<<pg, 256, 0, s>>>(g, static_cast<const __nv_bfloat16*>(q_tiled),
-                                           static_cast<const __nv_bfloat16*>(k_tiled), qp, kp);
-        FV_CHECK_LAUNCH();
-        rc = rows32 ? launch_score_select<64, 32>(g, qp, kp, scale, p, k_floor, kv_idx, kv_cnt, logits, s)
-                    : launch_score_select<64, 16>(g, qp, kp, scale, p, k_floor, kv_idx, kv_cnt, logits, s);
-    }
-    return rc;
+    const long long units = 2ll * g.B * g.H * g.nb;
+    const unsigned pblocks = static_cast<unsigned>((units + 7) / 8);
+    if (g.D == 128)
+        pool_kernel<128><<<pblocks, 256, 0, s>>>(g, static_cast<const __nv_bfloat16*>(q_tiled),
+                                                 static_cast<const __nv_bfloat16*>(k_tiled), qp, kp);
+    else
+        pool_kernel<64><<<pblocks, 256, 0, s>>>(g, static_cast<const __nv_bfloat16*>(q_tiled),
+                                                static_cast<const __nv_bfloat16*>(k_tiled), qp, kp);
+    FV_CHECK_LAUNCH();
+    const int tiles = (g.nb + SC_TILE - 1) / SC_TILE;
+    score_kernel<<<dim3(tiles, tiles, g.B * g.H), 256, 0, s>>>(g, qp, kp, scale, L);
+    FV_CHECK_LAUNCH();
+    const long long rows = static_cast<long long>(g.B) * g.H * g.nb;
+    if (g.nb <= 768) return launch_select<24>(rows, g.nb, L, p, k_floor, kv_idx, kv_cnt, s);
+    if (g.nb <= 1536) return launch_select<48>(rows, g.nb, L, p, k_floor, kv_idx, kv_cnt, s);
+    return launch_select<80>(rows, g.nb, L, p, k_floor, kv_idx, kv_cnt, s);
 }
