@@ -12,17 +12,19 @@
 //   score_kernel   L = scale * Qp Kp^T per (b, h): an fp32 register-tiled
 //                  product, 64 x 64 logits per CTA, 4 x 4 per thread, operands
 //                  staged in shared memory k-major.
-//   select_kernel  One warp per (b, h, query block) row, the row's logits in
-//                  registers.  Probability masses e_j = exp(L_j - max L) are
-//                  48-bit fixed point, so every partial sum is an exact integer
-//                  independent of summation order.  The first prefix (logit
-//                  descending, index ascending) whose mass reaches p * total
-//                  (Top-p) and the min(k, nb)-th entry (Top-k floor) are found
-//                  by linear bucketing of the logit range into 256 buckets with
-//                  a mass/count histogram, refined inside the boundary bucket
-//                  until at most 32 candidates remain, which one warp sorts
-//                  (bitonic) and scans.  Equal logits go by ascending index.
-//                  The kept indices are written in ascending order with ballots.
+//   select_kernel  One warp per (b, h, query block) row, the row's logits and
+//                  their masses e_j = exp(L_j - max L) in registers.  The
+//                  weight of a set {L >= t} is an exact fixed-point integer (a
+//                  lane's float partial sum scaled by 2^40, summed across the
+//                  warp), so it is monotone in t and identical on every lane.
+//                  The Top-p crossing (first prefix, logit descending then
+//                  index ascending, whose mass reaches p * total) is bracketed
+//                  by bisection on t with one warp reduction a step, until at
+//                  most 32 entries remain, which the warp sorts (bitonic on
+//                  64-bit order keys) and scans; the min(k, nb)-th entry (Top-k
+//                  floor) is found the same way with counts when the Top-p
+//                  prefix is shorter.  No shared-memory atomics.  The kept
+//                  indices are written in ascending order with ballots.
 #include "common.cuh"
 #include "ptx.cuh"
 
@@ -168,314 +170,184 @@ __global__ void __launch_bounds__(256) score_kernel(Geo g, const float* __restri
 // ------------------------------------------------------------------ selection
 
 constexpr int SEL_WARPS = 8;
-constexpr int SEL_MAX_LEVELS = 4;
+constexpr int SEL_VALUE_STEPS = 16;   // value-midpoint steps before key-space bisection
+
+// Monotone 32-bit key of a float: a < b  <=>  fkey(a) < fkey(b).  -0 is
+// folded into +0 first, so equal logits get equal keys.
+__device__ __forceinline__ uint32_t fkey(float v) {
+    const uint32_t b = __float_as_uint(v + 0.0f);
+    return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+
+__device__ __forceinline__ float key_to_float(uint32_t k) {
+    return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
 
 // Order key of (logit, index): ascending key = logit descending, then index
-// ascending.  -0 is folded into +0 so that equal logits get equal keys.
+// ascending.
 __device__ __forceinline__ unsigned long long order_key(float v, int j) {
-    const uint32_t b = __float_as_uint(v + 0.0f);
-    const uint32_t asc = (b & 0x80000000u) ? ~b : (b | 0x80000000u);
-    return (static_cast<unsigned long long>(~asc) << 32) | static_cast<uint32_t>(j);
+    return (static_cast<unsigned long long>(~fkey(v)) << 32) | static_cast<uint32_t>(j);
 }
 
-// Probability mass exp(l - lmax) in (0, 1] as 48-bit fixed point; with at
-// most 2560 entries every sum stays below 2^60.
-__device__ __forceinline__ unsigned long long fixed_mass(float l, float lmax) {
-    return static_cast<unsigned long long>(__expf(l - lmax) * 281474976710656.0f);
-}
+// Masses are fixed point with 40 fractional bits: a lane's float partial sum
+// (at most 80 entries of exp(l - lmax) <= 1) converts exactly, and the warp
+// sum of those integers is the same on every lane whatever the order.
+constexpr float SEL_FIX = 1099511627776.0f;   // 2^40
 
-struct SelSmem {
-    unsigned int cnt[256];
-    unsigned long long mass[256];
-    unsigned long long ckey[32];
-    unsigned long long cmass[32];
-};
-
-// Refinement levels of the boundary search: the candidates are the entries
-// whose level-t bucket equals bsel[t] for every level t < n.
-struct Levels {
-    float hi[SEL_MAX_LEVELS];
-    float scl[SEL_MAX_LEVELS];
-    int bsel[SEL_MAX_LEVELS];
-    int n;
-};
-
-// Monotone bucket of a logit inside [lo, hi]: larger logits, lower buckets.
-__device__ __forceinline__ int lin_bucket(float v, float hi, float scl) {
-    const int b = static_cast<int>((hi - v) * scl);
-    return b < 255 ? b : 255;
-}
-
-__device__ __forceinline__ bool in_levels(float v, const Levels& lv) {
-    bool in = true;
+// Sum over the row of [v >= t] * e (fixed point) and of [v >= t].
+template <int NPL, bool KEEP_E>
+__device__ __forceinline__ void sel_eval(const float (&v)[NPL], const float (&e)[NPL], float lmax, float t,
+                                         bool mass, unsigned long long& s, int& c) {
+    float m0 = 0.f, m1 = 0.f;
+    int n = 0;
 #pragma unroll
-    for (int t = 0; t < SEL_MAX_LEVELS; ++t)
-        if (t < lv.n) in = in && lin_bucket(v, lv.hi[t], lv.scl[t]) == lv.bsel[t];
-    return in;
-}
-
-// Boundary of the weighted prefix: the first entry, in (logit desc, index
-// asc) order, at which the running weight (fixed-point mass, or 1 per entry
-// when use_mass is false) reaches `target`.  Returns its order key; *rank is
-// its 1-based position.  If the target is never reached, returns ~0ull.
-// Slow path, taken only when a boundary bucket holds more than 32 entries:
-// the same search, refined level by level, re-reading the row from memory.
-__device__ __noinline__ unsigned long long find_boundary(const float* __restrict__ Lr, int nb, float lmax, float lmin,
-                                                         bool use_mass, double target, SelSmem& sm, int* rank) {
-    const int lane = threadIdx.x & 31;
-    Levels lv;
-    lv.n = 0;
-    double before = 0.0;        // weight of all entries ordered before the candidate set
-    int before_c = 0;
-    float hi = lmax, lo = lmin;
-    unsigned int ccount = static_cast<unsigned int>(nb);
-#pragma unroll 1
-    for (int level = 0; level <= SEL_MAX_LEVELS; ++level) {
-        if (hi == lo) {
-            // every candidate carries the same logit: take them by index
-            const unsigned long long each = use_mass ? fixed_mass(hi, lmax) : 1ull;
-            const double need = target - before;
-            long long t = each ? static_cast<long long>(ceil(need / static_cast<double>(each))) : 1;
-            if (t < 1) t = 1;
-            if (t > static_cast<long long>(ccount)) t = ccount;
-            int seen = 0;
-            unsigned long long key = ~0ull;
-            for (int j0 = 0; j0 < nb; j0 += 32) {
-                const int j = j0 + lane;
-                const float x = j < nb ? Lr[j] + 0.0f : 0.f;
-                const bool c = j < nb && x == hi && in_levels(x, lv);
-                const unsigned int bal = __ballot_sync(0xffffffffu, c);
-                const int pos = seen + __popc(bal & ((1u << lane) - 1u));
-                if (c && pos + 1 == t) key = order_key(x, j);
-                seen += __popc(bal);
+    for (int i = 0; i < NPL; ++i) {
+        const bool in = v[i] >= t;
+        n += in;
+        if (mass) {
+            const float x = KEEP_E ? e[i] : __expf(v[i] - lmax);
+            if (in) {
+                if (i & 1) m1 += x;
+                else m0 += x;
             }
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) key = min(key, __shfl_xor_sync(0xffffffffu, key, o));
-            *rank = before_c + static_cast<int>(t);
-            return key;
         }
-        if (ccount <= 32u || level == SEL_MAX_LEVELS) {
-            // at most 32 candidates: gather, sort by order key, scan
-            int seen = 0;
-            for (int j0 = 0; j0 < nb; j0 += 32) {
-                const int j = j0 + lane;
-                const float x = j < nb ? Lr[j] + 0.0f : 0.f;
-                const bool c = j < nb && in_levels(x, lv);
-                const unsigned int bal = __ballot_sync(0xffffffffu, c);
-                if (c) {
-                    const int pos = seen + __popc(bal & ((1u << lane) - 1u));
-                    if (pos < 32) {
-                        sm.ckey[pos] = order_key(x, j);
-                        sm.cmass[pos] = use_mass ? fixed_mass(x, lmax) : 1ull;
-                    }
-                }
-                seen += __popc(bal);
-            }
-            if (seen > 32) return ~0ull;   // cannot happen for finite logits
-            __syncwarp();
-            unsigned long long key = lane < seen ? sm.ckey[lane] : ~0ull;
-            unsigned long long w = lane < seen ? sm.cmass[lane] : 0ull;
-            __syncwarp();
-            // bitonic sort of (key, w) ascending by key across the warp
+    }
+    c = __reduce_add_sync(0xffffffffu, static_cast<unsigned int>(n));
+    if (mass) {
+        unsigned long long f = static_cast<unsigned long long>((m0 + m1) * SEL_FIX);
 #pragma unroll
-            for (int size = 2; size <= 32; size <<= 1) {
+        for (int o = 16; o > 0; o >>= 1) f += __shfl_xor_sync(0xffffffffu, f, o);
+        s = f;
+    } else {
+        s = static_cast<unsigned long long>(c);
+    }
+}
+
+// Boundary of a weighted prefix in (logit desc, index asc) order: the first
+// entry at which the running weight reaches `target`, where the weight of the
+// set {v >= t} is sel_eval's sum (mass) or count.  Precondition:
+// weight({v >= lmin}) >= target > 0, c_all = #{v >= lmin}.  The bracket [lo, hi) in key
+// space always holds the crossing (weight at lo >= target > weight at hi); it
+// is halved at the value midpoint for the first steps, then at the key
+// midpoint, until at most 32 entries remain (sorted and scanned by one warp)
+// or a single logit value remains (ties resolved by ascending index).
+// Returns the crossing's order key and its 1-based rank.
+template <int NPL, bool KEEP_E>
+__device__ unsigned long long sel_boundary(const float (&v)[NPL], const float (&e)[NPL], int nb, float lmax, float lmin,
+                                           bool mass, int c_all, double target,
+                                           unsigned long long* ck, int* rank) {
+    const int lane = threadIdx.x & 31;
+    uint32_t lo_k = fkey(lmin), hi_k = fkey(lmax) + 1u;
+    unsigned long long s_hi = 0ull;
+    int c_lo = c_all, c_hi = 0;
+    (void)nb;
+#pragma unroll 1
+    for (int it = 0; c_lo - c_hi > 32 && hi_k - lo_k > 1u; ++it) {
+        uint32_t mk;
+        if (it < SEL_VALUE_STEPS) {
+            const float a = key_to_float(lo_k), b = key_to_float(hi_k - 1u);
+            mk = fkey(0.5f * a + 0.5f * b);
+        } else {
+            mk = lo_k + (hi_k - lo_k) / 2u;
+        }
+        mk = min(max(mk, lo_k + 1u), hi_k - 1u);
+        unsigned long long s;
+        int c;
+        sel_eval<NPL, KEEP_E>(v, e, lmax, key_to_float(mk), mass, s, c);
+        if (static_cast<double>(s) >= target) {
+            lo_k = mk;
+            c_lo = c;
+        } else {
+            hi_k = mk;
+            s_hi = s;
+            c_hi = c;
+        }
+    }
+    const float tlo = key_to_float(lo_k), thi = key_to_float(hi_k);
+    const int cand = c_lo - c_hi;
+    if (cand <= 32) {
+        // gather the candidates, sort by order key, scan their weights
+        int seen = 0;
 #pragma unroll
-                for (int stride = size >> 1; stride > 0; stride >>= 1) {
-                    const unsigned long long ok = __shfl_xor_sync(0xffffffffu, key, stride);
-                    const unsigned long long ow = __shfl_xor_sync(0xffffffffu, w, stride);
-                    const bool ascending = (lane & size) == 0;
-                    const bool lower = (lane & stride) == 0;
-                    const bool swap = (ascending == lower) ? (ok < key) : (ok > key);
-                    if (swap) {
-                        key = ok;
-                        w = ow;
-                    }
-                }
+        for (int i = 0; i < NPL; ++i) {
+            const bool in = v[i] >= tlo && v[i] < thi;
+            const unsigned int bal = __ballot_sync(0xffffffffu, in);
+            if (in) ck[seen + __popc(bal & ((1u << lane) - 1u))] = order_key(v[i], lane + 32 * i);
+            seen += __popc(bal);
+        }
+        __syncwarp();
+        unsigned long long key = lane < cand ? ck[lane] : ~0ull;
+        __syncwarp();
+#pragma unroll
+        for (int size = 2; size <= 32; size <<= 1) {
+#pragma unroll
+            for (int stride = size >> 1; stride > 0; stride >>= 1) {
+                const unsigned long long ok = __shfl_xor_sync(0xffffffffu, key, stride);
+                const bool up = ((lane & size) == 0) == ((lane & stride) == 0);
+                if (up ? (ok < key) : (ok > key)) key = ok;
             }
-            // inclusive prefix of the weights in sorted order
-            unsigned long long pre = w;
+        }
+        int pick;
+        if (mass) {
+            const float x = key_to_float(~static_cast<uint32_t>(key >> 32));
+            unsigned long long pre = lane < cand ? static_cast<unsigned long long>(__expf(x - lmax) * SEL_FIX) : 0ull;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
                 const unsigned long long t = __shfl_up_sync(0xffffffffu, pre, o);
                 if (lane >= o) pre += t;
             }
-            const bool hit = lane < seen && before + static_cast<double>(pre) >= target;
-            const unsigned int bal = __ballot_sync(0xffffffffu, hit);
-            if (bal == 0u) return ~0ull;
-            const int src = __ffs(bal) - 1;
-            *rank = before_c + src + 1;
-            return __shfl_sync(0xffffffffu, key, src);
+            const unsigned int bal =
+                __ballot_sync(0xffffffffu, lane < cand && static_cast<double>(s_hi + pre) >= target);
+            pick = bal ? __ffs(bal) - 1 : cand - 1;   // rounding: all candidates
+        } else {
+            pick = static_cast<int>(target) - c_hi - 1;
         }
-        // histogram of the candidates over 256 linear buckets of [lo, hi]
-        const float scl = 256.0f / (hi - lo);
-        for (int b = lane; b < 256; b += 32) {
-            sm.cnt[b] = 0u;
-            sm.mass[b] = 0ull;
-        }
-        __syncwarp();
-        for (int j = lane; j < nb; j += 32) {
-            const float x = Lr[j] + 0.0f;
-            if (in_levels(x, lv)) {
-                const int b = lin_bucket(x, hi, scl);
-                atomicAdd(&sm.cnt[b], 1u);
-                if (use_mass) atomicAdd(&sm.mass[b], fixed_mass(x, lmax));
-            }
-        }
-        __syncwarp();
-        // first bucket at which the running weight reaches the target
-        unsigned long long wb[8];
-        unsigned int cb[8];
-        unsigned long long wsum = 0;
-        unsigned int csum = 0;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            cb[e] = sm.cnt[lane * 8 + e];
-            wb[e] = use_mass ? sm.mass[lane * 8 + e] : static_cast<unsigned long long>(cb[e]);
-            wsum += wb[e];
-            csum += cb[e];
-        }
-        unsigned long long wex = wsum;
-        unsigned int cex = csum;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const unsigned long long tw = __shfl_up_sync(0xffffffffu, wex, o);
-            const unsigned int tc = __shfl_up_sync(0xffffffffu, cex, o);
-            if (lane >= o) {
-                wex += tw;
-                cex += tc;
-            }
-        }
-        wex -= wsum;
-        cex -= csum;
-        int found = -1;
-        double run = before + static_cast<double>(wex);
-        int runc = before_c + static_cast<int>(cex);
-        double run_at = 0.0;
-        int runc_at = 0;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            if (found < 0 && cb[e] > 0u && run + static_cast<double>(wb[e]) >= target) {
-                found = lane * 8 + e;
-                run_at = run;
-                runc_at = runc;
-            }
-            run += static_cast<double>(wb[e]);
-            runc += static_cast<int>(cb[e]);
-        }
-        const unsigned int bal = __ballot_sync(0xffffffffu, found >= 0);
-        if (bal == 0u) return ~0ull;
-        const int src = __ffs(bal) - 1;
-        const int bsel = __shfl_sync(0xffffffffu, found, src);
-        before = __shfl_sync(0xffffffffu, run_at, src);
-        before_c = __shfl_sync(0xffffffffu, runc_at, src);
-        ccount = sm.cnt[bsel];
-        __syncwarp();
-#pragma unroll
-        for (int t = 0; t < SEL_MAX_LEVELS; ++t)
-            if (t == lv.n) {
-                lv.hi[t] = hi;
-                lv.scl[t] = scl;
-                lv.bsel[t] = bsel;
-            }
-        ++lv.n;
-        // the candidate range for the next level
-        float nhi = -INFINITY, nlo = INFINITY;
-        for (int j = lane; j < nb; j += 32) {
-            const float x = Lr[j] + 0.0f;
-            if (in_levels(x, lv)) {
-                nhi = fmaxf(nhi, x);
-                nlo = fminf(nlo, x);
-            }
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            nhi = fmaxf(nhi, __shfl_xor_sync(0xffffffffu, nhi, o));
-            nlo = fminf(nlo, __shfl_xor_sync(0xffffffffu, nlo, o));
-        }
-        hi = nhi;
-        lo = nlo;
+        pick = min(max(pick, 0), cand - 1);
+        *rank = c_hi + pick + 1;
+        return __shfl_sync(0xffffffffu, key, pick);
     }
-    return ~0ull;
-}
-
-// Gather the (at most 32) entries flagged by `pick`, sort them by order key
-// and return the first at which before + running weight reaches `target`
-// (key and 1-based rank within the sorted set).  ~0ull if never reached.
-template <int NPL, class Pick>
-__device__ __forceinline__ unsigned long long sort_scan_pick(const float (&v)[NPL], int nb, float lmax, bool use_mass,
-                                                             double before, double target, SelSmem& sm, Pick pick,
-                                                             int* rank) {
-    const int lane = threadIdx.x & 31;
-    int seen = 0;
+    // a single logit value remains: take the candidates by ascending index
+    long long need;
+    if (mass) {
+        const double w = static_cast<double>(static_cast<unsigned long long>(__expf(tlo - lmax) * SEL_FIX));
+        need = w > 0.0 ? static_cast<long long>(ceil((target - static_cast<double>(s_hi)) / w)) : cand;
+    } else {
+        need = static_cast<long long>(target) - c_hi;
+    }
+    need = min(max(need, 1ll), static_cast<long long>(cand));
+    int seen = 0, found = 0;
 #pragma unroll
     for (int i = 0; i < NPL; ++i) {
-        const int j = lane + 32 * i;
-        const bool c = j < nb && pick(i);
-        const unsigned int bal = __ballot_sync(0xffffffffu, c);
-        if (c) {
-            const int pos = seen + __popc(bal & ((1u << lane) - 1u));
-            sm.ckey[pos] = order_key(v[i], j);
-            sm.cmass[pos] = use_mass ? fixed_mass(v[i], lmax) : 1ull;
-        }
+        const bool in = v[i] == tlo;
+        const unsigned int bal = __ballot_sync(0xffffffffu, in);
+        if (in && seen + __popc(bal & ((1u << lane) - 1u)) + 1 == need) found = lane + 32 * i + 1;
         seen += __popc(bal);
     }
-    __syncwarp();
-    unsigned long long key = lane < seen ? sm.ckey[lane] : ~0ull;
-    unsigned long long w = lane < seen ? sm.cmass[lane] : 0ull;
-    __syncwarp();
-#pragma unroll
-    for (int size = 2; size <= 32; size <<= 1) {
-#pragma unroll
-        for (int stride = size >> 1; stride > 0; stride >>= 1) {
-            const unsigned long long ok = __shfl_xor_sync(0xffffffffu, key, stride);
-            const unsigned long long ow = __shfl_xor_sync(0xffffffffu, w, stride);
-            const bool ascending = (lane & size) == 0;
-            const bool lower = (lane & stride) == 0;
-            const bool swap = (ascending == lower) ? (ok < key) : (ok > key);
-            if (swap) {
-                key = ok;
-                w = ow;
-            }
-        }
-    }
-    unsigned long long pre = w;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const unsigned long long t = __shfl_up_sync(0xffffffffu, pre, o);
-        if (lane >= o) pre += t;
-    }
-    const unsigned int bal = __ballot_sync(0xffffffffu, lane < seen && before + static_cast<double>(pre) >= target);
-    if (bal == 0u) return ~0ull;
-    const int src = __ffs(bal) - 1;
-    *rank = src + 1;
-    return __shfl_sync(0xffffffffu, key, src);
+    found = __reduce_max_sync(0xffffffffu, static_cast<unsigned int>(found));
+    *rank = c_hi + static_cast<int>(need);
+    return order_key(tlo, found - 1);
 }
 
-// Shared first level: every entry's bucket among 256 linear buckets of
-// [lmin, lmax] (packed four per word), per-bucket counts and fixed-point
-// masses.  Then for each target (mass reaching p * total; count reaching
-// min(k, nb)) the boundary bucket is resolved directly when it holds at most
-// 32 entries; larger boundary buckets fall back to find_boundary.
-template <int NPL>
-__global__ void __launch_bounds__(32 * SEL_WARPS) select_kernel(int nb, long long rows, const float* __restrict__ L,
+// One warp per (b, h, query block) row.  Kept set: every entry whose order key
+// is at most that of the later of the Top-p crossing (first prefix whose mass
+// reaches p * total) and the min(k, nb)-th entry.
+template <int NPL, bool KEEP_E>
+__global__ void __launch_bounds__(32 * SEL_WARPS, NPL <= 24 ? 3 : 1) select_kernel(int nb, long long rows, const float* __restrict__ L,
                                                                 double p, int kfloor, int32_t* __restrict__ kv_idx,
                                                                 int32_t* __restrict__ kv_cnt) {
-    __shared__ SelSmem sel[SEL_WARPS];
+    __shared__ unsigned long long cand_keys[SEL_WARPS][32];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const long long row = static_cast<long long>(blockIdx.x) * SEL_WARPS + warp;
     if (row >= rows) return;
-    SelSmem& sm = sel[warp];
     const float* Lr = L + row * nb;
     float v[NPL];
     float lmax = -INFINITY, lmin = INFINITY;
 #pragma unroll
     for (int i = 0; i < NPL; ++i) {
         const int j = lane + 32 * i;
-        v[i] = j < nb ? Lr[j] + 0.0f : 0.f;
-        if (j < nb) {
-            lmax = fmaxf(lmax, v[i]);
-            lmin = fminf(lmin, v[i]);
-        }
+        v[i] = j < nb ? Lr[j] + 0.0f : -INFINITY;
+        lmax = fmaxf(lmax, v[i]);
+        if (j < nb) lmin = fminf(lmin, v[i]);
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
@@ -483,122 +355,33 @@ __global__ void __launch_bounds__(32 * SEL_WARPS) select_kernel(int nb, long lon
         lmin = fminf(lmin, __shfl_xor_sync(0xffffffffu, lmin, o));
     }
     const int kf = min(kfloor, nb);
-    unsigned long long thr = ~0ull;   // keep every entry whose order key is <= thr
+    unsigned long long thr = ~0ull;
     if (p < 1.0) {
-        const float scl = lmax > lmin ? 256.0f / (lmax - lmin) : 0.f;
-        for (int b = lane; b < 256; b += 32) {
-            sm.cnt[b] = 0u;
-            sm.mass[b] = 0ull;
-        }
-        __syncwarp();
-        uint32_t bk[(NPL + 3) / 4];
+        float e[NPL];
+        if (KEEP_E) {
 #pragma unroll
-        for (int q = 0; q < (NPL + 3) / 4; ++q) bk[q] = 0u;
-#pragma unroll
-        for (int i = 0; i < NPL; ++i) {
-            if (lane + 32 * i < nb) {
-                const int b = lin_bucket(v[i], lmax, scl);
-                bk[i >> 2] |= static_cast<uint32_t>(b) << (8 * (i & 3));
-                atomicAdd(&sm.cnt[b], 1u);
-                atomicAdd(&sm.mass[b], fixed_mass(v[i], lmax));
-            }
+            for (int i = 0; i < NPL; ++i) e[i] = __expf(v[i] - lmax);
         }
-        __syncwarp();
-        // per-lane bucket chunks (8 buckets a lane) and exclusive prefixes
-        unsigned long long wb[8];
-        unsigned int cb[8];
-        unsigned long long wsum = 0;
-        unsigned int csum = 0;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            cb[e] = sm.cnt[lane * 8 + e];
-            wb[e] = sm.mass[lane * 8 + e];
-            wsum += wb[e];
-            csum += cb[e];
-        }
-        unsigned long long wex = wsum, tot = wsum;
-        unsigned int cex = csum;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const unsigned long long tw = __shfl_up_sync(0xffffffffu, wex, o);
-            const unsigned int tc = __shfl_up_sync(0xffffffffu, cex, o);
-            if (lane >= o) {
-                wex += tw;
-                cex += tc;
-            }
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, o);
-        wex -= wsum;
-        cex -= csum;
-        const double target = p * static_cast<double>(tot);
-        // boundary bucket of the mass target and of the count target
-        int fm = -1, fk = -1;
-        double bm = 0.0;
-        int bcm = 0, bck = 0;
-        {
-            double run = static_cast<double>(wex);
-            unsigned int runc = cex;
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                if (fm < 0 && cb[e] > 0u && run + static_cast<double>(wb[e]) >= target) {
-                    fm = lane * 8 + e;
-                    bm = run;
-                    bcm = static_cast<int>(runc);
-                }
-                if (fk < 0 && cb[e] > 0u && static_cast<int>(runc + cb[e]) >= kf) {
-                    fk = lane * 8 + e;
-                    bck = static_cast<int>(runc);
-                }
-                run += static_cast<double>(wb[e]);
-                runc += cb[e];
-            }
-        }
-        const unsigned int balm = __ballot_sync(0xffffffffu, fm >= 0);
-        const unsigned int balk = __ballot_sync(0xffffffffu, fk >= 0);
-        if (balm != 0u) {
-            const int sm_ = __ffs(balm) - 1;
-            const int b_m = __shfl_sync(0xffffffffu, fm, sm_);
-            const double before_m = __shfl_sync(0xffffffffu, bm, sm_);
-            const int before_cm = __shfl_sync(0xffffffffu, bcm, sm_);
-            const unsigned int n_m = sm.cnt[b_m];
-            int rank = 0;
-            unsigned long long kp;
-            if (n_m <= 32u) {
-                kp = sort_scan_pick<NPL>(v, nb, lmax, true, before_m, target, sm,
-                                         [&](int i) { return static_cast<int>((bk[i >> 2] >> (8 * (i & 3))) & 255u) == b_m; },
-                                         &rank);
-                rank += before_cm;
-            } else {
-                kp = find_boundary(Lr, nb, lmax, lmin, true, target, sm, &rank);
-            }
-            if (kp != ~0ull) {
-                thr = kp;
-                if (rank < kf && balk != 0u) {
-                    const int sk = __ffs(balk) - 1;
-                    const int b_k = __shfl_sync(0xffffffffu, fk, sk);
-                    const int before_ck = __shfl_sync(0xffffffffu, bck, sk);
-                    const unsigned int n_k = sm.cnt[b_k];
-                    int rk = 0;
-                    if (n_k <= 32u) {
-                        thr = sort_scan_pick<NPL>(v, nb, lmax, false, static_cast<double>(before_ck), static_cast<double>(kf),
-                                                  sm,
-                                                  [&](int i) { return static_cast<int>((bk[i >> 2] >> (8 * (i & 3))) & 255u) == b_k; },
-                                                  &rk);
-                    } else {
-                        thr = find_boundary(Lr, nb, lmax, lmin, false, static_cast<double>(kf), sm, &rk);
-                    }
-                }
-            }
-        }
+        unsigned long long s_all;
+        int c_all;
+        sel_eval<NPL, KEEP_E>(v, e, lmax, lmin, true, s_all, c_all);
+        const double target = p * static_cast<double>(s_all);
+        int rank = 0;
+        thr = sel_boundary<NPL, KEEP_E>(v, e, nb, lmax, lmin, true, c_all, target, cand_keys[warp], &rank);
+        if (rank < kf)
+            thr = sel_boundary<NPL, KEEP_E>(v, e, nb, lmax, lmin, false, c_all, static_cast<double>(kf),
+                                            cand_keys[warp], &rank);
     }
     // emit the kept indices in ascending order
+    const float tv = key_to_float(~static_cast<uint32_t>(thr >> 32));
+    const int tj = static_cast<int>(thr & 0xffffffffu);
+    const bool all = thr == ~0ull;
     int32_t* out = kv_idx + row * nb;
     int written = 0;
 #pragma unroll
     for (int i = 0; i < NPL; ++i) {
         const int j = lane + 32 * i;
-        const bool keep = j < nb && order_key(v[i], j) <= thr;
+        const bool keep = j < nb && (all || v[i] > tv || (v[i] == tv && j <= tj));
         const unsigned int bal = __ballot_sync(0xffffffffu, keep);
         if (keep) out[written + __popc(bal & ((1u << lane) - 1u))] = j;
         written += __popc(bal);
@@ -606,12 +389,12 @@ __global__ void __launch_bounds__(32 * SEL_WARPS) select_kernel(int nb, long lon
     if (lane == 0) kv_cnt[row] = written;
 }
 
-template <int NPL>
+template <int NPL, bool KEEP_E>
 static int launch_select(long long rows, int nb, const float* L, double p, int kfloor, int32_t* kv_idx,
                          int32_t* kv_cnt, cudaStream_t s) {
     const long long blocks = (rows + SEL_WARPS - 1) / SEL_WARPS;
-    select_kernel<NPL><<<static_cast<unsigned>(blocks), 32 * SEL_WARPS, 0, s>>>(nb, rows, L, p, kfloor, kv_idx,
-                                                                              kv_cnt);
+    select_kernel<NPL, KEEP_E><<<static_cast<unsigned>(blocks), 32 * SEL_WARPS, 0, s>>>(nb, rows, L, p, kfloor,
+                                                                                      kv_idx, kv_cnt);
     FV_CHECK_LAUNCH();
     return FVATTN_OK;
 }
@@ -677,7 +460,7 @@ extern "C" int fvattn_route(const fvattn_geom* gp, const void* q_tiled, const vo
     score_kernel<<<dim3(tiles, tiles, g.B * g.H), 256, 0, s>>>(g, qp, kp, scale, L);
     FV_CHECK_LAUNCH();
     const long long rows = static_cast<long long>(g.B) * g.H * g.nb;
-    if (g.nb <= 768) return launch_select<24>(rows, g.nb, L, p, k_floor, kv_idx, kv_cnt, s);
-    if (g.nb <= 1536) return launch_select<48>(rows, g.nb, L, p, k_floor, kv_idx, kv_cnt, s);
-    return launch_select<80>(rows, g.nb, L, p, k_floor, kv_idx, kv_cnt, s);
+    if (g.nb <= 768) return launch_select<24, true>(rows, g.nb, L, p, k_floor, kv_idx, kv_cnt, s);
+    if (g.nb <= 1536) return launch_select<48, true>(rows, g.nb, L, p, k_floor, kv_idx, kv_cnt, s);
+    return launch_select<80, false>(rows, g.nb, L, p, k_floor, kv_idx, kv_cnt, s);
 }
