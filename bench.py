@@ -32,7 +32,7 @@ if ROOT not in sys.path:
 METRIC = "sparse-attn TFLOPS on executed blocks (% of bf16 peak) + end-to-end ms per layer"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 WORKLOAD = "720p"
-KERNELS_PER_STEP = 9   # reorder x3, pool, score/select, 2 work-list kernels, attention, inverse
+KERNELS_PER_STEP = 10  # reorder x3, pool, score, select, 2 work-list kernels, attention, inverse
 
 
 def load_peaks():
