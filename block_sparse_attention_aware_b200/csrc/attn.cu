@@ -36,6 +36,8 @@
 
 #include "common.cuh"
 #include "ptx.cuh"
+#include "sync.cuh"
+#include "tmap.cuh"
 
 namespace fv {
 
@@ -47,7 +49,6 @@ constexpr int V_STAGES = 2;             // V ring: a stage is free once its O +=
 constexpr uint32_t MAX_DYN_SMEM = 232448;   // sm_100 opt-in shared memory per block
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t O_COL = 256;          // S_w at columns 128*w, O_w at 256 + 128*w
-constexpr unsigned long long WAIT_LIMIT_NS = 4000000000ull;
 // Lazy rescaling: the running row maximum (log2 units) is only moved, and O
 // rescaled, when a new score exceeds it by more than this; until then
 // probabilities may reach 2^8, which bf16 P and fp32 sums hold exactly enough.
@@ -106,35 +107,6 @@ struct Smem {
     static constexpr uint32_t ALLOC = TOTAL > 120u * 1024u ? TOTAL : 120u * 1024u;
     static_assert(ALLOC <= MAX_DYN_SMEM, "shared-memory layout too large");
 };
-
-// Bounded mbarrier wait.  Returns false if the CTA aborted or the wait ran
-// past WAIT_LIMIT_NS (then it records the timeout and raises the abort flag).
-__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
-    if (mbar_try_wait(bar, parity)) return true;
-    unsigned long long t0 = 0;
-    for (uint32_t it = 1;; ++it) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((it & 255u) == 0u) {
-            if (*abort_flag) return false;
-            unsigned long long now = global_timer_ns();
-            if (t0 == 0) {
-                t0 = now;
-            } else if (now - t0 > WAIT_LIMIT_NS) {
-                record_status(FVATTN_ERR_TIMEOUT);
-                *abort_flag = 1;
-                return false;
-            }
-        }
-    }
-}
-
-// Warp-uniform variant: every lane waits, and the warp leaves together if
-// any lane gave up (the .sync.aligned tcgen05 loads that follow need the
-// whole warp).
-__device__ __forceinline__ bool wait_warp(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
-    const bool ok = wait_bar(bar, parity, abort_flag);
-    return __all_sync(0xffffffffu, ok);
-}
 
 // Real extent of a tile: frames, rows and cols that hold tokens, packed as
 // nf | ny << 8 | nx << 16 (each <= 128).
@@ -738,36 +710,11 @@ __global__ void __launch_bounds__(256) worklist_heads_kernel(int BH, const long 
 
 // ------------------------------------------------------------------ host side
 
-typedef CUresult (*PFN_encodeTiled)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                    const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                    CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-static PFN_encodeTiled get_encode() {
-    static PFN_encodeTiled fn = nullptr;
-    if (!fn) {
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
-            q != cudaDriverEntryPointSuccess)
-            return nullptr;
-        fn = reinterpret_cast<PFN_encodeTiled>(p);
-    }
-    return fn;
-}
-
 // 2-D view [rows, D] of a tiled tensor, boxes of bs rows x 64 columns,
 // 128-byte swizzle (the tcgen05 K-major / MN-major SW128 operand layout).
 static bool make_tmap(CUtensorMap* m, const void* base, long long rows, int D, int bs) {
-    PFN_encodeTiled enc = get_encode();
-    if (!enc) return false;
-    cuuint64_t dims[2] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows)};
-    cuuint64_t strides[1] = {static_cast<cuuint64_t>(D) * 2u};
-    cuuint32_t box[2] = {64u, static_cast<cuuint32_t>(bs)};
-    cuuint32_t estr[2] = {1u, 1u};
-    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
+    return make_tmap_2d(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, static_cast<unsigned long long>(rows),
+                        static_cast<unsigned long long>(D), 64u, static_cast<unsigned>(bs));
 }
 
 struct WsLayout {

@@ -5,13 +5,13 @@
 // a minimum budget; dynamic masks come from the current attention features).
 //
 // Three kernels:
-//   pool_kernel    HBM-bound.  One CTA per (tensor, b, h, block) sums the
+//   pool_kernel    HBM-bound.  One warp per (tensor, b, h, block) sums the
 //                  block's real rows with 16-byte loads, all issued before the
 //                  first add (padding rows are never read), and writes the fp32
-//                  mean.
-//   score_kernel   L = scale * Qp Kp^T per (b, h): an fp32 register-tiled
-//                  product, 64 x 64 logits per CTA, 4 x 4 per thread, operands
-//                  staged in shared memory k-major.
+//                  mean split into its tf32 part and the exact remainder.
+//   score_kernel   L = scale * Qp Kp^T per (b, h) on the tensor cores
+//                  (tcgen05 kind::tf32, TMEM accumulators) as three tf32
+//                  products hi*hi + hi*lo + lo*hi: about fp32 accuracy.
 //   select_kernel  One warp per (b, h, query block) row, the row's logits and
 //                  their masses e_j = exp(L_j - max L) in registers.  The
 //                  weight of a set {L >= t} is an exact fixed-point integer (a
@@ -27,6 +27,8 @@
 //                  indices are written in ascending order with ballots.
 #include "common.cuh"
 #include "ptx.cuh"
+#include "sync.cuh"
+#include "tmap.cuh"
 
 namespace fv {
 
@@ -36,10 +38,15 @@ namespace fv {
 // 16-byte column slice (D/8 slices per row) of every (32 / (D/8))-th row, so
 // one warp instruction reads 512 contiguous bytes; full tiles issue all their
 // loads before the first add.
+struct PoolOut {
+    float* hi[2];     // [q, k]: tf32 part of the mean (low 13 mantissa bits cleared)
+    float* lo[2];     // [q, k]: mean - hi (exact)
+    float* mean[2];   // [q, k]: the fp32 mean itself, or null
+};
+
 template <int D>
 __global__ void __launch_bounds__(256, 3) pool_kernel(Geo g, const __nv_bfloat16* __restrict__ qt,
-                                                   const __nv_bfloat16* __restrict__ kt,
-                                                   float* __restrict__ qp, float* __restrict__ kp) {
+                                                   const __nv_bfloat16* __restrict__ kt, PoolOut out) {
     constexpr int VPR = D / 8;             // 16-byte vectors per row
     constexpr int RPI = 32 / VPR;          // rows per warp instruction
     constexpr int UNR = 8;                 // loads in flight per lane
@@ -53,7 +60,7 @@ __global__ void __launch_bounds__(256, 3) pool_kernel(Geo g, const __nv_bfloat16
     const int blk = static_cast<int>(ub - bh * g.nb);
     const uint4* src = reinterpret_cast<const uint4*>((is_k ? kt : qt) +
                                                       (bh * g.Npad + static_cast<long long>(blk) * g.bs) * D);
-    float* dst = (is_k ? kp : qp) + (bh * g.nb + blk) * D;
+    const long long dst_off = (bh * g.nb + blk) * D;
     const int vec = lane % VPR;
     const int r0 = lane / VPR;
     const int bx = blk % g.nbx, by = (blk / g.nbx) % g.nby, bf = blk / (g.nbx * g.nby);
@@ -100,71 +107,230 @@ __global__ void __launch_bounds__(256, 3) pool_kernel(Geo g, const __nv_bfloat16
         for (int e = 0; e < 8; ++e) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], o);
     if (lane < VPR) {
         const float inv = 1.0f / static_cast<float>(nf * ny * nx);
-        float4* d4 = reinterpret_cast<float4*>(dst + lane * 8);
-        d4[0] = make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
-        d4[1] = make_float4(acc[4] * inv, acc[5] * inv, acc[6] * inv, acc[7] * inv);
+        float m[8], h[8], l[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            m[e] = acc[e] * inv;
+            h[e] = __uint_as_float(__float_as_uint(m[e]) & 0xffffe000u);
+            l[e] = m[e] - h[e];
+        }
+        const long long o = dst_off + lane * 8;
+        float* mp = is_k ? out.mean[1] : out.mean[0];
+        float4* dh = reinterpret_cast<float4*>((is_k ? out.hi[1] : out.hi[0]) + o);
+        float4* dl = reinterpret_cast<float4*>((is_k ? out.lo[1] : out.lo[0]) + o);
+        dh[0] = make_float4(h[0], h[1], h[2], h[3]);
+        dh[1] = make_float4(h[4], h[5], h[6], h[7]);
+        dl[0] = make_float4(l[0], l[1], l[2], l[3]);
+        dl[1] = make_float4(l[4], l[5], l[6], l[7]);
+        if (mp) {
+            float4* dm = reinterpret_cast<float4*>(mp + o);
+            dm[0] = make_float4(m[0], m[1], m[2], m[3]);
+            dm[1] = make_float4(m[4], m[5], m[6], m[7]);
+        }
     }
 }
 
-// ------------------------------------------------------------------ scores
+// ------------------------------------------------------------------ scoring
 
-constexpr int SC_TILE = 64;   // logits per CTA side
-constexpr int SC_KC = 32;     // head-dim slice staged per step
+// L = scale * Qp Kp^T per (b, h) on the tensor cores, in three tf32 products:
+// with x = x_hi + x_lo (x_hi the tf32 part), Qp Kp^T is taken as
+// hi*hi + hi*lo + lo*hi, which leaves only the lo*lo term (2^-22 relative)
+// out, close to an fp32 product.  A tile is 128 query blocks x 256 key
+// blocks; its accumulator lives in TMEM (256 fp32 columns, two tiles in
+// flight).  Persistent CTAs, warp-specialised:
+//   warp 0      TMA producer: per 32-wide slice of the head dimension, the
+//               hi and lo parts of the Q rows and the K rows (96 KB a stage,
+//               two stages), 128-byte swizzled, K-major.
+//   warp 1      TMEM owner and MMA issuer: 4 x 3 MMAs (M=128, N=256, K=8) a
+//               slice; a commit frees the stage, the tile's last commit hands
+//               the accumulator to the epilogue.
+//   warps 2-5   epilogue: each thread owns one query-block row of the tile
+//               (the warp's TMEM lane quarter), reads 32 columns at a time,
+//               scales and stores the real (row < nb, col < nb) logits.
+constexpr int SC_BM = 128;                 // query blocks per tile (MMA M)
+constexpr int SC_BN = 256;                 // key blocks per tile (MMA N)
+constexpr int SC_SLICE = 32;               // fp32 head-dim elements per stage (128 bytes)
+constexpr int SC_STAGES = 2;
+constexpr int SC_THREADS = 192;
+constexpr uint32_t SC_A_BYTES = SC_BM * 128u;
+constexpr uint32_t SC_B_BYTES = SC_BN * 128u;
+constexpr uint32_t SC_STAGE_BYTES = 2u * SC_A_BYTES + 2u * SC_B_BYTES;
+constexpr uint32_t SC_TMEM_COLS = 2u * SC_BN;
 
-// L[bh][i][j] = scale * <Qp[bh][i], Kp[bh][j]>; grid (tiles_j, tiles_i, B*H).
-__global__ void __launch_bounds__(256) score_kernel(Geo g, const float* __restrict__ qp, const float* __restrict__ kp,
-                                                    float scale, float* __restrict__ L) {
-    __shared__ __align__(16) float As[SC_KC][SC_TILE + 4];
-    __shared__ __align__(16) float Bs[SC_KC][SC_TILE + 4];
-    const int nb = g.nb, D = g.D;
-    const long long bh = blockIdx.z;
-    const int i0 = blockIdx.y * SC_TILE, j0 = blockIdx.x * SC_TILE;
-    const float* A = qp + bh * nb * D;
-    const float* Bm = kp + bh * nb * D;
-    const int tid = threadIdx.x;
-    const int ty = tid / 16, tx = tid % 16;
-    float acc[4][4];
-#pragma unroll
-    for (int a = 0; a < 4; ++a)
-#pragma unroll
-        for (int b = 0; b < 4; ++b) acc[a][b] = 0.f;
-    for (int k0 = 0; k0 < D; k0 += SC_KC) {
-        // 64 rows x 32 floats of each operand: 512 float4, two per thread,
-        // stored transposed (k-major)
-#pragma unroll
-        for (int rep = 0; rep < 2; ++rep) {
-            const int idx = tid + rep * 256;
-            const int r = idx / (SC_KC / 4), c4 = idx % (SC_KC / 4);
-            float4 va = make_float4(0.f, 0.f, 0.f, 0.f), vb = va;
-            if (i0 + r < nb) va = __ldg(reinterpret_cast<const float4*>(A + static_cast<long long>(i0 + r) * D + k0) + c4);
-            if (j0 + r < nb) vb = __ldg(reinterpret_cast<const float4*>(Bm + static_cast<long long>(j0 + r) * D + k0) + c4);
-            As[c4 * 4 + 0][r] = va.x; As[c4 * 4 + 1][r] = va.y; As[c4 * 4 + 2][r] = va.z; As[c4 * 4 + 3][r] = va.w;
-            Bs[c4 * 4 + 0][r] = vb.x; Bs[c4 * 4 + 1][r] = vb.y; Bs[c4 * 4 + 2][r] = vb.z; Bs[c4 * 4 + 3][r] = vb.w;
+struct ScoreCtrl {
+    unsigned long long full[SC_STAGES];
+    unsigned long long empty[SC_STAGES];
+    unsigned long long acc_full[2];
+    unsigned long long acc_empty[2];
+    unsigned long long drained;
+    uint32_t tmem_base;
+    int abort_flag;
+};
+
+constexpr uint32_t SC_CTRL_OFF = SC_STAGES * SC_STAGE_BYTES;
+constexpr uint32_t SC_SMEM = SC_CTRL_OFF + static_cast<uint32_t>(sizeof(ScoreCtrl));
+static_assert(SC_SMEM <= 232448u, "score kernel shared memory");
+
+struct ScoreArgs {
+    float* L;
+    float scale;
+    int nb;
+    int m_tiles, n_tiles;
+    int slices;            // D / 32
+    long long tiles;       // B*H * m_tiles * n_tiles
+};
+
+__global__ void __launch_bounds__(SC_THREADS, 1) score_kernel(const __grid_constant__ CUtensorMap tq_hi,
+                                                              const __grid_constant__ CUtensorMap tq_lo,
+                                                              const __grid_constant__ CUtensorMap tk_hi,
+                                                              const __grid_constant__ CUtensorMap tk_lo,
+                                                              ScoreArgs a) {
+    extern __shared__ __align__(1024) unsigned char sc_smem[];
+    ScoreCtrl& ctl = *reinterpret_cast<ScoreCtrl*>(sc_smem + SC_CTRL_OFF);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    volatile int* abort_flag = &ctl.abort_flag;
+    if (threadIdx.x == 0) {
+        if ((smem_u32(sc_smem) & 1023u) != 0u) record_status(FVATTN_ERR_BOUNDS);
+        for (int s = 0; s < SC_STAGES; ++s) {
+            mbar_init(smem_u32(&ctl.full[s]), 1);
+            mbar_init(smem_u32(&ctl.empty[s]), 1);
         }
-        __syncthreads();
-#pragma unroll 8
-        for (int k = 0; k < SC_KC; ++k) {
-            const float4 a = *reinterpret_cast<const float4*>(&As[k][ty * 4]);
-            const float4 b = *reinterpret_cast<const float4*>(&Bs[k][tx * 4]);
-            const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
-#pragma unroll
-            for (int x = 0; x < 4; ++x)
-#pragma unroll
-                for (int y = 0; y < 4; ++y) acc[x][y] = fmaf(av[x], bv[y], acc[x][y]);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(smem_u32(&ctl.acc_full[b]), 1);
+            mbar_init(smem_u32(&ctl.acc_empty[b]), 128);
         }
-        __syncthreads();
+        mbar_init(smem_u32(&ctl.drained), 1);
+        ctl.abort_flag = (smem_u32(sc_smem) & 1023u) != 0u;
+        fence_mbar_init();
     }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(&ctl.tmem_base), SC_TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = ctl.tmem_base;
+    const int per_head = a.m_tiles * a.n_tiles;
+
+    if (warp == 0) {
+        // ---- TMA producer
+        if (lane == 0 && !*abort_flag) {
+            prefetch_tmap(&tq_hi);
+            prefetch_tmap(&tq_lo);
+            prefetch_tmap(&tk_hi);
+            prefetch_tmap(&tk_lo);
+            long long seq = 0;
+            for (long long t = blockIdx.x; t < a.tiles; t += gridDim.x) {
+                const long long bh = t / per_head;
+                const int rem = static_cast<int>(t - bh * per_head);
+                const int qrow = static_cast<int>(bh * a.nb) + (rem / a.n_tiles) * SC_BM;
+                const int krow = static_cast<int>(bh * a.nb) + (rem % a.n_tiles) * SC_BN;
+                bool ok = true;
+                for (int ks = 0; ks < a.slices; ++ks, ++seq) {
+                    const int s = static_cast<int>(seq % SC_STAGES);
+                    if (!wait_bar(smem_u32(&ctl.empty[s]), ((seq / SC_STAGES) & 1) ^ 1, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t base = smem_u32(sc_smem + s * SC_STAGE_BYTES);
+                    const uint32_t fb = smem_u32(&ctl.full[s]);
+                    mbar_arrive_expect_tx(fb, SC_STAGE_BYTES);
+                    tma_load_2d(base, &tq_hi, ks * SC_SLICE, qrow, fb);
+                    tma_load_2d(base + SC_A_BYTES, &tq_lo, ks * SC_SLICE, qrow, fb);
+                    tma_load_2d(base + 2 * SC_A_BYTES, &tk_hi, ks * SC_SLICE, krow, fb);
+                    tma_load_2d(base + 2 * SC_A_BYTES + SC_B_BYTES, &tk_lo, ks * SC_SLICE, krow, fb);
+                }
+                if (!ok) break;
+            }
+            // copies still in flight finish before the CTA can exit
+            for (long long q = seq > SC_STAGES ? seq - SC_STAGES : 0; q < seq; ++q)
+                wait_bar_drain(smem_u32(&ctl.full[q % SC_STAGES]), (q / SC_STAGES) & 1);
+        }
+    } else if (warp == 1) {
+        // ---- MMA issuer
+        if (lane == 0 && !*abort_flag) {
+            constexpr uint32_t idesc = idesc_tf32_f32(SC_BM, SC_BN);
+            long long seq = 0, tcount = 0;
+            for (long long t = blockIdx.x; t < a.tiles; t += gridDim.x, ++tcount) {
+                const int b = static_cast<int>(tcount & 1);
+                if (!wait_bar(smem_u32(&ctl.acc_empty[b]), ((tcount >> 1) & 1) ^ 1, abort_flag)) break;
+                tc_fence_after();
+                const uint32_t d = tmem + static_cast<uint32_t>(b * SC_BN);
+                bool ok = true;
+                for (int ks = 0; ks < a.slices; ++ks, ++seq) {
+                    const int s = static_cast<int>(seq % SC_STAGES);
+                    if (!wait_bar(smem_u32(&ctl.full[s]), (seq / SC_STAGES) & 1, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t base = smem_u32(sc_smem + s * SC_STAGE_BYTES);
 #pragma unroll
-    for (int x = 0; x < 4; ++x) {
-        const int i = i0 + ty * 4 + x;
-        if (i >= nb) continue;
-        float* row = L + (bh * nb + i) * nb;
+                    for (int kk = 0; kk < SC_SLICE / 8; ++kk) {
+                        const uint32_t off = kk * 32u;   // 8 tf32 = 32 bytes inside the swizzle atom
+                        const uint64_t ah = sw128_desc(base + off, 16, 1024);
+                        const uint64_t al = sw128_desc(base + SC_A_BYTES + off, 16, 1024);
+                        const uint64_t bhd = sw128_desc(base + 2 * SC_A_BYTES + off, 16, 1024);
+                        const uint64_t bld = sw128_desc(base + 2 * SC_A_BYTES + SC_B_BYTES + off, 16, 1024);
+                        mma_tf32_ss(d, ah, bhd, idesc, (ks | kk) != 0);
+                        mma_tf32_ss(d, ah, bld, idesc, 1u);
+                        mma_tf32_ss(d, al, bhd, idesc, 1u);
+                    }
+                    mma_commit(smem_u32(&ctl.empty[s]));
+                }
+                if (!ok) break;
+                mma_commit(smem_u32(&ctl.acc_full[b]));
+            }
+            // MMAs still in flight finish before TMEM is released
+            mma_commit(smem_u32(&ctl.drained));
+            wait_bar_drain(smem_u32(&ctl.drained), 0);
+        }
+    } else {
+        // ---- epilogue: thread = one query-block row of the tile
+        const int quarter = warp & 3;
+        const int r_in = quarter * 32 + lane;
+        const bool vec_ok = (a.nb & 3) == 0;
+        long long tcount = 0;
+        for (long long t = blockIdx.x; t < a.tiles; t += gridDim.x, ++tcount) {
+            const int b = static_cast<int>(tcount & 1);
+            if (!wait_warp(smem_u32(&ctl.acc_full[b]), (tcount >> 1) & 1, abort_flag)) break;
+            tc_fence_after();
+            const long long bh = t / per_head;
+            const int rem = static_cast<int>(t - bh * per_head);
+            const int row = (rem / a.n_tiles) * SC_BM + r_in;
+            const int col0 = (rem % a.n_tiles) * SC_BN;
+            float* out = a.L + (bh * a.nb + row) * static_cast<long long>(a.nb);
+            const bool row_ok = row < a.nb;
+            for (int c = 0; c < SC_BN; c += 32) {
+                const int col = col0 + c;
+                if (col >= a.nb) break;
+                uint32_t r[32];
+                tmem_ld32(tmem + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(b * SC_BN + c), r);
+                tmem_wait_ld();
+                if (row_ok && vec_ok && col + 32 <= a.nb) {
+                    float4* o4 = reinterpret_cast<float4*>(out + col);
 #pragma unroll
-        for (int y = 0; y < 4; ++y) {
-            const int j = j0 + tx * 4 + y;
-            if (j < nb) row[j] = acc[x][y] * scale;
+                    for (int v = 0; v < 8; ++v)
+                        o4[v] = make_float4(__uint_as_float(r[4 * v]) * a.scale, __uint_as_float(r[4 * v + 1]) * a.scale,
+                                            __uint_as_float(r[4 * v + 2]) * a.scale,
+                                            __uint_as_float(r[4 * v + 3]) * a.scale);
+                } else if (row_ok) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        if (col + i < a.nb) out[col + i] = __uint_as_float(r[i]) * a.scale;
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(smem_u32(&ctl.acc_empty[b]));
         }
     }
+
+    // ---- teardown
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem, SC_TMEM_COLS);
 }
 
 // ------------------------------------------------------------------ selection
@@ -401,8 +567,10 @@ static int launch_select(long long rows, int nb, const float* L, double p, int k
 
 static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Workspace: tf32 hi / lo parts of the pooled Q and K ([B*H*nb, D] fp32
+// each), then the logits ([B*H*nb, nb] fp32).
 struct RouteWs {
-    size_t qp, kp, logits, total;
+    size_t qh, ql, kh, kl, logits, total;
 };
 
 static size_t al256(size_t x) { return (x + 255) / 256 * 256; }
@@ -411,11 +579,20 @@ static RouteWs route_ws(const fvattn_geom& g) {
     RouteWs w;
     const size_t BH = static_cast<size_t>(g.B) * g.H;
     const size_t pooled = al256(sizeof(float) * BH * g.nb * g.D);
-    w.qp = 0;
-    w.kp = pooled;
-    w.logits = 2 * pooled;
+    w.qh = 0;
+    w.ql = pooled;
+    w.kh = 2 * pooled;
+    w.kl = 3 * pooled;
+    w.logits = 4 * pooled;
     w.total = w.logits + al256(sizeof(float) * BH * g.nb * g.nb);
     return w;
+}
+
+static int score_sms() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    return n;
 }
 
 }  // namespace fv
@@ -439,25 +616,51 @@ extern "C" int fvattn_route(const fvattn_geom* gp, const void* q_tiled, const vo
     const Geo g = to_geo(*gp);
     const RouteWs wl = route_ws(*gp);
     char* ws = static_cast<char*>(workspace);
-    const bool need_ws = !q_pool || !k_pool || !logits;
-    if (need_ws && (!workspace || ws_bytes < wl.total || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0))
+    if (!workspace || ws_bytes < wl.total || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
         return FVATTN_ERR_INVALID;
-    float* qp = q_pool ? q_pool : reinterpret_cast<float*>(ws + wl.qp);
-    float* kp = k_pool ? k_pool : reinterpret_cast<float*>(ws + wl.kp);
+    if ((q_pool && !aligned16(q_pool)) || (k_pool && !aligned16(k_pool)) || (logits && !aligned16(logits)))
+        return FVATTN_ERR_INVALID;
     float* L = logits ? logits : reinterpret_cast<float*>(ws + wl.logits);
-    if (!aligned16(qp) || !aligned16(kp) || !aligned16(L)) return FVATTN_ERR_INVALID;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    PoolOut po;
+    po.hi[0] = reinterpret_cast<float*>(ws + wl.qh);
+    po.lo[0] = reinterpret_cast<float*>(ws + wl.ql);
+    po.hi[1] = reinterpret_cast<float*>(ws + wl.kh);
+    po.lo[1] = reinterpret_cast<float*>(ws + wl.kl);
+    po.mean[0] = q_pool;
+    po.mean[1] = k_pool;
     const long long units = 2ll * g.B * g.H * g.nb;
     const unsigned pblocks = static_cast<unsigned>((units + 7) / 8);
     if (g.D == 128)
         pool_kernel<128><<<pblocks, 256, 0, s>>>(g, static_cast<const __nv_bfloat16*>(q_tiled),
-                                                 static_cast<const __nv_bfloat16*>(k_tiled), qp, kp);
+                                                 static_cast<const __nv_bfloat16*>(k_tiled), po);
     else
         pool_kernel<64><<<pblocks, 256, 0, s>>>(g, static_cast<const __nv_bfloat16*>(q_tiled),
-                                                static_cast<const __nv_bfloat16*>(k_tiled), qp, kp);
+                                                static_cast<const __nv_bfloat16*>(k_tiled), po);
     FV_CHECK_LAUNCH();
-    const int tiles = (g.nb + SC_TILE - 1) / SC_TILE;
-    score_kernel<<<dim3(tiles, tiles, g.B * g.H), 256, 0, s>>>(g, qp, kp, scale, L);
+
+    const unsigned long long prow = static_cast<unsigned long long>(g.B) * g.H * g.nb;
+    CUtensorMap tqh, tql, tkh, tkl;
+    if (!make_tmap_2d(&tqh, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, po.hi[0], prow, g.D, SC_SLICE, SC_BM) ||
+        !make_tmap_2d(&tql, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, po.lo[0], prow, g.D, SC_SLICE, SC_BM) ||
+        !make_tmap_2d(&tkh, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, po.hi[1], prow, g.D, SC_SLICE, SC_BN) ||
+        !make_tmap_2d(&tkl, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, po.lo[1], prow, g.D, SC_SLICE, SC_BN))
+        return FVATTN_ERR_CUDA;
+    ScoreArgs sa;
+    sa.L = L;
+    sa.scale = scale;
+    sa.nb = g.nb;
+    sa.m_tiles = (g.nb + SC_BM - 1) / SC_BM;
+    sa.n_tiles = (g.nb + SC_BN - 1) / SC_BN;
+    sa.slices = g.D / SC_SLICE;
+    sa.tiles = static_cast<long long>(g.B) * g.H * sa.m_tiles * sa.n_tiles;
+    const int nsm = score_sms();
+    if (nsm <= 0) return FVATTN_ERR_CUDA;
+    if (cudaFuncSetAttribute(score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(SC_SMEM)) !=
+        cudaSuccess)
+        return FVATTN_ERR_CUDA;
+    const unsigned sgrid = static_cast<unsigned>(sa.tiles < nsm ? sa.tiles : nsm);
+    score_kernel<<<sgrid, SC_THREADS, SC_SMEM, s>>>(tqh, tql, tkh, tkl, sa);
     FV_CHECK_LAUNCH();
     const long long rows = static_cast<long long>(g.B) * g.H * g.nb;
     if (g.nb <= 768) return launch_select<24, true>(rows, g.nb, L, p, k_floor, kv_idx, kv_cnt, s);

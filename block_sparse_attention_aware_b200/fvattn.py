@@ -175,7 +175,7 @@ def route(g: Geom, qt: torch.Tensor, kt: torch.Tensor, p: float, k: int,
             out.q_pool = torch.empty((g.B, g.H, g.nb, g.D), dtype=torch.float32, device=dev)
             out.k_pool = torch.empty_like(out.q_pool)
             out.logits = torch.empty((g.B, g.H, g.nb, g.nb), dtype=torch.float32, device=dev)
-    if workspace is None and (out.q_pool is None or out.k_pool is None):
+    if workspace is None:
         workspace = route_workspace(g, dev)
     rc = load().fvattn_route(ctypes.byref(g), _ptr(qt), _ptr(kt), float(p), int(k), float(scale),
                              _ptr(out.kv_idx), _ptr(out.kv_cnt), _ptr(out.q_pool), _ptr(out.k_pool),

@@ -93,7 +93,9 @@ int fvattn_reorder(const fvattn_geom *g, const void *x, void *x_tiled, fvattn_st
 int fvattn_inverse_reorder(const fvattn_geom *g, const void *o_tiled, void *o,
                            fvattn_stream_t stream);
 
-/* Bytes of device workspace fvattn_route needs (pooled Q and K, fp32). */
+/* Bytes of device workspace fvattn_route needs: the pooled Q and K split
+ * into tf32 high and low parts (4 x [B, H, nb, D] fp32) and the logits
+ * ([B, H, nb, nb] fp32). */
 size_t fvattn_route_workspace_size(const fvattn_geom *g);
 
 /* Sparse-routing frontend (paperlayer.ai summary, section 3,
@@ -101,7 +103,9 @@ size_t fvattn_route_workspace_size(const fvattn_geom *g);
  * section 2: Top-p keeps the smallest cumulative-importance set, the Top-k
  * safety floor a minimum budget).  Per (b, h):
  *   Qp[i] = mean of the real tokens of query block i (fp32), Kp likewise;
- *   L[i][j] = scale * Qp[i] . Kp[j]                      (fp32)
+ *   L[i][j] = scale * Qp[i] . Kp[j]                      (fp32; on the tensor
+ *             cores as three tf32 products hi*hi + hi*lo + lo*hi of the
+ *             split Qp = hi + lo, Kp likewise: about fp32 accuracy)
  *   order blocks of row i by L descending, equal L by lower j;
  *   P = softmax(L[i]); m_p = smallest prefix whose mass reaches p
  *   (m_p = nb when p >= 1); m = max(m_p, min(k_floor, nb));
@@ -118,7 +122,7 @@ size_t fvattn_route_workspace_size(const fvattn_geom *g);
  *   q_pool, k_pool    optional [B, H, nb, D] fp32 outputs (may be NULL)
  *   logits            optional [B, H, nb, nb] fp32 output of L (may be NULL)
  *   workspace         device scratch of >= fvattn_route_workspace_size bytes,
- *                     256-byte aligned
+ *                     256-byte aligned (always required)
  * Logits must be finite (NaN inputs give an unspecified mask). */
 int fvattn_route(const fvattn_geom *g, const void *q_tiled, const void *k_tiled,
                  double p, int k_floor, float scale,

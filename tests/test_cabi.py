@@ -81,7 +81,7 @@ def test_workspace_sizes(fv):
     g = fv.geom(1, 40, 128, 21, 45, 80, 2, 8, 8)
     rw = lib.fvattn_route_workspace_size(ctypes.byref(g))
     aw = lib.fvattn_attn_workspace_size(ctypes.byref(g))
-    assert rw >= 2 * 40 * 660 * 128 * 4
+    assert rw >= 4 * 40 * 660 * 128 * 4 + 40 * 660 * 660 * 4
     assert aw >= 40 * 660 * 4 + 40 * 8 + 40 * 4 + 4
     assert rw % 256 == 0 and aw % 256 == 0
 
