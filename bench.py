@@ -32,7 +32,8 @@ if ROOT not in sys.path:
 METRIC = "sparse-attn TFLOPS on executed blocks (% of bf16 peak) + end-to-end ms per layer"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 WORKLOAD = "720p"
-KERNELS_PER_STEP = 10  # reorder x3, pool, score, select, 2 work-list kernels, attention, inverse
+# kernels per step besides routing's: reorder x3, 2 work-list kernels, attention, inverse reorder
+OTHER_KERNELS_PER_STEP = 7
 
 
 def load_peaks():
@@ -325,7 +326,7 @@ def run_fvattn(args):
                      "kernel": "sparse_attn_kernel<128>",
                      "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside back-to-back steps)",
                      "algorithmic_flops_per_launch": flops},
-        "gpu_launches": KERNELS_PER_STEP * args.steps,
+        "gpu_launches": (OTHER_KERNELS_PER_STEP + fvattn.route_kernel_launches(g)) * args.steps,
         "clocks": clock_info,
     }
 

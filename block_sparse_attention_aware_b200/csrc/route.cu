@@ -604,6 +604,11 @@ extern "C" size_t fvattn_route_workspace_size(const fvattn_geom* gp) {
     return route_ws(*gp).total;
 }
 
+extern "C" int fvattn_route_kernel_launches(const fvattn_geom* gp) {
+    if (!gp || gp->B <= 0 || gp->H <= 0) return 0;
+    return 3;   // pool, score, select
+}
+
 extern "C" int fvattn_route(const fvattn_geom* gp, const void* q_tiled, const void* k_tiled, double p, int k_floor,
                             float scale, int32_t* kv_idx, int32_t* kv_cnt, float* q_pool, float* k_pool,
                             float* logits, void* workspace, size_t ws_bytes, fvattn_stream_t stream) {
@@ -663,7 +668,17 @@ extern "C" int fvattn_route(const fvattn_geom* gp, const void* q_tiled, const vo
     score_kernel<<<sgrid, SC_THREADS, SC_SMEM, s>>>(tqh, tql, tkh, tkl, sa);
     FV_CHECK_LAUNCH();
     const long long rows = static_cast<long long>(g.B) * g.H * g.nb;
-    if (g.nb <= 768) return launch_select<24, true>(rows, g.nb, L, p, k_floor, kv_idx, kv_cnt, s);
-    if (g.nb <= 1536) return launch_select<48, true>(rows, g.nb, L, p, k_floor, kv_idx, kv_cnt, s);
+    // entries per lane: the smallest instantiated count that covers a row
+    const int npl = (g.nb + 31) / 32;
+    if (npl <= 4) return launch_select<4, true>(rows, g.nb, L, p, k_floor, kv_idx, kv_cnt, s);
+    if (npl <= 8) return launch_select<8, true>(rows, g.nb, L, p, k_floor, kv_idx, kv_cnt, s);
+    if (npl <= 10) return launch_select<10, true>(rows, g.nb, L, p, k_floor, kv_idx, kv_cnt, s);
+    if (npl <= 12) return launch_select<12, true>(rows, g.nb, L, p, k_floor, kv_idx, kv_cnt, s);
+    if (npl <= 16) return launch_select<16, true>(rows, g.nb, L, p, k_floor, kv_idx, kv_cnt, s);
+    if (npl <= 21) return launch_select<21, true>(rows, g.nb, L, p, k_floor, kv_idx, kv_cnt, s);
+    if (npl <= 24) return launch_select<24, true>(rows, g.nb, L, p, k_floor, kv_idx, kv_cnt, s);
+    if (npl <= 32) return launch_select<32, true>(rows, g.nb, L, p, k_floor, kv_idx, kv_cnt, s);
+    if (npl <= 40) return launch_select<40, true>(rows, g.nb, L, p, k_floor, kv_idx, kv_cnt, s);
+    if (npl <= 48) return launch_select<48, true>(rows, g.nb, L, p, k_floor, kv_idx, kv_cnt, s);
     return launch_select<80, false>(rows, g.nb, L, p, k_floor, kv_idx, kv_cnt, s);
 }

@@ -21,7 +21,8 @@ _lib = None
 
 OK, ERR_INVALID, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_BOUNDS = range(6)
 EXPORTED = ("fvattn_geom_init", "fvattn_reorder", "fvattn_inverse_reorder",
-            "fvattn_route_workspace_size", "fvattn_route", "fvattn_attn_workspace_size",
+            "fvattn_route_workspace_size", "fvattn_route_kernel_launches", "fvattn_route",
+            "fvattn_attn_workspace_size",
             "fvattn_num_sms", "fvattn_sparse_attn", "fvattn_sparse_attn_noalloc", "fvattn_get_status",
             "fvattn_status_string")
 
@@ -59,6 +60,8 @@ def load(path: str = LIB_PATH):
     L.fvattn_inverse_reorder.restype = I
     L.fvattn_route_workspace_size.argtypes = [G]
     L.fvattn_route_workspace_size.restype = S
+    L.fvattn_route_kernel_launches.argtypes = [G]
+    L.fvattn_route_kernel_launches.restype = I
     L.fvattn_route.argtypes = [G, P, P, ctypes.c_double, I, ctypes.c_float, P, P, P, P, P, P, S, P]
     L.fvattn_route.restype = I
     L.fvattn_attn_workspace_size.argtypes = [G]
@@ -110,6 +113,11 @@ def geom(B, H, D, F, Hs, Ws, tf, th, tw) -> Geom:
 def geom_of(w) -> Geom:
     """Geometry of a synth.Workload."""
     return geom(w.B, w.H, w.D, w.F, w.Hs, w.Ws, w.tf, w.th, w.tw)
+
+
+def route_kernel_launches(g: Geom) -> int:
+    """Kernel launches one fvattn_route call makes for this geometry."""
+    return load().fvattn_route_kernel_launches(ctypes.byref(g))
 
 
 def num_sms() -> int:

@@ -130,6 +130,10 @@ int fvattn_route(const fvattn_geom *g, const void *q_tiled, const void *k_tiled,
                  float *q_pool, float *k_pool, float *logits,
                  void *workspace, size_t ws_bytes, fvattn_stream_t stream);
 
+/* Number of kernel launches one fvattn_route call makes for this geometry
+ * (pooling, scoring, selection); 0 for a null pointer. */
+int fvattn_route_kernel_launches(const fvattn_geom *g);
+
 /* Bytes of device workspace fvattn_sparse_attn needs (work list, head
  * order, per-block validity masks, work counter). */
 size_t fvattn_attn_workspace_size(const fvattn_geom *g);

@@ -27,7 +27,7 @@ def _declared():
 def test_exports_every_declared_symbol(fv):
     lib = fv.load()
     names = _declared()
-    assert len(names) == 11
+    assert len(names) == 12
     assert sorted(fv.EXPORTED) == names
     for n in names:
         assert hasattr(lib, n), n
@@ -100,3 +100,11 @@ def test_product_path_has_no_oracle_import():
             if f.endswith((".py", ".cu", ".cuh", ".h")):
                 txt = open(os.path.join(dirpath, f)).read()
                 assert not re.search(r"(import\s+oracle|from\s+oracle|liboracle|fvattn_oracle)", txt), f
+
+
+def test_route_kernel_launches(fv):
+    """Routing is three kernels: pooling, scoring, selection."""
+    lib = fv.load()
+    assert lib.fvattn_route_kernel_launches(None) == 0
+    for B, H in ((1, 40), (2, 40), (1, 1)):
+        assert fv.route_kernel_launches(fv.geom(B, H, 128, 21, 45, 80, 2, 8, 8)) == 3
