@@ -25,6 +25,8 @@
 //                  floor) is found the same way with counts when the Top-p
 //                  prefix is shorter.  No shared-memory atomics.  The kept
 //                  indices are written in ascending order with ballots.
+#include <cstring>
+
 #include "common.cuh"
 #include "ptx.cuh"
 #include "sync.cuh"
@@ -45,7 +47,7 @@ struct PoolOut {
 };
 
 template <int D>
-__global__ void __launch_bounds__(256, 3) pool_kernel(Geo g, const __nv_bfloat16* __restrict__ qt,
+__global__ void __launch_bounds__(256, 4) pool_kernel(Geo g, const __nv_bfloat16* __restrict__ qt,
                                                    const __nv_bfloat16* __restrict__ kt, PoolOut out) {
     constexpr int VPR = D / 8;             // 16-byte vectors per row
     constexpr int RPI = 32 / VPR;          // rows per warp instruction
@@ -145,8 +147,12 @@ __global__ void __launch_bounds__(256, 3) pool_kernel(Geo g, const __nv_bfloat16
 //               slice; a commit frees the stage, the tile's last commit hands
 //               the accumulator to the epilogue.
 //   warps 2-5   epilogue: each thread owns one query-block row of the tile
-//               (the warp's TMEM lane quarter), reads 32 columns at a time,
-//               scales and stores the real (row < nb, col < nb) logits.
+//               (the warp's TMEM lane quarter), reads 32 columns at a time
+//               and scales them.  When rows are 16-byte multiples (nb % 4 ==
+//               0) a warp stages its 32 x 32 block in shared memory (128-byte
+//               swizzle, two buffers) and writes it with one TMA store into
+//               the [B*H, nb, nb] logits, which clips rows and columns past
+//               nb; otherwise threads store their real logits directly.
 constexpr int SC_BM = 128;                 // query blocks per tile (MMA M)
 constexpr int SC_BN = 256;                 // key blocks per tile (MMA N)
 constexpr int SC_SLICE = 32;               // fp32 head-dim elements per stage (128 bytes)
@@ -156,6 +162,7 @@ constexpr uint32_t SC_A_BYTES = SC_BM * 128u;
 constexpr uint32_t SC_B_BYTES = SC_BN * 128u;
 constexpr uint32_t SC_STAGE_BYTES = 2u * SC_A_BYTES + 2u * SC_B_BYTES;
 constexpr uint32_t SC_TMEM_COLS = 2u * SC_BN;
+constexpr uint32_t SC_OUT_BYTES = 32u * 128u;   // one warp's 32 x 32 fp32 staging block
 
 struct ScoreCtrl {
     unsigned long long full[SC_STAGES];
@@ -167,7 +174,8 @@ struct ScoreCtrl {
     int abort_flag;
 };
 
-constexpr uint32_t SC_CTRL_OFF = SC_STAGES * SC_STAGE_BYTES;
+constexpr uint32_t SC_OUT_OFF = SC_STAGES * SC_STAGE_BYTES;            // 4 warps x 2 buffers
+constexpr uint32_t SC_CTRL_OFF = SC_OUT_OFF + 8u * SC_OUT_BYTES;
 constexpr uint32_t SC_SMEM = SC_CTRL_OFF + static_cast<uint32_t>(sizeof(ScoreCtrl));
 static_assert(SC_SMEM <= 232448u, "score kernel shared memory");
 
@@ -177,6 +185,7 @@ struct ScoreArgs {
     int nb;
     int m_tiles, n_tiles;
     int slices;            // D / 32
+    int tma_out;           // logits stored through t_out (nb % 4 == 0)
     long long tiles;       // B*H * m_tiles * n_tiles
 };
 
@@ -184,6 +193,7 @@ __global__ void __launch_bounds__(SC_THREADS, 1) score_kernel(const __grid_const
                                                               const __grid_constant__ CUtensorMap tq_lo,
                                                               const __grid_constant__ CUtensorMap tk_hi,
                                                               const __grid_constant__ CUtensorMap tk_lo,
+                                                              const __grid_constant__ CUtensorMap t_out,
                                                               ScoreArgs a) {
     extern __shared__ __align__(1024) unsigned char sc_smem[];
     ScoreCtrl& ctl = *reinterpret_cast<ScoreCtrl*>(sc_smem + SC_CTRL_OFF);
@@ -291,14 +301,18 @@ __global__ void __launch_bounds__(SC_THREADS, 1) score_kernel(const __grid_const
         const int quarter = warp & 3;
         const int r_in = quarter * 32 + lane;
         const bool vec_ok = (a.nb & 3) == 0;
+        const uint32_t stage0 = smem_u32(sc_smem + SC_OUT_OFF + static_cast<uint32_t>(quarter) * 2u * SC_OUT_BYTES);
+        if (lane == 0 && a.tma_out) prefetch_tmap(&t_out);
         long long tcount = 0;
+        int nstore = 0;
         for (long long t = blockIdx.x; t < a.tiles; t += gridDim.x, ++tcount) {
             const int b = static_cast<int>(tcount & 1);
             if (!wait_warp(smem_u32(&ctl.acc_full[b]), (tcount >> 1) & 1, abort_flag)) break;
             tc_fence_after();
             const long long bh = t / per_head;
-            const int rem = static_cast<int>(t - bh * per_head);
-            const int row = (rem / a.n_tiles) * SC_BM + r_in;
+            const int rem = static_cast<int>(t % per_head);
+            const int row0 = (rem / a.n_tiles) * SC_BM;
+            const int row = row0 + r_in;
             const int col0 = (rem % a.n_tiles) * SC_BN;
             float* out = a.L + (bh * a.nb + row) * static_cast<long long>(a.nb);
             const bool row_ok = row < a.nb;
@@ -308,7 +322,30 @@ __global__ void __launch_bounds__(SC_THREADS, 1) score_kernel(const __grid_const
                 uint32_t r[32];
                 tmem_ld32(tmem + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(b * SC_BN + c), r);
                 tmem_wait_ld();
-                if (row_ok && vec_ok && col + 32 <= a.nb) {
+                if (a.tma_out) {
+                    // swizzled staging: 16-byte chunk j of row `lane` at chunk j ^ (lane & 7)
+                    const uint32_t buf = stage0 + static_cast<uint32_t>(nstore & 1) * SC_OUT_BYTES;
+                    if (lane == 0) bulk_wait_group_read<1>();   // this buffer's previous store has read it
+                    __syncwarp();
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const uint32_t dst = buf + static_cast<uint32_t>(lane) * 128u +
+                                             static_cast<uint32_t>((j ^ (lane & 7)) * 16);
+                        asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(dst),
+                                     "f"(__uint_as_float(r[4 * j]) * a.scale),
+                                     "f"(__uint_as_float(r[4 * j + 1]) * a.scale),
+                                     "f"(__uint_as_float(r[4 * j + 2]) * a.scale),
+                                     "f"(__uint_as_float(r[4 * j + 3]) * a.scale)
+                                     : "memory");
+                    }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_store_3d(&t_out, buf, col, row0 + quarter * 32, static_cast<int>(bh));
+                        bulk_commit_group();
+                    }
+                    ++nstore;
+                } else if (row_ok && vec_ok && col + 32 <= a.nb) {
                     float4* o4 = reinterpret_cast<float4*>(out + col);
 #pragma unroll
                     for (int v = 0; v < 8; ++v)
@@ -324,6 +361,8 @@ __global__ void __launch_bounds__(SC_THREADS, 1) score_kernel(const __grid_const
             tc_fence_before();
             mbar_arrive(smem_u32(&ctl.acc_empty[b]));
         }
+        // logits stores complete before the kernel ends
+        if (lane == 0 && a.tma_out) bulk_wait_group_all();
     }
 
     // ---- teardown
@@ -658,6 +697,13 @@ extern "C" int fvattn_route(const fvattn_geom* gp, const void* q_tiled, const vo
     sa.m_tiles = (g.nb + SC_BM - 1) / SC_BM;
     sa.n_tiles = (g.nb + SC_BN - 1) / SC_BN;
     sa.slices = g.D / SC_SLICE;
+    sa.tma_out = (g.nb % 4) == 0;
+    CUtensorMap tout;
+    std::memset(&tout, 0, sizeof(tout));
+    if (sa.tma_out &&
+        !make_tmap_3d(&tout, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, L, static_cast<unsigned long long>(g.B) * g.H, g.nb,
+                      g.nb, 1, 32, 32))
+        return FVATTN_ERR_CUDA;
     sa.tiles = static_cast<long long>(g.B) * g.H * sa.m_tiles * sa.n_tiles;
     const int nsm = score_sms();
     if (nsm <= 0) return FVATTN_ERR_CUDA;
@@ -665,7 +711,7 @@ extern "C" int fvattn_route(const fvattn_geom* gp, const void* q_tiled, const vo
         cudaSuccess)
         return FVATTN_ERR_CUDA;
     const unsigned sgrid = static_cast<unsigned>(sa.tiles < nsm ? sa.tiles : nsm);
-    score_kernel<<<sgrid, SC_THREADS, SC_SMEM, s>>>(tqh, tql, tkh, tkl, sa);
+    score_kernel<<<sgrid, SC_THREADS, SC_SMEM, s>>>(tqh, tql, tkh, tkl, tout, sa);
     FV_CHECK_LAUNCH();
     const long long rows = static_cast<long long>(g.B) * g.H * g.nb;
     // entries per lane: the smallest instantiated count that covers a row

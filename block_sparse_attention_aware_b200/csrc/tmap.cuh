@@ -39,4 +39,21 @@ inline bool make_tmap_2d(CUtensorMap* m, CUtensorMapDataType dt, unsigned elem_b
     return r == CUDA_SUCCESS;
 }
 
+// Row-major [d2, d1, d0] matrix (d0 innermost), boxes of box2 x box1 x box0
+// elements with 128-byte swizzle (box0 * element size must be 128 bytes).
+// Coordinates past an extent are not written by stores and read as zero.
+inline bool make_tmap_3d(CUtensorMap* m, CUtensorMapDataType dt, unsigned elem_bytes, const void* base,
+                         unsigned long long d2, unsigned long long d1, unsigned long long d0, unsigned box2,
+                         unsigned box1, unsigned box0) {
+    PFN_encodeTiled enc = get_encode();
+    if (!enc) return false;
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(d0), static_cast<cuuint64_t>(d1), static_cast<cuuint64_t>(d2)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(d0) * elem_bytes, static_cast<cuuint64_t>(d0 * d1) * elem_bytes};
+    cuuint32_t box[3] = {static_cast<cuuint32_t>(box0), static_cast<cuuint32_t>(box1), static_cast<cuuint32_t>(box2)};
+    cuuint32_t estr[3] = {1u, 1u, 1u};
+    CUresult r = enc(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 }  // namespace fv
