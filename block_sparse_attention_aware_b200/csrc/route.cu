@@ -537,7 +537,7 @@ __device__ unsigned long long sel_boundary(const float (&v)[NPL], const float (&
 // is at most that of the later of the Top-p crossing (first prefix whose mass
 // reaches p * total) and the min(k, nb)-th entry.
 template <int NPL, bool KEEP_E>
-__global__ void __launch_bounds__(32 * SEL_WARPS, NPL <= 24 ? 3 : 1) select_kernel(int nb, long long rows, const float* __restrict__ L,
+__global__ void __launch_bounds__(32 * SEL_WARPS, NPL <= 24 ? 4 : 1) select_kernel(int nb, long long rows, const float* __restrict__ L,
                                                                 double p, int kfloor, int32_t* __restrict__ kv_idx,
                                                                 int32_t* __restrict__ kv_cnt) {
     __shared__ unsigned long long cand_keys[SEL_WARPS][32];
