@@ -24,6 +24,7 @@ import subprocess
 import sys
 import threading
 import time
+import types
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
@@ -34,6 +35,12 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 WORKLOAD = "720p"
 # kernels per step besides routing's: reorder x3, 2 work-list kernels, attention, inverse reorder
 OTHER_KERNELS_PER_STEP = 7
+
+# DRAM bytes (read + write) of one sparse_attn_kernel<128> launch on the 720p layer: an ncu capture
+# of the same layer restricted to 4 heads read 315.8 MB and wrote 73.9 MB; K/V reuse stays inside a
+# head, so traffic scales with the head count (x10 for 40 heads).
+ATTN_TRAFFIC_720P = {"bytes": (315.790080e6 + 73.944064e6) * 10,
+                     "how": "ncu dram__bytes_read.sum + dram__bytes_write.sum of the 4-head 720p layer, x10 heads"}
 
 
 def load_peaks():
@@ -53,7 +60,9 @@ def workload_config(w, g):
                     f"p={w.p}, k={w.k}",
         "global_batch": w.B, "seq_len": w.N, "heads": w.H, "head_dim": w.D,
         "block": f"{w.tf}x{w.th}x{w.tw}", "nb": g.nb, "p": w.p, "k_floor": w.k,
-        "l2": "no flush: every input tensor (774 MB raster, 865 MB tiled) is larger than the 126 MB L2",
+        "l2": (f"no flush: every input tensor ({w.B * w.N * w.H * w.D * 2 / 1e6:.0f} MB raster) is larger "
+               "than the 126 MB L2") if w.B * w.N * w.H * w.D * 2 > 126e6 else
+              "small layer: inputs fit in L2 (no flush; not a bandwidth measurement)",
         "parallelism": "replicas (independent layer per GPU)",
     }
 
@@ -112,7 +121,7 @@ class ClockSampler:
 
 # ---------------------------------------------------------------- CPU oracle (baseline / reference arm)
 
-def oracle_sample_time(w, qt, kt, vt, q_raster, kv_idx_full, kv_cnt_full, heads=4, items_per_head=12):
+def oracle_sample_time(w, qt, kt, vt, q_raster, kv_idx_full, kv_cnt_full, heads=8, items_per_head=16):
     """Time the oracle, as it stands, on a bounded sample of one layer and
     extrapolate to the whole layer.
 
@@ -188,7 +197,7 @@ def run_reference(args):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": t * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f64", "data": "synthetic (seeded, CPU generator)",
-        "config": {"workload": f"{w.name}-shaped layer", "global_batch": w.B, "seq_len": w.N},
+        "config": workload_config(w, types.SimpleNamespace(bs=geo["bs"], nb=geo["nb"])),
         "cpu_baseline": {"kind": "oracle", "value": val, "unit": "TFLOP/s", "cores": threads,
                          "sample": descs[-1]},
         "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -197,6 +206,66 @@ def run_reference(args):
 
 
 # ---------------------------------------------------------------- GPU arm
+
+def _imbalance(layer, nsm):
+    import numpy as np
+    st = layer.sm_stats.cpu().numpy().astype(np.float64)
+    busy = st[:nsm]
+    used = busy > 0
+    return float(busy[used].max() / busy[used].mean()) if used.any() else None
+
+
+def p_sweep(layer, w, g, nsm, stream):
+    """Route + attend at each p of the workload's sweep; per-head kept blocks
+    and the SM busy-time imbalance of the attention kernel."""
+    import torch
+    out = []
+    for p in w.p_sweep:
+        layer.p = p
+        layer.route()
+        layer.attend(stats=True)
+        e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+        e0.record(stream)
+        layer.route()
+        e1.record(stream)
+        layer.attend(stats=True)
+        e2.record(stream)
+        torch.cuda.synchronize()
+        cnt = layer.routed.kv_cnt
+        pairs = int(cnt.sum())
+        per_head = cnt.view(g.B * g.H, g.nb).sum(dim=1).cpu().tolist()
+        ms = e1.elapsed_time(e2)
+        out.append({"p": p, "density": pairs / float(g.B * g.H * g.nb * g.nb), "executed_block_pairs": pairs,
+                    "route_ms": e0.elapsed_time(e1), "attention_ms": ms,
+                    "attention_tflops": 4.0 * g.bs * g.bs * g.D * pairs / (ms / 1e3) / 1e12,
+                    "sm_imbalance_max_over_mean": _imbalance(layer, nsm),
+                    "head_blocks": per_head,
+                    "head_blocks_max_over_mean": max(per_head) / (sum(per_head) / len(per_head))})
+    return out
+
+
+def layer_stack(layer, w, g, dev, stream, barrier):
+    """Every seeded layer of the workload once: inputs drawn (untimed), then
+    one whole layer step timed with CUDA events; the stack time is the sum."""
+    import torch
+    from block_sparse_attention_aware_b200 import synth
+    per_layer, flops = [], 0.0
+    for li in range(w.layers):
+        q, k, v, _ = synth.make_qkv(w, layer=li, device=dev)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        layer(q, k, v)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        per_layer.append(e0.elapsed_time(e1))
+        flops += 4.0 * g.bs * g.bs * g.D * float(layer.routed.kv_cnt.sum())
+        del q, k, v
+    total = sum(per_layer)
+    return {"layers": w.layers, "total_ms": total, "per_layer_ms": per_layer,
+            "tflops_executed_blocks": flops / (total / 1e3) / 1e12,
+            "note": "each layer step timed alone (inputs of 40 layers do not fit in HBM together)"}
+
 
 def run_fvattn(args):
     import numpy as np
@@ -304,8 +373,11 @@ def run_fvattn(args):
         "ms_per_step": t_max / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16",
-        "data": f"synthetic: seeded Gaussian Wan2.2 720p-shaped Q/K/V (seed {w.seed}+rank), "
-                "per-head log-uniform Q scales, shared rank-8 spatio-temporal component",
+        "data": (f"synthetic: seeded Gaussian Wan2.2 {w.name}-shaped Q/K/V (seed {w.seed}+rank), "
+                 + {"loguniform": "per-head log-uniform Q scales in [0.25, 4]",
+                    "skew": "Q scale 4 on heads 0-19 and 0.25 on heads 20-39",
+                    "fixed": f"fixed per-head Q scales {list(w.qscale_values)}"}[w.qscale]
+                 + (", shared rank-8 spatio-temporal component" if w.lowrank else "")),
         "config": workload_config(w, g),
         "value_note": "executed-block attention FLOPs of all ranks / (max-over-ranks time of one whole "
                       "layer step: reorder x3 + route + attention + inverse reorder)",
@@ -322,13 +394,25 @@ def run_fvattn(args):
         "stages_gbs": {"reorder_qkv": reorder_gbs, "route": route_gbs, "inverse_reorder": inverse_gbs,
                        "route_pct_of_hbm": 100.0 * route_gbs / peaks["hbm_gbs"]},
         "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": sustained, "unit": "TFLOP/s",
-                     "frac": attn_tflops / sustained, "traffic": None,
+                     "frac": attn_tflops / sustained,
+                     "traffic": ATTN_TRAFFIC_720P["bytes"] if (w.name == "720p" and not args.heads) else None,
+                     "traffic_how": ATTN_TRAFFIC_720P["how"] if (w.name == "720p" and not args.heads) else None,
+                     "algorithmic_bytes_per_launch": 4 * tiled_bytes,
                      "kernel": "sparse_attn_kernel<128>",
                      "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside back-to-back steps)",
                      "algorithmic_flops_per_launch": flops},
         "gpu_launches": (OTHER_KERNELS_PER_STEP + fvattn.route_kernel_launches(g)) * args.steps,
         "clocks": clock_info,
     }
+
+    # p sweep (load-skew workload): per p, one routed + attended step after one warm-up
+    if w.p_sweep:
+        line["sweep"] = p_sweep(layer, w, g, nsm, stream)
+        layer.p = w.p
+
+    # full-depth stack: every seeded layer once (inputs drawn outside the timed region)
+    if w.layers > 1 and args.stack:
+        line["stack"] = layer_stack(layer, w, g, dev, stream, barrier)
 
     # end to end through the public API from pinned host buffers
     if args.e2e_steps > 0:
@@ -375,6 +459,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--workload", default=WORKLOAD, help="named workload of synth.WORKLOADS")
+    ap.add_argument("--stack", action="store_true",
+                    help="also time every seeded layer of a multi-layer workload once (cfg720p: 40 layers)")
     ap.add_argument("--heads", type=int, default=0,
                     help="profiling-size variant: the same layer with fewer heads (0 = all)")
     args = ap.parse_args()
