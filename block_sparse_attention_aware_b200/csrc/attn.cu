@@ -29,6 +29,12 @@
 //               K-major layout; O rescaled only when the row maximum grows by
 //               more than 2^8.  At the end of an item the groups swap (m, l)
 //               per row and each writes half of the output columns.
+// Query groups (bs < 128): one 128-row tile holds G = 128 / bs consecutive
+// query blocks (their rows are contiguous in the tiled layout), so the MMA
+// tile is never half empty.  The tile walks the union of the G kv lists in
+// ascending block order, from per-block membership bitmaps built by
+// group_bits_kernel; each chunk carries one key mask per query block of the
+// tile, so a row only sees the keys of its own block's list.
 // Every wait is bounded; a wait that runs out records FVATTN_ERR_TIMEOUT,
 // raises a CTA-wide abort flag and all roles leave their loops, so the CTA
 // always reaches the TMEM release.
@@ -53,11 +59,20 @@ constexpr uint32_t O_COL = 256;          // S_w at columns 128*w, O_w at 256 + 1
 // rescaled, when a new score exceeds it by more than this; until then
 // probabilities may reach 2^8, which bf16 P and fp32 sums hold exactly enough.
 constexpr float RESCALE_THRESHOLD = 8.0f;
+constexpr int MAX_GROUP = 8;             // query blocks per tile at bs = 16
 
 struct AttnArgs {
     Geo g;
     const int32_t* kv_idx;
     const int32_t* kv_cnt;
+    // Query groups: G = 128 / bs consecutive query blocks share one 128-row
+    // tile.  For G > 1 an item is (b*h, group) and walks the union of the
+    // group's kv lists, given as per-block membership bitmaps.
+    int G;                       // query blocks per tile (1 when bs = 128)
+    int ngroups;                 // ceil(nb / G)
+    int nwords;                  // 32-bit words per bitmap, ceil(nb / 32)
+    const uint32_t* gbits;       // [B*H][ngroups][G][nwords] (G > 1)
+    const int32_t* gcnt;         // [B*H][ngroups] union sizes (G > 1)
     const int32_t* head_order;   // [B*H] heads, heaviest first
     const int32_t* item_order;   // [B*H][nb] query blocks of each head, longest first
     int* counter;                // next item to hand out
@@ -77,8 +92,8 @@ struct __align__(16) Ctrl {
     unsigned long long mrg_full, mrg_empty;    // end-of-item exchange of (m, l)
     unsigned long long item_full[2], item_empty[2];
     unsigned long long blocks_done;
-    int item[2][4];              // bh, qb, cnt, valid
-    uint32_t mask[MAX_K_STAGES][4];  // key-validity bits of the chunk held by a K stage
+    int item[2][4];              // bh, first query block, cnt (kv blocks to walk), valid
+    uint32_t mask[MAX_K_STAGES][MAX_GROUP][4];  // per query block of the tile: its valid keys of a K stage's chunk
     uint32_t tmem_base;
     int abort_flag;
     float mrg_m[2][128];         // [group][row] running maximum (log2 units)
@@ -134,7 +149,60 @@ __device__ __forceinline__ int chunk_block(const int32_t* list, int cl, int bpc,
     return j;
 }
 
-template <int D>
+// Walk of the union of a query group's kv lists in ascending block order.
+// Lane t < G holds the current word of block t's membership bitmap; the
+// walk position (word index, bits left of the union word) is warp-uniform.
+struct UnionWalk {
+    const uint32_t* maps;   // [G][nwords]
+    int G, nwords, wi;
+    uint32_t word, rem;
+
+    __device__ __forceinline__ void init(const uint32_t* m, int groups, int nw) {
+        maps = m;
+        G = groups;
+        nwords = nw;
+        wi = -1;
+        word = 0u;
+        rem = 0u;
+    }
+    // Next union block j and its membership bits (bit t: in block t's list);
+    // false once the union is exhausted.  Warp-uniform.
+    __device__ __forceinline__ bool next(int lane, int& j, uint32_t& mem) {
+        while (rem == 0u) {
+            if (++wi >= nwords) return false;
+            word = lane < G ? __ldg(maps + lane * nwords + wi) : 0u;
+            rem = __reduce_or_sync(0xffffffffu, word);
+        }
+        const int bit = __ffs(static_cast<int>(rem)) - 1;
+        rem &= rem - 1u;
+        j = wi * 32 + bit;
+        mem = __ballot_sync(0xffffffffu, (word >> bit) & 1u);
+        return true;
+    }
+};
+
+// Slots of the next chunk of a group walk: lane s < (returned count) gets
+// slot s's block and membership bits.
+__device__ __forceinline__ int union_chunk(UnionWalk& u, int bpc, int lane, int& j, uint32_t& mem) {
+    int n = 0;
+    j = 0;
+    mem = 0u;
+    for (int s2 = 0; s2 < bpc; ++s2) {
+        int jj;
+        uint32_t mm;
+        if (!u.next(lane, jj, mm)) break;
+        if (lane == s2) {
+            j = jj;
+            mem = mm;
+        }
+        ++n;
+    }
+    return n;
+}
+
+// GRP: 128-row tiles of G = 128 / bs > 1 query blocks walking the union of
+// their kv lists (bs < 128); otherwise one query block per tile.
+template <int D, bool GRP>
 __global__ void __launch_bounds__(ATT_THREADS, 1)
     sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const AttnArgs a) {
@@ -238,11 +306,16 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                 }
                 break;
             }
-            const int hs = t / g.nb;
-            const int r = t - hs * g.nb;
+            const int G = GRP ? a.G : 1;
+            const int units = GRP ? a.ngroups : g.nb;
+            const int hs = t / units;
+            const int r = t - hs * units;
             const int bh = __ldg(a.head_order + hs);
-            const int qb = __ldg(a.item_order + static_cast<long long>(bh) * g.nb + r);
-            int cnt = __ldg(a.kv_cnt + static_cast<long long>(bh) * g.nb + qb);
+            const int u = __ldg(a.item_order + static_cast<long long>(bh) * units + r);
+            const int qb = u * G;                     // first query block of the tile
+            const int nq = min(G, g.nb - qb);         // query blocks in the tile
+            int cnt = GRP ? __ldg(a.gcnt + static_cast<long long>(bh) * a.ngroups + u)
+                          : __ldg(a.kv_cnt + static_cast<long long>(bh) * g.nb + qb);
             if (cnt < 1 || cnt > g.nb) {
                 if (lane == 0) record_status(FVATTN_ERR_BOUNDS);
                 cnt = cnt < 1 ? 1 : g.nb;
@@ -257,37 +330,78 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
             if (!wait_warp(smem_u32(&ctl.q_empty), (item_seq & 1) ^ 1, abort_flag)) break;
             const int row_base = bh * static_cast<int>(g.Npad);
             if (lane == 0) {
-                mbar_arrive_expect_tx(smem_u32(&ctl.q_full), static_cast<uint32_t>(bs * D * 2));
+                mbar_arrive_expect_tx(smem_u32(&ctl.q_full), static_cast<uint32_t>(nq * bs * D * 2));
+                for (int tq = 0; tq < (GRP ? nq : 1); ++tq)
 #pragma unroll
-                for (int h = 0; h < D / 64; ++h)
-                    tma_load_2d(sQ + h * 16384u, &tmQ, h * 64, row_base + qb * bs, smem_u32(&ctl.q_full));
+                    for (int h = 0; h < D / 64; ++h)
+                        tma_load_2d(sQ + h * 16384u + static_cast<uint32_t>(tq * bs) * 128u, &tmQ, h * 64,
+                                    row_base + (qb + tq) * bs, smem_u32(&ctl.q_full));
             }
             const int32_t* list = a.kv_idx + (static_cast<long long>(bh) * g.nb + qb) * g.nb;
+            UnionWalk uw;
+            if (GRP) uw.init(a.gbits + (static_cast<long long>(bh) * a.ngroups + u) * G * a.nwords, G, a.nwords);
             const int nc = (cnt + bpc - 1) / bpc;
-            int j_next = chunk_block(list, 0, bpc, min(bpc, cnt), lane, g.nb);
+            // chunk cl's blocks (lane s < nblk: slot s) and membership bits, one chunk ahead
+            int j_next = 0, n_next = 0;
+            uint32_t m_next = 0u;
+            if (GRP) {
+                n_next = union_chunk(uw, bpc, lane, j_next, m_next);
+            } else {
+                n_next = min(bpc, cnt);
+                j_next = chunk_block(list, 0, bpc, n_next, lane, g.nb);
+                m_next = 1u;
+            }
             for (int cl = 0; cl < nc; ++cl, ++c_seq) {
                 const int stage = c_seq % KS;
-                const int nblk = min(bpc, cnt - cl * bpc);
+                const int nblk = n_next;
                 const int j = j_next;
-                if (cl + 1 < nc) j_next = chunk_block(list, cl + 1, bpc, min(bpc, cnt - (cl + 1) * bpc), lane, g.nb);
+                const uint32_t mem = m_next;
+                if (cl + 1 < nc) {
+                    if (GRP) {
+                        n_next = union_chunk(uw, bpc, lane, j_next, m_next);
+                    } else {
+                        n_next = min(bpc, cnt - (cl + 1) * bpc);
+                        j_next = chunk_block(list, cl + 1, bpc, n_next, lane, g.nb);
+                    }
+                }
                 const int ext = lane < nblk ? block_extent(g, j) : 0;
                 if (!wait_warp(smem_u32(&ctl.k_empty[stage]), ((c_seq / KS) & 1) ^ 1, abort_flag)) {
                     ok = false;
                     break;
                 }
-                uint32_t words[4];
+                if (GRP) {
+                    // per query block t of the tile: key column real and its block in t's list
+                    for (int tq = 0; tq < G; ++tq) {
+                        uint32_t words[4];
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const int e = __shfl_sync(0xffffffffu, ext, c_slot[q]);
-                    const bool valid = (c_of[q] < (e & 255)) && (c_oy[q] < ((e >> 8) & 255)) && (c_ox[q] < (e >> 16));
-                    words[q] = __ballot_sync(0xffffffffu, valid);
+                        for (int q = 0; q < 4; ++q) {
+                            const int e = __shfl_sync(0xffffffffu, ext, c_slot[q]);
+                            const uint32_t mm = __shfl_sync(0xffffffffu, mem, c_slot[q]);
+                            const bool valid = (c_of[q] < (e & 255)) && (c_oy[q] < ((e >> 8) & 255)) &&
+                                               (c_ox[q] < (e >> 16)) && ((mm >> tq) & 1u);
+                            words[q] = __ballot_sync(0xffffffffu, valid);
+                        }
+                        if (lane == 0) {
+#pragma unroll
+                            for (int q = 0; q < 4; ++q) ctl.mask[stage][tq][q] = words[q];
+                        }
+                    }
+                } else {
+                    (void)mem;
+                    uint32_t words[4];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const int e = __shfl_sync(0xffffffffu, ext, c_slot[q]);
+                        const bool valid = (c_of[q] < (e & 255)) && (c_oy[q] < ((e >> 8) & 255)) && (c_ox[q] < (e >> 16));
+                        words[q] = __ballot_sync(0xffffffffu, valid);
+                    }
+                    if (lane == 0) {
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) ctl.mask[stage][0][q] = words[q];
+                    }
                 }
                 const uint32_t bar = smem_u32(&ctl.k_full[stage]);
-                if (lane == 0) {
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) ctl.mask[stage][q] = words[q];
-                    mbar_arrive_expect_tx(bar, static_cast<uint32_t>(nblk * bs * D * 2));
-                }
+                if (lane == 0) mbar_arrive_expect_tx(bar, static_cast<uint32_t>(nblk * bs * D * 2));
                 __syncwarp();
                 if (lane < nblk) {
                     const uint32_t kb = sK + stage * L::KV_BYTES + lane * bs * 128u;
@@ -313,14 +427,31 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
             if (lane == 0) mbar_arrive(smem_u32(&ctl.item_empty[slot]));
             if (!valid) break;
             const int row_base = bh * static_cast<int>(g.Npad);
+            const int G = GRP ? a.G : 1;
             const int32_t* list = a.kv_idx + (static_cast<long long>(bh) * g.nb + qb) * g.nb;
+            UnionWalk uw;
+            if (GRP) uw.init(a.gbits + (static_cast<long long>(bh) * a.ngroups + qb / G) * G * a.nwords, G, a.nwords);
             const int nc = (cnt + bpc - 1) / bpc;
-            int j_next = chunk_block(list, 0, bpc, min(bpc, cnt), lane, g.nb);
+            int j_next = 0, n_next = 0;
+            uint32_t m_unused = 0u;
+            if (GRP) {
+                n_next = union_chunk(uw, bpc, lane, j_next, m_unused);
+            } else {
+                n_next = min(bpc, cnt);
+                j_next = chunk_block(list, 0, bpc, n_next, lane, g.nb);
+            }
             for (int cl = 0; cl < nc; ++cl, ++c_seq) {
                 const int stage = c_seq % V_STAGES;
-                const int nblk = min(bpc, cnt - cl * bpc);
+                const int nblk = n_next;
                 const int j = j_next;
-                if (cl + 1 < nc) j_next = chunk_block(list, cl + 1, bpc, min(bpc, cnt - (cl + 1) * bpc), lane, g.nb);
+                if (cl + 1 < nc) {
+                    if (GRP) {
+                        n_next = union_chunk(uw, bpc, lane, j_next, m_unused);
+                    } else {
+                        n_next = min(bpc, cnt - (cl + 1) * bpc);
+                        j_next = chunk_block(list, cl + 1, bpc, n_next, lane, g.nb);
+                    }
+                }
                 if (!wait_warp(smem_u32(&ctl.v_empty[stage]), ((c_seq / V_STAGES) & 1) ^ 1, abort_flag)) {
                     ok = false;
                     break;
@@ -434,6 +565,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         const uint32_t sb = trow + static_cast<uint32_t>(w) * 128u;
         const uint32_t ob = trow + O_COL + static_cast<uint32_t>(w) * 128u;
         const uint32_t pbase = sP + static_cast<uint32_t>(w) * L::P_BYTES + static_cast<uint32_t>(row) * 128u;
+        const int tgrp = GRP ? row / bs : 0;   // this row's query block in the tile
         const float sl2 = a.scale_log2;
         int item_seq = 0;
         uint32_t c_seq = 0;
@@ -462,7 +594,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                     ok = false;
                     break;
                 }
-                const uint32_t* mrow = ctl.mask[kst];
+                const uint32_t* mrow = ctl.mask[kst][tgrp];
                 const uint32_t mw0 = mrow[0], mw1 = mrow[1], mw2 = mrow[2], mw3 = mrow[3];
                 const bool partial = (mw0 & mw1 & mw2 & mw3) != 0xFFFFFFFFu;   // chunk holds padding keys
                 tc_fence_after();
@@ -495,7 +627,8 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                                         fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * sl2;
                 const bool grow = mxs > m_ref + RESCALE_THRESHOLD;
                 const float m_new = grow ? mxs : m_ref;
-                const float alpha = ex2_approx(m_ref - m_new);
+                // (a row may see no key of its block in a chunk: max -inf, no growth, alpha 1)
+                const float alpha = grow ? ex2_approx(m_ref - m_new) : 1.0f;
                 const float neg = -m_new;
                 m_ref = m_new;
                 // P_w and O_w were last used by this group's previous PV
@@ -589,7 +722,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
             const bool use0 = __any_sync(0xffffffffu, l0 > 0.f), use1 = __any_sync(0xffffffffu, l1 > 0.f);
             tc_fence_after();
             __nv_bfloat16* orow = a.o + ((static_cast<long long>(bh) * g.Npad) + static_cast<long long>(qb) * bs + row) * D;
-            const bool store = row < bs;
+            const bool store = GRP ? row < min(a.G, g.nb - qb) * bs : row < bs;   // rows of real query blocks
             // this group writes output columns [w*D/2, w*D/2 + D/2)
 #pragma unroll 1
             for (int q = 0; q < D / 64; ++q) {
@@ -649,19 +782,69 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
 
 // ------------------------------------------------------------------ work list
 
-// One CTA per (b, h): order the head's query blocks by kv_cnt, longest first
-// (ties by lower block index), and record the head's total cost.
-__global__ void __launch_bounds__(256) worklist_head_kernel(Geo g, const int32_t* __restrict__ kv_cnt,
+// One warp per (b*h, query group) when G = 128 / bs > 1: membership bitmaps
+// of the group's G kv lists (bit j of map t: block j is in query block t's
+// list; order and repeats in a list do not matter) and the size of their
+// union, which is the number of kv blocks the group's tile walks.
+__global__ void __launch_bounds__(256) group_bits_kernel(Geo g, int G, int ngroups, int nwords,
+                                                         const int32_t* __restrict__ kv_idx,
+                                                         const int32_t* __restrict__ kv_cnt, uint32_t* __restrict__ gbits,
+                                                         int32_t* __restrict__ gcnt) {
+    extern __shared__ uint32_t gb_smem[];   // [8 warps][G * nwords]
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const long long unit = static_cast<long long>(blockIdx.x) * 8 + warp;
+    if (unit >= static_cast<long long>(g.B) * g.H * ngroups) return;
+    const int nb = g.nb;
+    const long long bh = unit / ngroups;
+    const int grp = static_cast<int>(unit - bh * ngroups);
+    uint32_t* bits = gb_smem + warp * G * nwords;
+    for (int i = lane; i < G * nwords; i += 32) bits[i] = 0u;
+    __syncwarp();
+    for (int t = 0; t < G; ++t) {
+        const int qb = grp * G + t;
+        if (qb >= nb) break;
+        int cnt = kv_cnt[bh * nb + qb];
+        if (cnt < 1 || cnt > nb) {
+            if (lane == 0) record_status(FVATTN_ERR_BOUNDS);
+            cnt = cnt < 1 ? 1 : nb;
+        }
+        const int32_t* list = kv_idx + (bh * nb + qb) * nb;
+        for (int e = lane; e < cnt; e += 32) {
+            int j = list[e];
+            if (j < 0 || j >= nb) {
+                record_status(FVATTN_ERR_BOUNDS);
+                j = 0;
+            }
+            atomicOr(&bits[t * nwords + (j >> 5)], 1u << (j & 31));
+        }
+    }
+    __syncwarp();
+    int un = 0;
+    for (int wd = lane; wd < nwords; wd += 32) {
+        uint32_t o = 0u;
+        for (int t = 0; t < G; ++t) o |= bits[t * nwords + wd];
+        un += __popc(o);
+    }
+    un = static_cast<int>(__reduce_add_sync(0xffffffffu, static_cast<unsigned int>(un)));
+    uint32_t* dst = gbits + unit * G * nwords;
+    for (int i = lane; i < G * nwords; i += 32) dst[i] = bits[i];
+    if (lane == 0) gcnt[unit] = un;
+}
+
+// One CTA per (b, h): order the head's `units` work units (query blocks, or
+// query groups when G > 1) by cost (kv blocks walked), longest first (ties by
+// lower index), and record the head's total cost.
+__global__ void __launch_bounds__(256) worklist_head_kernel(Geo g, int units, const int32_t* __restrict__ cost_in,
                                                             int32_t* __restrict__ item_order,
                                                             long long* __restrict__ head_cost) {
     extern __shared__ int wl_hist[];   // [nb + 2]
     const int nb = g.nb;
     const long long bh = blockIdx.x;
-    const int32_t* cnt = kv_cnt + bh * nb;
+    const int32_t* cnt = cost_in + bh * units;
     for (int i = threadIdx.x; i < nb + 2; i += blockDim.x) wl_hist[i] = 0;
     __syncthreads();
     long long part = 0;
-    for (int i = threadIdx.x; i < nb; i += blockDim.x) {
+    for (int i = threadIdx.x; i < units; i += blockDim.x) {
         int c = cnt[i];
         c = c < 1 ? 1 : (c > nb ? nb : c);
         atomicAdd(&wl_hist[c], 1);
@@ -676,18 +859,18 @@ __global__ void __launch_bounds__(256) worklist_head_kernel(Geo g, const int32_t
         long long tot = 0;
         for (int w = 0; w < (int)(blockDim.x >> 5); ++w) tot += red[w];
         head_cost[bh] = tot;
-        // descending exclusive scan: start[c] = #items with a larger count
+        // descending exclusive scan: start[c] = #units with a larger cost
         int run = 0;
         for (int c = nb; c >= 1; --c) {
             int h = wl_hist[c];
             wl_hist[c] = run;
             run += h;
         }
-        // stable placement in ascending block order
-        for (int i = 0; i < nb; ++i) {
+        // stable placement in ascending unit order
+        for (int i = 0; i < units; ++i) {
             int c = cnt[i];
             c = c < 1 ? 1 : (c > nb ? nb : c);
-            item_order[bh * nb + wl_hist[c]++] = i;
+            item_order[bh * units + wl_hist[c]++] = i;
         }
     }
 }
@@ -717,8 +900,11 @@ static bool make_tmap(CUtensorMap* m, const void* base, long long rows, int D, i
                         static_cast<unsigned long long>(D), 64u, static_cast<unsigned>(bs));
 }
 
+// Workspace: work list (item order, head cost and order, counter) and, when
+// G = 128 / bs > 1, the query groups' membership bitmaps and union sizes.
 struct WsLayout {
-    size_t item_order, head_cost, head_order, counter, total;
+    size_t item_order, head_cost, head_order, counter, gbits, gcnt, total;
+    int G, ngroups, nwords;
 };
 
 static size_t al256(size_t x) { return (x + 255) / 256 * 256; }
@@ -726,11 +912,20 @@ static size_t al256(size_t x) { return (x + 255) / 256 * 256; }
 static WsLayout ws_layout(const fvattn_geom& g) {
     WsLayout w;
     size_t BH = static_cast<size_t>(g.B) * g.H;
+    w.G = g.bs > 0 && g.bs < 128 ? 128 / g.bs : 1;
+    w.ngroups = (g.nb + w.G - 1) / w.G;
+    w.nwords = (g.nb + 31) / 32;
     w.item_order = 0;
     w.head_cost = al256(sizeof(int32_t) * BH * g.nb);
     w.head_order = w.head_cost + al256(sizeof(long long) * BH);
     w.counter = w.head_order + al256(sizeof(int32_t) * BH);
-    w.total = w.counter + 256;
+    w.gbits = w.counter + 256;
+    w.gcnt = w.gbits;
+    w.total = w.gbits;
+    if (w.G > 1) {
+        w.gcnt = w.gbits + al256(sizeof(uint32_t) * BH * w.ngroups * w.G * w.nwords);
+        w.total = w.gcnt + al256(sizeof(int32_t) * BH * w.ngroups);
+    }
     return w;
 }
 
@@ -743,14 +938,14 @@ static int cached_num_sms() {
 
 static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-template <int D>
+template <int D, bool GRP>
 static int launch_attn(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const AttnArgs& args,
                        int grid, cudaStream_t s) {
     using L = Smem<D>;
-    if (cudaFuncSetAttribute(sparse_attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(sparse_attn_kernel<D, GRP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(L::ALLOC)) != cudaSuccess)
         return FVATTN_ERR_CUDA;
-    sparse_attn_kernel<D><<<grid, ATT_THREADS, L::ALLOC, s>>>(tq, tk, tv, args);
+    sparse_attn_kernel<D, GRP><<<grid, ATT_THREADS, L::ALLOC, s>>>(tq, tk, tv, args);
     FV_CHECK_LAUNCH();
     return FVATTN_OK;
 }
@@ -789,9 +984,19 @@ extern "C" int fvattn_sparse_attn(const fvattn_geom* gp, const void* q_t, const 
     long long* head_cost = reinterpret_cast<long long*>(ws + wl.head_cost);
     int32_t* head_order = reinterpret_cast<int32_t*>(ws + wl.head_order);
     int* counter = reinterpret_cast<int*>(ws + wl.counter);
+    uint32_t* gbits = wl.G > 1 ? reinterpret_cast<uint32_t*>(ws + wl.gbits) : nullptr;
+    int32_t* gcnt = wl.G > 1 ? reinterpret_cast<int32_t*>(ws + wl.gcnt) : nullptr;
     const int BH = g.B * g.H;
+    const int units = wl.G > 1 ? wl.ngroups : g.nb;
 
-    worklist_head_kernel<<<BH, 256, sizeof(int) * (g.nb + 2), s>>>(g, kv_cnt, item_order, head_cost);
+    if (wl.G > 1) {
+        const long long warps = static_cast<long long>(BH) * wl.ngroups;
+        group_bits_kernel<<<static_cast<unsigned>((warps + 7) / 8), 256, sizeof(uint32_t) * 8 * wl.G * wl.nwords, s>>>(
+            g, wl.G, wl.ngroups, wl.nwords, kv_idx, kv_cnt, gbits, gcnt);
+        FV_CHECK_LAUNCH();
+    }
+    worklist_head_kernel<<<BH, 256, sizeof(int) * (g.nb + 2), s>>>(g, units, wl.G > 1 ? gcnt : kv_cnt, item_order,
+                                                                   head_cost);
     FV_CHECK_LAUNCH();
     worklist_heads_kernel<<<1, 256, 0, s>>>(BH, head_cost, head_order, counter);
     FV_CHECK_LAUNCH();
@@ -810,9 +1015,18 @@ extern "C" int fvattn_sparse_attn(const fvattn_geom* gp, const void* q_t, const 
     args.o = static_cast<__nv_bfloat16*>(o_t);
     args.sm_stats = sm_stats;
     args.scale_log2 = scale * 1.4426950408889634f;
-    args.total_items = BH * g.nb;
+    args.G = wl.G;
+    args.ngroups = wl.ngroups;
+    args.nwords = wl.nwords;
+    args.gbits = gbits;
+    args.gcnt = gcnt;
+    args.total_items = BH * units;
     int nsm = cached_num_sms();
     if (nsm <= 0) return FVATTN_ERR_CUDA;
     const int grid = nsm;
-    return g.D == 128 ? launch_attn<128>(tq, tk, tv, args, grid, s) : launch_attn<64>(tq, tk, tv, args, grid, s);
+    if (wl.G > 1)
+        return g.D == 128 ? launch_attn<128, true>(tq, tk, tv, args, grid, s)
+                          : launch_attn<64, true>(tq, tk, tv, args, grid, s);
+    return g.D == 128 ? launch_attn<128, false>(tq, tk, tv, args, grid, s)
+                      : launch_attn<64, false>(tq, tk, tv, args, grid, s);
 }

@@ -134,8 +134,9 @@ int fvattn_route(const fvattn_geom *g, const void *q_tiled, const void *k_tiled,
  * (pooling, scoring, selection); 0 for a null pointer. */
 int fvattn_route_kernel_launches(const fvattn_geom *g);
 
-/* Bytes of device workspace fvattn_sparse_attn needs (work list, head
- * order, per-block validity masks, work counter). */
+/* Bytes of device workspace fvattn_sparse_attn needs: the work list (item
+ * order, head cost and order, counter) and, for bs < 128, the query groups'
+ * kv-list membership bitmaps and union sizes. */
 size_t fvattn_attn_workspace_size(const fvattn_geom *g);
 
 /* Number of CTAs (one per SM) the persistent attention kernel launches on
@@ -150,7 +151,10 @@ int fvattn_num_sms(void);
  *         kv_cnt[b,h,i] blocks kv_idx[b,h,i,0..cnt)
  * computed with bf16 tensor-core products, fp32 online softmax and fp32
  * accumulation, written as bf16.  scale must be finite and > 0.  Work items
- * are taken longest-first by a persistent kernel with one CTA per SM.
+ * are taken longest-first by a persistent kernel with one CTA per SM.  For
+ * bs < 128 an item is a 128-row tile of 128 / bs consecutive query blocks
+ * that walks the union of their kv lists, each row masked to its own
+ * block's list (the order of a list does not matter).
  *   q_t, k_t, v_t  [B, H, Npad, D] bf16 from fvattn_reorder (padding zero)
  *   kv_idx, kv_cnt as written by fvattn_route (each row: cnt in [1, nb],
  *                  distinct indices in [0, nb)); out-of-range entries set
@@ -158,7 +162,7 @@ int fvattn_num_sms(void);
  *   o_t            [B, H, Npad, D] bf16 output (all rows written)
  *   sm_stats       optional (may be NULL) uint64[2 * fvattn_num_sms()]:
  *                  [0, n) busy nanoseconds of each CTA, [n, 2n) kv blocks
- *                  each CTA attended to
+ *                  each CTA walked (for bs < 128: union blocks per tile)
  *   workspace      >= fvattn_attn_workspace_size bytes, 256-byte aligned */
 int fvattn_sparse_attn(const fvattn_geom *g, const void *q_t, const void *k_t, const void *v_t,
                        const int32_t *kv_idx, const int32_t *kv_cnt, float scale,
