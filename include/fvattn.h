@@ -173,7 +173,7 @@ int fvattn_sparse_attn(const fvattn_geom *g, const void *q_t, const void *k_t, c
  * for fvattn_attn_workspace_size(g) of up to about 500 000 work items
  * (B*H*nb) at bs = 128 (e.g. B*H <= 200 at nb = 2560).  For bs < 128 the
  * query groups' bitmaps (about B*H*nb*ceil(nb/32)*4 bytes) count too: a
- * 40-head layer at bs = 64 fits up to nb = 576. */
+ * 40-head layer at bs = 64 fits up to nb = 608. */
 #define FVATTN_NOALLOC_SCRATCH_BYTES (2u * 1024u * 1024u)
 
 /* fvattn_sparse_attn without a workspace argument, for callers that cannot
