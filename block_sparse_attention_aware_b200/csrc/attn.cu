@@ -619,7 +619,9 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
 #pragma unroll
                     for (int hq = 0; hq < 2; ++hq)
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) mx[i & 7] = fmaxf(mx[i & 7], __uint_as_float(sr[hq][i]));
+                        for (int i = 0; i < 32; i += 2)
+                            mx[(i >> 1) & 7] = fmax3(mx[(i >> 1) & 7], __uint_as_float(sr[hq][i]),
+                                                     __uint_as_float(sr[hq][i + 1]));
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(smem_u32(&ctl.k_empty[kst]));   // mask consumed
@@ -651,9 +653,10 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                 }
                 // pass 2: P = 2^(s*scale*log2e - m), row sum, bf16 P row into
                 // P_w (128-byte swizzle, K-major operand); two TMEM loads in flight
-                float sm[8];
+                unsigned long long sm2[4];   // four chains of (even, odd) column sums
 #pragma unroll
-                for (int i = 0; i < 8; ++i) sm[i] = 0.f;
+                for (int i = 0; i < 4; ++i) sm2[i] = 0ull;
+                const unsigned long long sl2x2 = f2_pack(sl2, sl2), negx2 = f2_pack(neg, neg);
 #pragma unroll 1
                 for (int q2 = 0; q2 < 4; q2 += 2) {
                     uint32_t v[2][32];
@@ -667,14 +670,17 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                         uint32_t wv[16];
 #pragma unroll
                         for (int i = 0; i < 32; i += 2) {
-                            float p0 = ex2_approx(fmaf(__uint_as_float(v[hq][i]), sl2, neg));
-                            float p1 = ex2_approx(fmaf(__uint_as_float(v[hq][i + 1]), sl2, neg));
+                            float x0, x1;
+                            f2_unpack(f2_fma(f2_pack(__uint_as_float(v[hq][i]), __uint_as_float(v[hq][i + 1])), sl2x2,
+                                             negx2),
+                                      x0, x1);
+                            float p0 = ex2_approx(x0);
+                            float p1 = ex2_approx(x1);
                             if (partial) {
                                 p0 = ((mword >> i) & 1u) ? p0 : 0.f;
                                 p1 = ((mword >> (i + 1)) & 1u) ? p1 : 0.f;
                             }
-                            sm[i & 7] += p0;
-                            sm[(i + 1) & 7] += p1;
+                            sm2[(i >> 1) & 3] = f2_add(sm2[(i >> 1) & 3], f2_pack(p0, p1));
                             wv[i >> 1] = pack_bf16x2(p0, p1);
                         }
                         const int half = q >> 1;
@@ -691,6 +697,9 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(smem_u32(&ctl.s_free[w]));   // S_w consumed
+                float sm[8];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) f2_unpack(sm2[i], sm[2 * i], sm[2 * i + 1]);
                 const float sum = ((sm[0] + sm[1]) + (sm[2] + sm[3])) + ((sm[4] + sm[5]) + (sm[6] + sm[7]));
                 l = l * alpha + sum;
                 fence_proxy_async_smem();
