@@ -36,10 +36,10 @@ WORKLOAD = "720p"
 # kernels per step besides routing's: reorder x3, 2 work-list kernels, attention, inverse reorder
 OTHER_KERNELS_PER_STEP = 7
 
-# DRAM bytes (read + write) of one sparse_attn_kernel<128> launch on the 720p layer: an ncu capture
-# of the same layer restricted to 4 heads read 315.8 MB and wrote 73.9 MB; K/V reuse stays inside a
+# DRAM bytes (read + write) of one sparse_attn_kernel<128, 0> launch on the 720p layer: an ncu capture
+# of the same layer restricted to 4 heads read 342.1 MB and wrote 73.6 MB; K/V reuse stays inside a
 # head, so traffic scales with the head count (x10 for 40 heads).
-ATTN_TRAFFIC_720P = {"bytes": (315.790080e6 + 73.944064e6) * 10,
+ATTN_TRAFFIC_720P = {"bytes": (342.073088e6 + 73.583616e6) * 10,
                      "how": "ncu dram__bytes_read.sum + dram__bytes_write.sum of the 4-head 720p layer, x10 heads"}
 
 
@@ -398,7 +398,7 @@ def run_fvattn(args):
                      "traffic": ATTN_TRAFFIC_720P["bytes"] if (w.name == "720p" and not args.heads) else None,
                      "traffic_how": ATTN_TRAFFIC_720P["how"] if (w.name == "720p" and not args.heads) else None,
                      "algorithmic_bytes_per_launch": 4 * tiled_bytes,
-                     "kernel": "sparse_attn_kernel<128>",
+                     "kernel": f"sparse_attn_kernel<{g.D}, {int(g.bs < 128)}>",
                      "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside back-to-back steps)",
                      "algorithmic_flops_per_launch": flops},
         "gpu_launches": (OTHER_KERNELS_PER_STEP + fvattn.route_kernel_launches(g)) * args.steps,
