@@ -244,12 +244,17 @@ static int og_cmp_int(const void *pa, const void *pb) {
  *   c_r   = P_pi(1) + ... + P_pi(r), summed left to right       (double)
  *   m_p   = min { r : c_r >= p }   ("reaches p": inclusive)
  *           p >= 1 gives m_p = nb (floating sums may never reach 1)
+ *           p <= 0 gives m_p = 0: Top-p off, the fixed Top-k mode
  *   m     = max(m_p, min(k, nb))  (the union of two prefixes of pi is the
  *                                  longer prefix)
+ *   m    <- min(nb, m + k_extra)  (importance-order augmentation: the next
+ *                                  k_extra blocks of pi, this build's
+ *                                  single-GPU reading of the pages' slack
+ *                                  augmentation; k_extra = 0 leaves m)
  *   kept  = first m of pi, written out in ascending block index
  * Near-tie flag: set when c_{m_p} or c_{m_p - 1} is within `tie_band` of p.
  * Returns m; writes m_p and the flag. */
-static int og_select_row(const float *L, int nb, double p, int k, double tie_band,
+static int og_select_row(const float *L, int nb, double p, int k, int k_extra, double tie_band,
                          int *idx_out, int *mp_out, int *tie_out, og_entry *e, double *prob) {
     for (int j = 0; j < nb; ++j) { e[j].key = L[j]; e[j].idx = j; }
     qsort(e, (size_t)nb, sizeof(og_entry), og_cmp);
@@ -258,7 +263,9 @@ static int og_select_row(const float *L, int nb, double p, int k, double tie_ban
     for (int r = 0; r < nb; ++r) { prob[r] = exp((double)e[r].key - lmax); z += prob[r]; }
     for (int r = 0; r < nb; ++r) prob[r] /= z;
     int mp = nb, tie = 0;
-    if (p < 1.0) {
+    if (p <= 0.0) {
+        mp = 0;
+    } else if (p < 1.0) {
         double c = 0.0, c_prev = 0.0;
         mp = nb;
         for (int r = 0; r < nb; ++r) {
@@ -272,6 +279,7 @@ static int og_select_row(const float *L, int nb, double p, int k, double tie_ban
     }
     int kf = k < nb ? k : nb;
     int m = mp > kf ? mp : kf;
+    m = (k_extra > nb - m) ? nb : m + k_extra;
     for (int r = 0; r < m; ++r) idx_out[r] = e[r].idx;
     qsort(idx_out, (size_t)m, sizeof(int), og_cmp_int);
     *mp_out = mp;
@@ -282,8 +290,8 @@ static int og_select_row(const float *L, int nb, double p, int k, double tie_ban
 /* Exported: select on `rows` rows of fp32 logits [rows, nb].
  * idx: [rows, nb] (first cnt entries written, rest set to -1);
  * cnt, mp, tie: [rows]. */
-void oracle_select(const float *L, int rows, int nb, double p, int k, double tie_band,
-                   int *idx, int *cnt, int *mp, int *tie) {
+void oracle_select_aug(const float *L, int rows, int nb, double p, int k, int k_extra, double tie_band,
+                       int *idx, int *cnt, int *mp, int *tie) {
     #pragma omp parallel
     {
         og_entry *e = (og_entry *)malloc(sizeof(og_entry) * (size_t)nb);
@@ -292,12 +300,18 @@ void oracle_select(const float *L, int rows, int nb, double p, int k, double tie
         for (int r = 0; r < rows; ++r) {
             int *row_idx = idx + (long)r * nb;
             for (int j = 0; j < nb; ++j) row_idx[j] = -1;
-            cnt[r] = og_select_row(L + (long)r * nb, nb, p, k, tie_band, row_idx,
+            cnt[r] = og_select_row(L + (long)r * nb, nb, p, k, k_extra, tie_band, row_idx,
                                    &mp[r], &tie[r], e, prob);
         }
         free(e);
         free(prob);
     }
+}
+
+/* Exported: Top-p with the Top-k floor only (k_extra = 0). */
+void oracle_select(const float *L, int rows, int nb, double p, int k, double tie_band,
+                   int *idx, int *cnt, int *mp, int *tie) {
+    oracle_select_aug(L, rows, nb, p, k, 0, tie_band, idx, cnt, mp, tie);
 }
 
 /* ------------------------------------------------------------------ */

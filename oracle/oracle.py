@@ -50,6 +50,7 @@ def lib():
         L.oracle_pool.argtypes = [P, P] + geo
         L.oracle_logits.argtypes = [P, P, P, I, I, I, Dd]
         L.oracle_select.argtypes = [P, I, I, Dd, I, Dd, P, P, P, P]
+        L.oracle_select_aug.argtypes = [P, I, I, Dd, I, I, Dd, P, P, P, P]
         L.oracle_attention.argtypes = [P, P, P, P, P, P, I, Dd, P] + geo
         L.oracle_num_threads.restype = I
         L.oracle_set_num_threads.argtypes = [I]
@@ -128,8 +129,9 @@ def logits(qp: np.ndarray, kp: np.ndarray, scale: float) -> np.ndarray:
     return out
 
 
-def select(L: np.ndarray, p: float, k: int, tie_band: float = TIE_BAND):
-    """Top-p with Top-k floor on fp32 logits [..., nb].
+def select(L: np.ndarray, p: float, k: int, tie_band: float = TIE_BAND, k_extra: int = 0):
+    """Top-p with Top-k floor on fp32 logits [..., nb]; p = 0 is the fixed
+    Top-k mode and k_extra appends that many further blocks of the order.
 
     Returns (idx, cnt, m_p, near_tie): idx [..., nb] int32 with the kept
     block ids ascending in the first cnt entries and -1 after them.
@@ -141,8 +143,12 @@ def select(L: np.ndarray, p: float, k: int, tie_band: float = TIE_BAND):
     cnt = np.empty(L32.shape[:-1], dtype=np.int32)
     mp = np.empty(L32.shape[:-1], dtype=np.int32)
     tie = np.empty(L32.shape[:-1], dtype=np.int32)
-    lib().oracle_select(_ptr(L32), rows, nb, float(p), int(k), float(tie_band),
-                        _ptr(idx), _ptr(cnt), _ptr(mp), _ptr(tie))
+    if k_extra:
+        lib().oracle_select_aug(_ptr(L32), rows, nb, float(p), int(k), int(k_extra), float(tie_band),
+                                _ptr(idx), _ptr(cnt), _ptr(mp), _ptr(tie))
+    else:
+        lib().oracle_select(_ptr(L32), rows, nb, float(p), int(k), float(tie_band),
+                            _ptr(idx), _ptr(cnt), _ptr(mp), _ptr(tie))
     return idx, cnt, mp, tie
 
 

@@ -212,10 +212,12 @@ def _read_golden(name):
             line = line.split("#", 1)[0].strip()
             if not line:
                 continue
-            logit_s, p_s, k_s, kept_s = [s.strip() for s in line.split("|")]
+            fields = [s.strip() for s in line.split("|")]
+            logit_s, p_s, k_s, kept_s = fields[:4]
+            extra = int(fields[4]) if len(fields) > 4 else 0
             logits = [float(v) for v in logit_s.split()]
             kept = [int(v) for v in kept_s.split()]
-            cases.append((logits, float(p_s), int(k_s), kept))
+            cases.append((logits, float(p_s), int(k_s), kept, extra))
     return cases
 
 
@@ -224,7 +226,48 @@ def test_select_golden_hand_cases(orc):
     derivation)."""
     cases = _read_golden("select_hand_cases.txt")
     assert len(cases) >= 6
-    for logits, p, k, kept in cases:
-        idx, cnt, _, tie = orc.select(np.array([logits], dtype=np.float32), p, k)
+    assert sum(1 for c in cases if c[1] == 0.0) >= 3 and sum(1 for c in cases if c[4] > 0) >= 3
+    for logits, p, k, kept, extra in cases:
+        idx, cnt, _, tie = orc.select(np.array([logits], dtype=np.float32), p, k, k_extra=extra)
         assert tie[0] == 0
-        assert idx[0, :cnt[0]].tolist() == kept, (logits, p, k)
+        assert idx[0, :cnt[0]].tolist() == kept, (logits, p, k, extra)
+
+
+def _order(row):
+    """Block order by (logit descending, index ascending), from numpy's lexsort."""
+    return np.lexsort((np.arange(row.size), -row.astype(np.float64)))
+
+
+def test_fixed_topk_mode_matches_sorted_order(orc):
+    """p = 0: exactly min(k, nb) blocks, the first of the (logit desc, index
+    asc) order, including rows with repeated logits."""
+    rng = np.random.default_rng(11)
+    for nb in (1, 5, 37, 200):
+        L = rng.normal(size=(30, nb)).astype(np.float32)
+        L[::3, : nb // 2] = 0.5   # ties
+        for k in (1, 3, nb, nb + 4):
+            idx, cnt, mp, _ = orc.select(L, 0.0, k)
+            assert np.all(mp == 0)
+            assert np.all(cnt == min(k, nb))
+            for r in range(L.shape[0]):
+                want = np.sort(_order(L[r])[: min(k, nb)])
+                assert np.array_equal(idx[r, : cnt[r]], want)
+
+
+def test_augmentation_appends_the_next_blocks(orc):
+    """k_extra = e keeps min(nb, m + e) blocks, m the plain Top-p/Top-k count;
+    the added blocks are the next ones of the order, so sets are nested."""
+    rng = np.random.default_rng(12)
+    nb = 64
+    L = (rng.normal(size=(40, nb)) * rng.uniform(0.2, 5.0, size=(40, 1))).astype(np.float32)
+    base_idx, base_cnt, base_mp, _ = orc.select(L, 0.8, 3)
+    prev = [set(base_idx[r, : base_cnt[r]].tolist()) for r in range(L.shape[0])]
+    for e in (1, 2, 7, nb):
+        idx, cnt, mp, _ = orc.select(L, 0.8, 3, k_extra=e)
+        assert np.array_equal(mp, base_mp)
+        assert np.all(cnt == np.minimum(nb, base_cnt + e))
+        for r in range(L.shape[0]):
+            kept = set(idx[r, : cnt[r]].tolist())
+            assert prev[r] <= kept
+            assert kept == set(_order(L[r])[: cnt[r]].tolist())
+            prev[r] = kept
