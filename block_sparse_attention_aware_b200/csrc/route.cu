@@ -533,12 +533,13 @@ __device__ unsigned long long sel_boundary(const float (&v)[NPL], const float (&
     return order_key(tlo, found - 1);
 }
 
-// One warp per (b, h, query block) row.  Kept set: every entry whose order key
-// is at most that of the later of the Top-p crossing (first prefix whose mass
-// reaches p * total) and the min(k, nb)-th entry.
+// One warp per (b, h, query block) row.  Kept set: the first m entries of the
+// order, m = min(nb, max(m_p, min(k, nb)) + kextra), m_p the Top-p crossing
+// (first prefix whose mass reaches p * total; 0 when p = 0, nb when p >= 1).
 template <int NPL, bool KEEP_E>
 __global__ void __launch_bounds__(32 * SEL_WARPS, NPL <= 24 ? 4 : 1) select_kernel(int nb, long long rows, const float* __restrict__ L,
-                                                                double p, int kfloor, int32_t* __restrict__ kv_idx,
+                                                                double p, int kfloor, int kextra,
+                                                                int32_t* __restrict__ kv_idx,
                                                                 int32_t* __restrict__ kv_cnt) {
     __shared__ unsigned long long cand_keys[SEL_WARPS][32];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -569,13 +570,22 @@ __global__ void __launch_bounds__(32 * SEL_WARPS, NPL <= 24 ? 4 : 1) select_kern
         }
         unsigned long long s_all;
         int c_all;
-        sel_eval<NPL, KEEP_E>(v, e, lmax, lmin, true, s_all, c_all);
-        const double target = p * static_cast<double>(s_all);
-        int rank = 0;
-        thr = sel_boundary<NPL, KEEP_E>(v, e, nb, lmax, lmin, true, c_all, target, cand_keys[warp], &rank);
-        if (rank < kf)
-            thr = sel_boundary<NPL, KEEP_E>(v, e, nb, lmax, lmin, false, c_all, static_cast<double>(kf),
+        int rank = 0;   // m_p
+        if (p > 0.0) {
+            sel_eval<NPL, KEEP_E>(v, e, lmax, lmin, true, s_all, c_all);
+            const double target = p * static_cast<double>(s_all);
+            thr = sel_boundary<NPL, KEEP_E>(v, e, nb, lmax, lmin, true, c_all, target, cand_keys[warp], &rank);
+        } else {
+            sel_eval<NPL, KEEP_E>(v, e, lmax, lmin, false, s_all, c_all);
+        }
+        // floor and augmentation: the want-th entry of the order, if later
+        const long long want = min(static_cast<long long>(nb), static_cast<long long>(max(rank, kf)) + kextra);
+        if (want >= c_all) {
+            thr = ~0ull;
+        } else if (want > rank) {
+            thr = sel_boundary<NPL, KEEP_E>(v, e, nb, lmax, lmin, false, c_all, static_cast<double>(want),
                                             cand_keys[warp], &rank);
+        }
     }
     // emit the kept indices in ascending order
     const float tv = key_to_float(~static_cast<uint32_t>(thr >> 32));
@@ -595,10 +605,10 @@ __global__ void __launch_bounds__(32 * SEL_WARPS, NPL <= 24 ? 4 : 1) select_kern
 }
 
 template <int NPL, bool KEEP_E>
-static int launch_select(long long rows, int nb, const float* L, double p, int kfloor, int32_t* kv_idx,
+static int launch_select(long long rows, int nb, const float* L, double p, int kfloor, int kextra, int32_t* kv_idx,
                          int32_t* kv_cnt, cudaStream_t s) {
     const long long blocks = (rows + SEL_WARPS - 1) / SEL_WARPS;
-    select_kernel<NPL, KEEP_E><<<static_cast<unsigned>(blocks), 32 * SEL_WARPS, 0, s>>>(nb, rows, L, p, kfloor,
+    select_kernel<NPL, KEEP_E><<<static_cast<unsigned>(blocks), 32 * SEL_WARPS, 0, s>>>(nb, rows, L, p, kfloor, kextra,
                                                                                       kv_idx, kv_cnt);
     FV_CHECK_LAUNCH();
     return FVATTN_OK;
@@ -648,13 +658,13 @@ extern "C" int fvattn_route_kernel_launches(const fvattn_geom* gp) {
     return 3;   // pool, score, select
 }
 
-extern "C" int fvattn_route(const fvattn_geom* gp, const void* q_tiled, const void* k_tiled, double p, int k_floor,
-                            float scale, int32_t* kv_idx, int32_t* kv_cnt, float* q_pool, float* k_pool,
-                            float* logits, void* workspace, size_t ws_bytes, fvattn_stream_t stream) {
+static int route_impl(const fvattn_geom* gp, const void* q_tiled, const void* k_tiled, double p, int k_floor,
+                      int k_extra, float scale, int32_t* kv_idx, int32_t* kv_cnt, float* q_pool, float* k_pool,
+                      float* logits, void* workspace, size_t ws_bytes, fvattn_stream_t stream) {
     if (!gp || !q_tiled || !k_tiled || !kv_idx || !kv_cnt) return FVATTN_ERR_INVALID;
     if (!aligned16(q_tiled) || !aligned16(k_tiled) || !aligned16(kv_idx) || !aligned16(kv_cnt))
         return FVATTN_ERR_INVALID;
-    if (!(p > 0.0 && p <= 1.0) || k_floor < 1 || !isfinite(scale)) return FVATTN_ERR_INVALID;
+    if (!(p >= 0.0 && p <= 1.0) || k_floor < 1 || k_extra < 0 || !isfinite(scale)) return FVATTN_ERR_INVALID;
     if (gp->nb <= 0 || gp->nb > 2560) return FVATTN_ERR_UNSUPPORTED;
     if (gp->D != 64 && gp->D != 128) return FVATTN_ERR_UNSUPPORTED;
     const Geo g = to_geo(*gp);
@@ -716,15 +726,31 @@ extern "C" int fvattn_route(const fvattn_geom* gp, const void* q_tiled, const vo
     const long long rows = static_cast<long long>(g.B) * g.H * g.nb;
     // entries per lane: the smallest instantiated count that covers a row
     const int npl = (g.nb + 31) / 32;
-    if (npl <= 4) return launch_select<4, true>(rows, g.nb, L, p, k_floor, kv_idx, kv_cnt, s);
-    if (npl <= 8) return launch_select<8, true>(rows, g.nb, L, p, k_floor, kv_idx, kv_cnt, s);
-    if (npl <= 10) return launch_select<10, true>(rows, g.nb, L, p, k_floor, kv_idx, kv_cnt, s);
-    if (npl <= 12) return launch_select<12, true>(rows, g.nb, L, p, k_floor, kv_idx, kv_cnt, s);
-    if (npl <= 16) return launch_select<16, true>(rows, g.nb, L, p, k_floor, kv_idx, kv_cnt, s);
-    if (npl <= 21) return launch_select<21, true>(rows, g.nb, L, p, k_floor, kv_idx, kv_cnt, s);
-    if (npl <= 24) return launch_select<24, true>(rows, g.nb, L, p, k_floor, kv_idx, kv_cnt, s);
-    if (npl <= 32) return launch_select<32, true>(rows, g.nb, L, p, k_floor, kv_idx, kv_cnt, s);
-    if (npl <= 40) return launch_select<40, true>(rows, g.nb, L, p, k_floor, kv_idx, kv_cnt, s);
-    if (npl <= 48) return launch_select<48, true>(rows, g.nb, L, p, k_floor, kv_idx, kv_cnt, s);
-    return launch_select<80, false>(rows, g.nb, L, p, k_floor, kv_idx, kv_cnt, s);
+    if (npl <= 4) return launch_select<4, true>(rows, g.nb, L, p, k_floor, k_extra, kv_idx, kv_cnt, s);
+    if (npl <= 8) return launch_select<8, true>(rows, g.nb, L, p, k_floor, k_extra, kv_idx, kv_cnt, s);
+    if (npl <= 10) return launch_select<10, true>(rows, g.nb, L, p, k_floor, k_extra, kv_idx, kv_cnt, s);
+    if (npl <= 12) return launch_select<12, true>(rows, g.nb, L, p, k_floor, k_extra, kv_idx, kv_cnt, s);
+    if (npl <= 16) return launch_select<16, true>(rows, g.nb, L, p, k_floor, k_extra, kv_idx, kv_cnt, s);
+    if (npl <= 21) return launch_select<21, true>(rows, g.nb, L, p, k_floor, k_extra, kv_idx, kv_cnt, s);
+    if (npl <= 24) return launch_select<24, true>(rows, g.nb, L, p, k_floor, k_extra, kv_idx, kv_cnt, s);
+    if (npl <= 32) return launch_select<32, true>(rows, g.nb, L, p, k_floor, k_extra, kv_idx, kv_cnt, s);
+    if (npl <= 40) return launch_select<40, true>(rows, g.nb, L, p, k_floor, k_extra, kv_idx, kv_cnt, s);
+    if (npl <= 48) return launch_select<48, true>(rows, g.nb, L, p, k_floor, k_extra, kv_idx, kv_cnt, s);
+    return launch_select<80, false>(rows, g.nb, L, p, k_floor, k_extra, kv_idx, kv_cnt, s);
+}
+
+extern "C" int fvattn_route(const fvattn_geom* gp, const void* q_tiled, const void* k_tiled, double p, int k_floor,
+                            float scale, int32_t* kv_idx, int32_t* kv_cnt, float* q_pool, float* k_pool,
+                            float* logits, void* workspace, size_t ws_bytes, fvattn_stream_t stream) {
+    if (!(p > 0.0)) return FVATTN_ERR_INVALID;
+    return route_impl(gp, q_tiled, k_tiled, p, k_floor, 0, scale, kv_idx, kv_cnt, q_pool, k_pool, logits, workspace,
+                      ws_bytes, stream);
+}
+
+extern "C" int fvattn_route_aug(const fvattn_geom* gp, const void* q_tiled, const void* k_tiled, double p,
+                                int k_floor, int k_extra, float scale, int32_t* kv_idx, int32_t* kv_cnt,
+                                float* q_pool, float* k_pool, float* logits, void* workspace, size_t ws_bytes,
+                                fvattn_stream_t stream) {
+    return route_impl(gp, q_tiled, k_tiled, p, k_floor, k_extra, scale, kv_idx, kv_cnt, q_pool, k_pool, logits,
+                      workspace, ws_bytes, stream);
 }

@@ -21,7 +21,7 @@ _lib = None
 
 OK, ERR_INVALID, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_BOUNDS = range(6)
 EXPORTED = ("fvattn_geom_init", "fvattn_reorder", "fvattn_inverse_reorder",
-            "fvattn_route_workspace_size", "fvattn_route_kernel_launches", "fvattn_route",
+            "fvattn_route_workspace_size", "fvattn_route_kernel_launches", "fvattn_route", "fvattn_route_aug",
             "fvattn_attn_workspace_size",
             "fvattn_num_sms", "fvattn_sparse_attn", "fvattn_sparse_attn_noalloc", "fvattn_get_status",
             "fvattn_status_string")
@@ -64,6 +64,8 @@ def load(path: str = LIB_PATH):
     L.fvattn_route_kernel_launches.restype = I
     L.fvattn_route.argtypes = [G, P, P, ctypes.c_double, I, ctypes.c_float, P, P, P, P, P, P, S, P]
     L.fvattn_route.restype = I
+    L.fvattn_route_aug.argtypes = [G, P, P, ctypes.c_double, I, I, ctypes.c_float, P, P, P, P, P, P, S, P]
+    L.fvattn_route_aug.restype = I
     L.fvattn_attn_workspace_size.argtypes = [G]
     L.fvattn_attn_workspace_size.restype = S
     L.fvattn_num_sms.argtypes = []
@@ -170,8 +172,10 @@ def attn_workspace(g: Geom, device="cuda") -> torch.Tensor:
 
 def route(g: Geom, qt: torch.Tensor, kt: torch.Tensor, p: float, k: int,
           scale: Optional[float] = None, debug: bool = False, out: Optional[RouteOut] = None,
-          workspace: Optional[torch.Tensor] = None, stream=None) -> RouteOut:
-    """fvattn_route: pooled block scores -> Top-p (+ Top-k floor) kv lists."""
+          workspace: Optional[torch.Tensor] = None, stream=None, k_extra: int = 0) -> RouteOut:
+    """fvattn_route: pooled block scores -> Top-p (+ Top-k floor) kv lists.
+    p = 0 (fixed Top-k mode) or k_extra > 0 (augmentation) go through
+    fvattn_route_aug."""
     _need_cuda(qt, kt)
     dev = qt.device
     if scale is None:
@@ -185,11 +189,18 @@ def route(g: Geom, qt: torch.Tensor, kt: torch.Tensor, p: float, k: int,
             out.logits = torch.empty((g.B, g.H, g.nb, g.nb), dtype=torch.float32, device=dev)
     if workspace is None:
         workspace = route_workspace(g, dev)
-    rc = load().fvattn_route(ctypes.byref(g), _ptr(qt), _ptr(kt), float(p), int(k), float(scale),
-                             _ptr(out.kv_idx), _ptr(out.kv_cnt), _ptr(out.q_pool), _ptr(out.k_pool),
-                             _ptr(out.logits), _ptr(workspace),
-                             0 if workspace is None else workspace.numel(), _stream(stream))
-    _check("fvattn_route", rc)
+    if k_extra or p == 0:
+        rc = load().fvattn_route_aug(ctypes.byref(g), _ptr(qt), _ptr(kt), float(p), int(k), int(k_extra),
+                                     float(scale), _ptr(out.kv_idx), _ptr(out.kv_cnt), _ptr(out.q_pool),
+                                     _ptr(out.k_pool), _ptr(out.logits), _ptr(workspace),
+                                     0 if workspace is None else workspace.numel(), _stream(stream))
+        _check("fvattn_route_aug", rc)
+    else:
+        rc = load().fvattn_route(ctypes.byref(g), _ptr(qt), _ptr(kt), float(p), int(k), float(scale),
+                                 _ptr(out.kv_idx), _ptr(out.kv_cnt), _ptr(out.q_pool), _ptr(out.k_pool),
+                                 _ptr(out.logits), _ptr(workspace),
+                                 0 if workspace is None else workspace.numel(), _stream(stream))
+        _check("fvattn_route", rc)
     return out
 
 

@@ -130,6 +130,22 @@ int fvattn_route(const fvattn_geom *g, const void *q_tiled, const void *k_tiled,
                  float *q_pool, float *k_pool, float *logits,
                  void *workspace, size_t ws_bytes, fvattn_stream_t stream);
 
+/* Routing variants, this build's single-GPU readings of two passages
+ * (paperlayer.ai summary, section 2, "Sparse Attention": Top-k keeps a fixed
+ * number of blocks, against which Top-p is compared; section 3, "Slack-Aware
+ * Sparse Augmentation": extra high-value blocks taken in routing's
+ * importance order):
+ *   p = 0        fixed Top-k mode: m_p = 0, so m = min(k_floor, nb);
+ *   k_extra >= 0 importance-order augmentation: the next k_extra blocks of
+ *                the same order are kept too, m = min(nb, m + k_extra).
+ * p in [0, 1], k_floor >= 1, k_extra >= 0; otherwise as fvattn_route
+ * (fvattn_route is this call with k_extra = 0 and p > 0). */
+int fvattn_route_aug(const fvattn_geom *g, const void *q_tiled, const void *k_tiled,
+                     double p, int k_floor, int k_extra, float scale,
+                     int32_t *kv_idx, int32_t *kv_cnt,
+                     float *q_pool, float *k_pool, float *logits,
+                     void *workspace, size_t ws_bytes, fvattn_stream_t stream);
+
 /* Number of kernel launches one fvattn_route call makes for this geometry
  * (pooling, scoring, selection); 0 for a null pointer. */
 int fvattn_route_kernel_launches(const fvattn_geom *g);

@@ -27,7 +27,7 @@ def _declared():
 def test_exports_every_declared_symbol(fv):
     lib = fv.load()
     names = _declared()
-    assert len(names) == 12
+    assert len(names) == 13
     assert sorted(fv.EXPORTED) == names
     for n in names:
         assert hasattr(lib, n), n
@@ -67,6 +67,15 @@ def test_null_and_misaligned_pointers_rejected(fv):
                             ctypes.c_void_p(64), None, None, None, None, 0, None) == fv.ERR_INVALID
     assert lib.fvattn_route(gp, ctypes.c_void_p(16), ctypes.c_void_p(32), 1.5, 1, 0.125, ctypes.c_void_p(48),
                             ctypes.c_void_p(64), None, None, None, None, 0, None) == fv.ERR_INVALID
+    # routing variants: p in [0, 1], k_extra >= 0; plain routing needs p > 0
+    assert lib.fvattn_route(gp, ctypes.c_void_p(16), ctypes.c_void_p(32), 0.0, 1, 0.125, ctypes.c_void_p(48),
+                            ctypes.c_void_p(64), None, None, None, ctypes.c_void_p(256), 1 << 30, None) == fv.ERR_INVALID
+    assert lib.fvattn_route_aug(gp, ctypes.c_void_p(16), ctypes.c_void_p(32), 0.5, 1, -1, 0.125, ctypes.c_void_p(48),
+                                ctypes.c_void_p(64), None, None, None, ctypes.c_void_p(256), 1 << 30,
+                                None) == fv.ERR_INVALID
+    assert lib.fvattn_route_aug(gp, ctypes.c_void_p(16), ctypes.c_void_p(32), 1.5, 1, 0, 0.125, ctypes.c_void_p(48),
+                                ctypes.c_void_p(64), None, None, None, ctypes.c_void_p(256), 1 << 30,
+                                None) == fv.ERR_INVALID
     # workspace too small
     assert lib.fvattn_route(gp, ctypes.c_void_p(16), ctypes.c_void_p(32), 0.9, 1, 0.125, ctypes.c_void_p(48),
                             ctypes.c_void_p(64), None, None, None, ctypes.c_void_p(256), 16, None) == fv.ERR_INVALID

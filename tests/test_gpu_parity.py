@@ -43,11 +43,11 @@ def _gpu_inputs(w, device="cuda", layer=0):
     return q.contiguous(), k.contiguous(), v.contiguous()
 
 
-def _check_mask(orc, logits_gpu, kv_idx, kv_cnt, p, k):
+def _check_mask(orc, logits_gpu, kv_idx, kv_cnt, p, k, k_extra=0):
     """Oracle select on the GPU logits; returns (mismatched rows, near-tie rows)."""
     L = logits_gpu.cpu().numpy()
     nb = L.shape[-1]
-    idx_o, cnt_o, _, tie = orc.select(L.reshape(-1, nb), p, k)
+    idx_o, cnt_o, _, tie = orc.select(L.reshape(-1, nb), p, k, k_extra=k_extra)
     cnt_g = kv_cnt.cpu().numpy().reshape(-1)
     idx_g = kv_idx.cpu().numpy().reshape(-1, nb)
     bad = []
@@ -211,6 +211,34 @@ def test_attention_edge_routing(fv, orc, p, k):
     bad, unexcused, _ = _check_mask(orc, layer.routed.logits, layer.routed.kv_idx, layer.routed.kv_cnt, p, k)
     assert unexcused == []
     items = list(range(w.B * w.H * g.nb))
+    mx, mean = _attn_check(orc, w, g, layer.qt, layer.kt, layer.vt, layer.ot, layer.routed.kv_idx,
+                           layer.routed.kv_cnt, items, layer.scale)
+    assert mx <= MAX_ABS and mean <= MEAN_ABS, (mx, mean)
+
+
+@pytest.mark.parametrize("p,k,k_extra", [(0.0, 3, 0), (0.0, 1, 2), (0.7, 2, 3), (0.9, 1, 10_000)])
+def test_route_variants(fv, orc, p, k, k_extra):
+    """Fixed Top-k mode (p = 0) and importance-order augmentation (k_extra):
+    masks equal the oracle's on the GPU logits outside near ties, counts follow
+    min(nb, max(m_p, min(k, nb)) + k_extra), and attention runs on them."""
+    w = synth.custom_workload(B=1, H=3, D=128, F=3, Hs=24, Ws=32, tf=2, th=8, tw=8, seed=31, p=p, k=k,
+                              qscale="fixed", qscale_values=(0.5, 3.0, 9.0), lowrank=True)
+    g = fv.geom_of(w)
+    q, kk, v = _gpu_inputs(w)
+    layer = fv.Layer(g, p, k, debug=True)
+    layer.reorder_qkv(q, kk, v)
+    fv.route(g, layer.qt, layer.kt, p, k, layer.scale, out=layer.routed, workspace=layer.route_ws, k_extra=k_extra)
+    layer.attend()
+    torch.cuda.synchronize()
+    assert fv.get_status() == 0
+    bad, unexcused, _ = _check_mask(orc, layer.routed.logits, layer.routed.kv_idx, layer.routed.kv_cnt, p, k,
+                                    k_extra)
+    assert unexcused == []
+    cnt = layer.routed.kv_cnt.cpu().numpy().reshape(-1)
+    if p == 0.0:
+        assert np.all(cnt == min(g.nb, min(k, g.nb) + k_extra))
+    assert cnt.min() >= min(g.nb, min(k, g.nb) + k_extra)
+    items = list(range(0, w.B * w.H * g.nb, 3))
     mx, mean = _attn_check(orc, w, g, layer.qt, layer.kt, layer.vt, layer.ot, layer.routed.kv_idx,
                            layer.routed.kv_cnt, items, layer.scale)
     assert mx <= MAX_ABS and mean <= MEAN_ABS, (mx, mean)
