@@ -405,6 +405,16 @@ def run_fvattn(args):
         "clocks": clock_info,
     }
 
+    # the same step with the inverse reorder fused into the attention epilogue
+    ef0, ef1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    layer(q, k, v, fused_inverse=True)
+    ef0.record(stream)
+    for _ in range(args.steps):
+        layer(q, k, v, fused_inverse=True)
+    ef1.record(stream)
+    torch.cuda.synchronize()
+    line["fused_inverse_step_ms"] = ef0.elapsed_time(ef1) / args.steps
+
     # p sweep (load-skew workload): per p, one routed + attended step after one warm-up
     if w.p_sweep:
         line["sweep"] = p_sweep(layer, w, g, nsm, stream)

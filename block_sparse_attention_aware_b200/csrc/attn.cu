@@ -76,7 +76,8 @@ struct AttnArgs {
     const int32_t* head_order;   // [B*H] heads, heaviest first
     const int32_t* item_order;   // [B*H][nb] query blocks of each head, longest first
     int* counter;                // next item to hand out
-    __nv_bfloat16* o;            // [B, H, Npad, D]
+    __nv_bfloat16* o;            // [B, H, Npad, D], or [B, N, H, D] when raster
+    int raster;                  // write O rows straight to the raster layout (real tokens only)
     unsigned long long* sm_stats;
     float scale_log2;            // scale * log2(e), > 0
     int total_items;
@@ -730,8 +731,21 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
             const float f0 = a0 * inv, f1 = a1 * inv;
             const bool use0 = __any_sync(0xffffffffu, l0 > 0.f), use1 = __any_sync(0xffffffffu, l1 > 0.f);
             tc_fence_after();
-            __nv_bfloat16* orow = a.o + ((static_cast<long long>(bh) * g.Npad) + static_cast<long long>(qb) * bs + row) * D;
-            const bool store = GRP ? row < min(a.G, g.nb - qb) * bs : row < bs;   // rows of real query blocks
+            const bool in_tile = GRP ? row < min(a.G, g.nb - qb) * bs : row < bs;   // rows of real query blocks
+            __nv_bfloat16* orow;
+            bool store;
+            if (a.raster) {
+                // the inverse reorder fused in: tile row -> raster token (b, n, h), padding rows dropped
+                int tf_, ty_, tx_;
+                const bool real = in_tile && token_of_pos(g, static_cast<long long>(qb) * bs + row, tf_, ty_, tx_);
+                const long long b_ = bh / g.H, h_ = bh - b_ * g.H;
+                const long long n_ = real ? (static_cast<long long>(tf_) * g.Hs + ty_) * g.Ws + tx_ : 0;
+                orow = a.o + ((b_ * g.N + n_) * g.H + h_) * D;
+                store = real;
+            } else {
+                orow = a.o + ((static_cast<long long>(bh) * g.Npad) + static_cast<long long>(qb) * bs + row) * D;
+                store = in_tile;
+            }
             // this group writes output columns [w*D/2, w*D/2 + D/2)
 #pragma unroll 1
             for (int q = 0; q < D / 64; ++q) {
@@ -970,10 +984,9 @@ extern "C" size_t fvattn_attn_workspace_size(const fvattn_geom* gp) {
 
 extern "C" int fvattn_num_sms(void) { return cached_num_sms(); }
 
-extern "C" int fvattn_sparse_attn(const fvattn_geom* gp, const void* q_t, const void* k_t, const void* v_t,
-                                  const int32_t* kv_idx, const int32_t* kv_cnt, float scale, void* o_t,
-                                  unsigned long long* sm_stats, void* workspace, size_t ws_bytes,
-                                  fvattn_stream_t stream) {
+static int attn_impl(const fvattn_geom* gp, const void* q_t, const void* k_t, const void* v_t, const int32_t* kv_idx,
+                     const int32_t* kv_cnt, float scale, void* o_t, int raster, unsigned long long* sm_stats,
+                     void* workspace, size_t ws_bytes, fvattn_stream_t stream) {
     if (!gp || !q_t || !k_t || !v_t || !kv_idx || !kv_cnt || !o_t || !workspace) return FVATTN_ERR_INVALID;
     if (!aligned16(q_t) || !aligned16(k_t) || !aligned16(v_t) || !aligned16(o_t) || !aligned16(kv_idx) ||
         !aligned16(kv_cnt) || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
@@ -1022,6 +1035,7 @@ extern "C" int fvattn_sparse_attn(const fvattn_geom* gp, const void* q_t, const 
     args.item_order = item_order;
     args.counter = counter;
     args.o = static_cast<__nv_bfloat16*>(o_t);
+    args.raster = raster;
     args.sm_stats = sm_stats;
     args.scale_log2 = scale * 1.4426950408889634f;
     args.G = wl.G;
@@ -1038,4 +1052,18 @@ extern "C" int fvattn_sparse_attn(const fvattn_geom* gp, const void* q_t, const 
                           : launch_attn<64, true>(tq, tk, tv, args, grid, s);
     return g.D == 128 ? launch_attn<128, false>(tq, tk, tv, args, grid, s)
                       : launch_attn<64, false>(tq, tk, tv, args, grid, s);
+}
+
+extern "C" int fvattn_sparse_attn(const fvattn_geom* gp, const void* q_t, const void* k_t, const void* v_t,
+                                  const int32_t* kv_idx, const int32_t* kv_cnt, float scale, void* o_t,
+                                  unsigned long long* sm_stats, void* workspace, size_t ws_bytes,
+                                  fvattn_stream_t stream) {
+    return attn_impl(gp, q_t, k_t, v_t, kv_idx, kv_cnt, scale, o_t, 0, sm_stats, workspace, ws_bytes, stream);
+}
+
+extern "C" int fvattn_sparse_attn_raster(const fvattn_geom* gp, const void* q_t, const void* k_t, const void* v_t,
+                                         const int32_t* kv_idx, const int32_t* kv_cnt, float scale, void* o,
+                                         unsigned long long* sm_stats, void* workspace, size_t ws_bytes,
+                                         fvattn_stream_t stream) {
+    return attn_impl(gp, q_t, k_t, v_t, kv_idx, kv_cnt, scale, o, 1, sm_stats, workspace, ws_bytes, stream);
 }

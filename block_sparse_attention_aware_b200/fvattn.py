@@ -23,7 +23,8 @@ OK, ERR_INVALID, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_BOUNDS = range(6)
 EXPORTED = ("fvattn_geom_init", "fvattn_reorder", "fvattn_inverse_reorder",
             "fvattn_route_workspace_size", "fvattn_route_kernel_launches", "fvattn_route", "fvattn_route_aug",
             "fvattn_attn_workspace_size",
-            "fvattn_num_sms", "fvattn_sparse_attn", "fvattn_sparse_attn_noalloc", "fvattn_get_status",
+            "fvattn_num_sms", "fvattn_sparse_attn", "fvattn_sparse_attn_raster", "fvattn_sparse_attn_noalloc",
+            "fvattn_get_status",
             "fvattn_status_string")
 
 
@@ -72,6 +73,8 @@ def load(path: str = LIB_PATH):
     L.fvattn_num_sms.restype = I
     L.fvattn_sparse_attn.argtypes = [G, P, P, P, P, P, ctypes.c_float, P, P, P, S, P]
     L.fvattn_sparse_attn.restype = I
+    L.fvattn_sparse_attn_raster.argtypes = [G, P, P, P, P, P, ctypes.c_float, P, P, P, S, P]
+    L.fvattn_sparse_attn_raster.restype = I
     L.fvattn_sparse_attn_noalloc.argtypes = [G, P, P, P, P, P, ctypes.c_float, P, P, P]
     L.fvattn_sparse_attn_noalloc.restype = I
     L.fvattn_get_status.argtypes = [P]
@@ -228,6 +231,27 @@ def sparse_attn(g: Geom, qt, kt, vt, kv_idx, kv_cnt, scale: Optional[float] = No
 NOALLOC_SCRATCH_BYTES = 2 * 1024 * 1024
 
 
+
+def sparse_attn_raster(g: Geom, qt, kt, vt, kv_idx, kv_cnt, scale: Optional[float] = None,
+                       out: Optional[torch.Tensor] = None, sm_stats: Optional[torch.Tensor] = None,
+                       workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """fvattn_sparse_attn_raster: sparse attention writing O in the raster
+    [B, N, H, D] layout (the inverse reorder fused into the epilogue)."""
+    _need_cuda(qt, kt, vt, kv_idx, kv_cnt, out, sm_stats)
+    if scale is None:
+        scale = 1.0 / math.sqrt(g.D)
+    if out is None:
+        out = torch.empty((g.B, g.N, g.H, g.D), dtype=torch.bfloat16, device=qt.device)
+    if workspace is None:
+        workspace = attn_workspace(g, qt.device)
+    if sm_stats is not None:
+        assert sm_stats.dtype == torch.int64 and sm_stats.numel() >= 2 * num_sms()
+    rc = load().fvattn_sparse_attn_raster(ctypes.byref(g), _ptr(qt), _ptr(kt), _ptr(vt), _ptr(kv_idx),
+                                          _ptr(kv_cnt), float(scale), _ptr(out), _ptr(sm_stats),
+                                          _ptr(workspace), workspace.numel(), _stream(stream))
+    _check("fvattn_sparse_attn_raster", rc)
+    return out
+
 def sparse_attn_noalloc(g: Geom, qt, kt, vt, kv_idx, kv_cnt, scale: Optional[float] = None,
                         out: Optional[torch.Tensor] = None, sm_stats: Optional[torch.Tensor] = None,
                         stream=None) -> torch.Tensor:
@@ -291,9 +315,17 @@ class Layer:
     def restore(self, stream=None):
         return inverse_reorder(self.g, self.ot, self.o, stream)
 
-    def __call__(self, q, k, v, stats: bool = False, stream=None):
+    def attend_raster(self, stats: bool = False, stream=None):
+        """Sparse attention with the inverse reorder fused in: O straight to self.o."""
+        return sparse_attn_raster(self.g, self.qt, self.kt, self.vt, self.routed.kv_idx, self.routed.kv_cnt,
+                                  self.scale, out=self.o, sm_stats=self.sm_stats if stats else None,
+                                  workspace=self.attn_ws, stream=stream)
+
+    def __call__(self, q, k, v, stats: bool = False, stream=None, fused_inverse: bool = False):
         self.reorder_qkv(q, k, v, stream)
         self.route(stream)
+        if fused_inverse:
+            return self.attend_raster(stats, stream)
         self.attend(stats, stream)
         return self.restore(stream)
 

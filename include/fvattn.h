@@ -185,6 +185,21 @@ int fvattn_sparse_attn(const fvattn_geom *g, const void *q_t, const void *k_t, c
                        void *o_t, unsigned long long *sm_stats,
                        void *workspace, size_t ws_bytes, fvattn_stream_t stream);
 
+/* fvattn_sparse_attn with the inverse reorder fused into its epilogue
+ * (paperlayer.ai summary, section 3, "Pipeline": attention, then
+ * restoration of the original layout): each output row goes straight to its
+ * raster position, and padding rows are not written.
+ *   o  [B, N, H, D] bf16, the same bits fvattn_sparse_attn followed by
+ *      fvattn_inverse_reorder would write.
+ * Other arguments and errors as fvattn_sparse_attn.  It needs no tiled O
+ * buffer (865 MB at the 720p layer); on B200 its scattered raster stores make
+ * the attention step about 3% slower than fvattn_sparse_attn plus
+ * fvattn_inverse_reorder. */
+int fvattn_sparse_attn_raster(const fvattn_geom *g, const void *q_t, const void *k_t, const void *v_t,
+                              const int32_t *kv_idx, const int32_t *kv_cnt, float scale,
+                              void *o, unsigned long long *sm_stats,
+                              void *workspace, size_t ws_bytes, fvattn_stream_t stream);
+
 /* Maximum scratch, in bytes, of fvattn_sparse_attn_noalloc (2 MiB): enough
  * for fvattn_attn_workspace_size(g) of up to about 500 000 work items
  * (B*H*nb) at bs = 128 (e.g. B*H <= 200 at nb = 2560).  For bs < 128 the

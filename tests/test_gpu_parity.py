@@ -216,6 +216,23 @@ def test_attention_edge_routing(fv, orc, p, k):
     assert mx <= MAX_ABS and mean <= MEAN_ABS, (mx, mean)
 
 
+@pytest.mark.parametrize("name,w", SMALL, ids=[s[0] for s in SMALL])
+def test_fused_inverse_reorder_bit_exact(fv, name, w):
+    """fvattn_sparse_attn_raster writes the same bits as fvattn_sparse_attn
+    followed by fvattn_inverse_reorder (every item is computed the same way
+    whichever CTA takes it)."""
+    g = fv.geom_of(w)
+    q, k, v = _gpu_inputs(w)
+    layer = fv.Layer(g, w.p, w.k)
+    want = layer(q, k, v).clone()
+    got = torch.full_like(want, float("nan"))
+    fv.sparse_attn_raster(g, layer.qt, layer.kt, layer.vt, layer.routed.kv_idx, layer.routed.kv_cnt,
+                          layer.scale, out=got, workspace=layer.attn_ws)
+    torch.cuda.synchronize()
+    assert fv.get_status() == 0
+    assert torch.equal(got.view(torch.int16), want.view(torch.int16))
+
+
 @pytest.mark.parametrize("p,k,k_extra", [(0.0, 3, 0), (0.0, 1, 2), (0.7, 2, 3), (0.9, 1, 10_000)])
 def test_route_variants(fv, orc, p, k, k_extra):
     """Fixed Top-k mode (p = 0) and importance-order augmentation (k_extra):
