@@ -156,22 +156,24 @@ __device__ __forceinline__ int chunk_block(const int32_t* list, int cl, int bpc,
 struct UnionWalk {
     const uint32_t* maps;   // [G][nwords]
     int G, nwords, wi;
-    uint32_t word, rem;
+    uint32_t word, rem, ahead;   // ahead: lane t's word wi + 1, loaded one word early
 
-    __device__ __forceinline__ void init(const uint32_t* m, int groups, int nw) {
+    __device__ __forceinline__ void init(const uint32_t* m, int groups, int nw, int lane) {
         maps = m;
         G = groups;
         nwords = nw;
         wi = -1;
         word = 0u;
         rem = 0u;
+        ahead = lane < G ? __ldg(maps + lane * nwords) : 0u;
     }
     // Next union block j and its membership bits (bit t: in block t's list);
     // false once the union is exhausted.  Warp-uniform.
     __device__ __forceinline__ bool next(int lane, int& j, uint32_t& mem) {
         while (rem == 0u) {
             if (++wi >= nwords) return false;
-            word = lane < G ? __ldg(maps + lane * nwords + wi) : 0u;
+            word = ahead;
+            ahead = (lane < G && wi + 1 < nwords) ? __ldg(maps + lane * nwords + wi + 1) : 0u;
             rem = __reduce_or_sync(0xffffffffu, word);
         }
         const int bit = __ffs(static_cast<int>(rem)) - 1;
@@ -340,7 +342,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
             }
             const int32_t* list = a.kv_idx + (static_cast<long long>(bh) * g.nb + qb) * g.nb;
             UnionWalk uw;
-            if (GRP) uw.init(a.gbits + (static_cast<long long>(bh) * a.ngroups + u) * G * a.nwords, G, a.nwords);
+            if (GRP) uw.init(a.gbits + (static_cast<long long>(bh) * a.ngroups + u) * G * a.nwords, G, a.nwords, lane);
             const int nc = (cnt + bpc - 1) / bpc;
             // chunk cl's blocks (lane s < nblk: slot s) and membership bits, one chunk ahead
             int j_next = 0, n_next = 0;
@@ -431,7 +433,8 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
             const int G = GRP ? a.G : 1;
             const int32_t* list = a.kv_idx + (static_cast<long long>(bh) * g.nb + qb) * g.nb;
             UnionWalk uw;
-            if (GRP) uw.init(a.gbits + (static_cast<long long>(bh) * a.ngroups + qb / G) * G * a.nwords, G, a.nwords);
+            if (GRP) uw.init(a.gbits + (static_cast<long long>(bh) * a.ngroups + qb / G) * G * a.nwords, G, a.nwords,
+                             lane);
             const int nc = (cnt + bpc - 1) / bpc;
             int j_next = 0, n_next = 0;
             uint32_t m_unused = 0u;
