@@ -40,6 +40,8 @@
 // always reaches the TMEM release.
 #include <cuda.h>
 
+#include <type_traits>
+
 #include "common.cuh"
 #include "ptx.cuh"
 #include "sync.cuh"
@@ -57,8 +59,9 @@ constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t O_COL = 256;          // S_w at columns 128*w, O_w at 256 + 128*w
 // Lazy rescaling: the running row maximum (log2 units) is only moved, and O
 // rescaled, when a new score exceeds it by more than this; until then
-// probabilities may reach 2^8, which bf16 P and fp32 sums hold exactly enough.
-constexpr float RESCALE_THRESHOLD = 8.0f;
+// probabilities may reach 2^32, which bf16 P (8-bit exponent) and fp32 sums
+// and accumulators hold with their usual relative precision.
+constexpr float RESCALE_THRESHOLD = 32.0f;
 constexpr int MAX_GROUP = 8;             // query blocks per tile at bs = 16
 
 struct AttnArgs {
@@ -600,49 +603,67 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                 }
                 const uint32_t* mrow = ctl.mask[kst][tgrp];
                 const uint32_t mw0 = mrow[0], mw1 = mrow[1], mw2 = mrow[2], mw3 = mrow[3];
-                const bool partial = (mw0 & mw1 & mw2 & mw3) != 0xFFFFFFFFu;   // chunk holds padding keys
+                const bool partial = (mw0 & mw1 & mw2 & mw3) != 0xFFFFFFFFu;   // chunk holds masked keys
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(&ctl.k_empty[kst]));   // mask in registers: stage free
                 tc_fence_after();
-                // pass 1: row maximum of the raw scores, eight independent chains
+                // Exp pass: P = 2^(s*scale*log2e + negv), row sum on fp32 pairs, bf16 P row into P_w
+                // (128-byte swizzle, K-major operand), two TMEM loads in flight; with TRACK it also
+                // takes the row maximum of the (masked) raw scores.
+                unsigned long long sm2[4];   // four chains of (even, odd) column sums
                 float mx[8];
+                auto exp_pass = [&](auto track, float negv) {
+                    constexpr bool TRACK = decltype(track)::value;
 #pragma unroll
-                for (int i = 0; i < 8; ++i) mx[i] = -INFINITY;
+                    for (int i = 0; i < 4; ++i) sm2[i] = 0ull;
+                    if (TRACK) {
 #pragma unroll
-                for (int q2 = 0; q2 < 4; q2 += 2) {
-                    uint32_t sr[2][32];
-                    tmem_ld32(sb + q2 * 32u, sr[0]);
-                    tmem_ld32(sb + q2 * 32u + 32u, sr[1]);
-                    tmem_wait_ld();
-                    if (partial) {
-                        const uint32_t mwa = q2 == 0 ? mw0 : mw2, mwb = q2 == 0 ? mw1 : mw3;
+                        for (int i = 0; i < 8; ++i) mx[i] = -INFINITY;
+                    }
+                    const unsigned long long sl2x2 = f2_pack(sl2, sl2), negx2 = f2_pack(negv, negv);
+#pragma unroll 1
+                    for (int q2 = 0; q2 < 4; q2 += 2) {
+                        uint32_t v[2][32];
+                        tmem_ld32(sb + q2 * 32u, v[0]);
+                        tmem_ld32(sb + q2 * 32u + 32u, v[1]);
+                        tmem_wait_ld();
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) {
-                            if (!((mwa >> i) & 1u)) sr[0][i] = 0xFF800000u;
-                            if (!((mwb >> i) & 1u)) sr[1][i] = 0xFF800000u;
+                        for (int hq = 0; hq < 2; ++hq) {
+                            const int q = q2 + hq;
+                            const uint32_t mword = q == 0 ? mw0 : (q == 1 ? mw1 : (q == 2 ? mw2 : mw3));
+                            uint32_t wv[16];
+#pragma unroll
+                            for (int i = 0; i < 32; i += 2) {
+                                const float s0 = __uint_as_float(v[hq][i]), s1 = __uint_as_float(v[hq][i + 1]);
+                                float x0, x1;
+                                f2_unpack(f2_fma(f2_pack(s0, s1), sl2x2, negx2), x0, x1);
+                                float p0 = ex2_approx(x0);
+                                float p1 = ex2_approx(x1);
+                                if (partial) {
+                                    const bool k0 = (mword >> i) & 1u, k1 = (mword >> (i + 1)) & 1u;
+                                    p0 = k0 ? p0 : 0.f;
+                                    p1 = k1 ? p1 : 0.f;
+                                    if (TRACK)
+                                        mx[(i >> 1) & 7] = fmax3(mx[(i >> 1) & 7], k0 ? s0 : -INFINITY, k1 ? s1 : -INFINITY);
+                                } else if (TRACK) {
+                                    mx[(i >> 1) & 7] = fmax3(mx[(i >> 1) & 7], s0, s1);
+                                }
+                                sm2[(i >> 1) & 3] = f2_add(sm2[(i >> 1) & 3], f2_pack(p0, p1));
+                                wv[i >> 1] = pack_bf16x2(p0, p1);
+                            }
+                            const int half = q >> 1;
+#pragma unroll
+                            for (int k4 = 0; k4 < 4; ++k4) {
+                                const int chunk = (((q & 1) << 2) | k4) ^ (row & 7);
+                                const uint32_t addr = pbase + half * 16384u + chunk * 16u;
+                                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(wv[4 * k4]),
+                                             "r"(wv[4 * k4 + 1]), "r"(wv[4 * k4 + 2]), "r"(wv[4 * k4 + 3])
+                                             : "memory");
+                            }
                         }
                     }
-#pragma unroll
-                    for (int hq = 0; hq < 2; ++hq)
-#pragma unroll
-                        for (int i = 0; i < 32; i += 2)
-                            mx[(i >> 1) & 7] = fmax3(mx[(i >> 1) & 7], __uint_as_float(sr[hq][i]),
-                                                     __uint_as_float(sr[hq][i + 1]));
-                }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(smem_u32(&ctl.k_empty[kst]));   // mask consumed
-                const float mxs = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                                        fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * sl2;
-                const bool grow = mxs > m_ref + RESCALE_THRESHOLD;
-                const float m_new = grow ? mxs : m_ref;
-                // (a row may see no key of its block in a chunk: max -inf, no growth, alpha 1)
-                const float alpha = grow ? ex2_approx(m_ref - m_new) : 1.0f;
-                const float neg = -m_new;
-                m_ref = m_new;
-                // P_w and O_w were last used by this group's previous PV
-                if (!wait_warp(smem_u32(&ctl.p_free[w]), (n & 1) ^ 1, abort_flag)) {
-                    ok = false;
-                    break;
-                }
-                if (mine_any && __any_sync(0xffffffffu, grow)) {
+                };
+                auto rescale_o = [&](float alpha) {
                     tc_fence_after();
 #pragma unroll 1
                     for (int q = 0; q < D / 32; ++q) {
@@ -654,48 +675,60 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                         tmem_st32(ob + q * 32u, o);
                     }
                     tmem_wait_st();
-                }
-                // pass 2: P = 2^(s*scale*log2e - m), row sum, bf16 P row into
-                // P_w (128-byte swizzle, K-major operand); two TMEM loads in flight
-                unsigned long long sm2[4];   // four chains of (even, odd) column sums
+                };
+                float alpha = 1.0f;
+                if (!mine_any) {
+                    // the group's first chunk of the item: row maximum first, then P against it
 #pragma unroll
-                for (int i = 0; i < 4; ++i) sm2[i] = 0ull;
-                const unsigned long long sl2x2 = f2_pack(sl2, sl2), negx2 = f2_pack(neg, neg);
-#pragma unroll 1
-                for (int q2 = 0; q2 < 4; q2 += 2) {
-                    uint32_t v[2][32];
-                    tmem_ld32(sb + q2 * 32u, v[0]);
-                    tmem_ld32(sb + q2 * 32u + 32u, v[1]);
-                    tmem_wait_ld();
+                    for (int i = 0; i < 8; ++i) mx[i] = -INFINITY;
 #pragma unroll
-                    for (int hq = 0; hq < 2; ++hq) {
-                        const int q = q2 + hq;
-                        const uint32_t mword = q == 0 ? mw0 : (q == 1 ? mw1 : (q == 2 ? mw2 : mw3));
-                        uint32_t wv[16];
+                    for (int q2 = 0; q2 < 4; q2 += 2) {
+                        uint32_t sr[2][32];
+                        tmem_ld32(sb + q2 * 32u, sr[0]);
+                        tmem_ld32(sb + q2 * 32u + 32u, sr[1]);
+                        tmem_wait_ld();
+                        if (partial) {
+                            const uint32_t mwa = q2 == 0 ? mw0 : mw2, mwb = q2 == 0 ? mw1 : mw3;
 #pragma unroll
-                        for (int i = 0; i < 32; i += 2) {
-                            float x0, x1;
-                            f2_unpack(f2_fma(f2_pack(__uint_as_float(v[hq][i]), __uint_as_float(v[hq][i + 1])), sl2x2,
-                                             negx2),
-                                      x0, x1);
-                            float p0 = ex2_approx(x0);
-                            float p1 = ex2_approx(x1);
-                            if (partial) {
-                                p0 = ((mword >> i) & 1u) ? p0 : 0.f;
-                                p1 = ((mword >> (i + 1)) & 1u) ? p1 : 0.f;
+                            for (int i = 0; i < 32; ++i) {
+                                if (!((mwa >> i) & 1u)) sr[0][i] = 0xFF800000u;
+                                if (!((mwb >> i) & 1u)) sr[1][i] = 0xFF800000u;
                             }
-                            sm2[(i >> 1) & 3] = f2_add(sm2[(i >> 1) & 3], f2_pack(p0, p1));
-                            wv[i >> 1] = pack_bf16x2(p0, p1);
                         }
-                        const int half = q >> 1;
 #pragma unroll
-                        for (int k4 = 0; k4 < 4; ++k4) {
-                            const int chunk = (((q & 1) << 2) | k4) ^ (row & 7);
-                            const uint32_t addr = pbase + half * 16384u + chunk * 16u;
-                            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(wv[4 * k4]),
-                                         "r"(wv[4 * k4 + 1]), "r"(wv[4 * k4 + 2]), "r"(wv[4 * k4 + 3])
-                                         : "memory");
-                        }
+                        for (int hq = 0; hq < 2; ++hq)
+#pragma unroll
+                            for (int i = 0; i < 32; i += 2)
+                                mx[(i >> 1) & 7] = fmax3(mx[(i >> 1) & 7], __uint_as_float(sr[hq][i]),
+                                                         __uint_as_float(sr[hq][i + 1]));
+                    }
+                    // (a row may see no key of its block in a chunk: it keeps max -inf, P 0)
+                    m_ref = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                                  fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * sl2;
+                    // P_w was last used by this group's previous PV
+                    if (!wait_warp(smem_u32(&ctl.p_free[w]), (n & 1) ^ 1, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    exp_pass(std::false_type{}, -m_ref);
+                } else {
+                    // later chunks: one pass against the running reference maximum, which is only
+                    // moved (and O rescaled, and the chunk redone) when a row maximum exceeds it by
+                    // more than 2^RESCALE_THRESHOLD; until then P stays below 2^RESCALE_THRESHOLD
+                    if (!wait_warp(smem_u32(&ctl.p_free[w]), (n & 1) ^ 1, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    exp_pass(std::true_type{}, -m_ref);
+                    const float mxs = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                                            fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * sl2;
+                    const bool grow = mxs > m_ref + RESCALE_THRESHOLD;
+                    if (__any_sync(0xffffffffu, grow)) {
+                        const float m_new = grow ? mxs : m_ref;
+                        alpha = grow ? ex2_approx(m_ref - m_new) : 1.0f;
+                        m_ref = m_new;
+                        rescale_o(alpha);
+                        exp_pass(std::false_type{}, -m_ref);
                     }
                 }
                 tc_fence_before();
