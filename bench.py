@@ -205,6 +205,23 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+# ---------------------------------------------------------------- ranks
+
+def aggregate_over_ranks(t_local: float, work_local: float, world: int, device):
+    """Whole-job figures of a replicated step: the slowest rank's time (the
+    job finishes when it does) and the work of all ranks.  Every rank calls
+    this with its own values; with one rank it returns them unchanged."""
+    import torch
+    if world <= 1:
+        return float(t_local), float(work_local)
+    import torch.distributed as dist
+    t = torch.tensor([t_local], dtype=torch.float64, device=device)
+    wk = torch.tensor([work_local], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dist.all_reduce(wk, op=dist.ReduceOp.SUM)
+    return float(t.item()), float(wk.item())
+
+
 # ---------------------------------------------------------------- GPU arm
 
 def _imbalance(layer, nsm):
@@ -330,16 +347,10 @@ def run_fvattn(args):
     status = fvattn.get_status()
     assert status == 0, f"device status {status}"
     t_total = start.elapsed_time(end) / 1e3
-    t_max = torch.tensor([t_total], dtype=torch.float64, device=dev)
     cnt = layer.routed.kv_cnt
     pairs = int(cnt.sum())
     flops = 4.0 * g.bs * g.bs * g.D * pairs
-    flops_t = torch.tensor([flops], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t_max, op=dist.ReduceOp.MAX)
-        dist.all_reduce(flops_t, op=dist.ReduceOp.SUM)
-    t_max = float(t_max.item())
-    flops_all = float(flops_t.item())
+    t_max, flops_all = aggregate_over_ranks(t_total, flops, world, dev)
 
     stage = {n: [] for n in ("reorder_qkv", "route", "attention", "inverse_reorder")}
     for e in ev:
@@ -440,10 +451,8 @@ def run_fvattn(args):
             fvattn.attention_from_host(layer, qh, kh, vh, oh)
         s1.record(stream)
         torch.cuda.synchronize()
-        te = torch.tensor([s0.elapsed_time(s1) / 1e3], dtype=torch.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(te, op=dist.ReduceOp.MAX)
-        te = float(te.item()) / args.e2e_steps
+        te, _ = aggregate_over_ranks(s0.elapsed_time(s1) / 1e3, 0.0, world, dev)
+        te /= args.e2e_steps
         line["e2e"] = {"value": flops_all / te / 1e12, "unit": "TFLOP/s", "ms_per_step": te * 1e3,
                        "h2d_bytes_per_step": 3 * raster_bytes, "d2h_bytes_per_step": raster_bytes,
                        "steps": args.e2e_steps}
