@@ -58,6 +58,7 @@ class Workload:
     lowrank_rank: int = 8
     layers: int = 1
     p_sweep: tuple = ()
+    order: str = "raster"          # block order: "raster" tile order or "hilbert"
 
     @property
     def N(self) -> int:

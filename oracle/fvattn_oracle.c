@@ -48,6 +48,9 @@ typedef struct {
     int nbf, nby, nbx;                   /* tiles along frame, row, col */
     int bs, nb;                          /* tokens per block, blocks */
     long N, Npad;                        /* raster tokens, padded tokens */
+    int order;                           /* 0: raster tile order, 1: Hilbert */
+    int *tile_of_block;                  /* order 1: raster tile index of block b */
+    int *block_of_tile;                  /* order 1: block index of raster tile t */
 } og_geom;
 
 static int ceil_div(int a, int b) { return (a + b - 1) / b; }
@@ -66,6 +69,94 @@ static void og_make(og_geom *g, int B, int H, int D, int F, int Hs, int Ws,
     g->nb = g->nbf * g->nby * g->nbx;
     g->N = (long)F * Hs * Ws;
     g->Npad = (long)g->nb * g->bs;
+    g->order = 0;
+    g->tile_of_block = NULL;
+    g->block_of_tile = NULL;
+}
+
+/* Index of cell (c[0], c[1], c[2]) along the 3-D Hilbert curve that fills a
+ * cube of side 2^bits, after J. Skilling, "Programming the Hilbert curve"
+ * (AIP Conf. Proc. 707, 2004): the coordinates are turned into the curve's
+ * "transposed" index (an inverse-undo sweep from the top bit down, then Gray
+ * encoding), whose bits, read top bit first and coordinate 0 first within a
+ * bit, are the index. */
+static unsigned long long og_hilbert3(const unsigned c_in[3], int bits) {
+    unsigned c[3] = {c_in[0], c_in[1], c_in[2]};
+    const unsigned top = 1u << (bits - 1);
+    for (unsigned q = top; q > 1u; q >>= 1) {
+        const unsigned low = q - 1u;
+        for (int i = 0; i < 3; ++i) {
+            if (c[i] & q) {
+                c[0] ^= low;                       /* invert the low bits */
+            } else {
+                const unsigned t = (c[0] ^ c[i]) & low;   /* exchange low bits with c[0] */
+                c[0] ^= t;
+                c[i] ^= t;
+            }
+        }
+    }
+    for (int i = 1; i < 3; ++i) c[i] ^= c[i - 1];   /* Gray encode */
+    unsigned t = 0;
+    for (unsigned q = top; q > 1u; q >>= 1)
+        if (c[2] & q) t ^= q - 1u;
+    for (int i = 0; i < 3; ++i) c[i] ^= t;
+    unsigned long long h = 0;
+    for (int b = bits - 1; b >= 0; --b)
+        for (int i = 0; i < 3; ++i) h = (h << 1) | ((c[i] >> b) & 1u);
+    return h;
+}
+
+typedef struct { unsigned long long key; int tile; } og_hkey;
+
+static int og_cmp_hkey(const void *pa, const void *pb) {
+    const og_hkey *a = (const og_hkey *)pa, *b = (const og_hkey *)pb;
+    return (a->key > b->key) - (a->key < b->key);
+}
+
+/* Hilbert block order (paperlayer.ai summary, section 3, "Sparse-routing
+ * frontend": Hilbert-curve block reordering keeps spatially adjacent tokens
+ * in nearby blocks).  Reading taken: the tile grid (frame, row, col) =
+ * (nbf, nby, nbx) sits in the smallest cube of side 2^bits that holds it,
+ * and blocks are numbered by increasing curve index of their tile.  Tokens
+ * inside a tile keep raster order. */
+static void og_block_order(int nbf, int nby, int nbx, int *tile_of_block, int *block_of_tile) {
+    const int nb = nbf * nby * nbx;
+    int side = nbf > nby ? nbf : nby;
+    if (nbx > side) side = nbx;
+    int bits = 1;
+    while ((1 << bits) < side) ++bits;
+    og_hkey *k = (og_hkey *)malloc(sizeof(og_hkey) * (size_t)nb);
+    for (int t = 0; t < nb; ++t) {
+        const unsigned c[3] = {(unsigned)(t / (nby * nbx)), (unsigned)((t / nbx) % nby), (unsigned)(t % nbx)};
+        k[t].key = og_hilbert3(c, bits);
+        k[t].tile = t;
+    }
+    qsort(k, (size_t)nb, sizeof(og_hkey), og_cmp_hkey);
+    for (int b = 0; b < nb; ++b) {
+        tile_of_block[b] = k[b].tile;
+        if (block_of_tile) block_of_tile[k[b].tile] = b;
+    }
+    free(k);
+}
+
+static void og_set_order(og_geom *g, int order) {
+    g->order = order;
+    if (order == 1) {
+        g->tile_of_block = (int *)malloc(sizeof(int) * (size_t)g->nb);
+        g->block_of_tile = (int *)malloc(sizeof(int) * (size_t)g->nb);
+        og_block_order(g->nbf, g->nby, g->nbx, g->tile_of_block, g->block_of_tile);
+    }
+}
+
+static void og_free(og_geom *g) {
+    free(g->tile_of_block);
+    free(g->block_of_tile);
+    g->tile_of_block = g->block_of_tile = NULL;
+}
+
+/* Exported: the Hilbert block order of a tile grid, tile_of_block[nb]. */
+void oracle_block_order(int nbf, int nby, int nbx, int *tile_of_block) {
+    og_block_order(nbf, nby, nbx, tile_of_block, NULL);
 }
 
 /* Video-aware block organisation (paperlayer.ai summary, section 3,
@@ -76,6 +167,7 @@ static void og_make(og_geom *g, int B, int H, int D, int F, int Hs, int Ws,
  * block * bs + offset. */
 static long og_tiled_pos(const og_geom *g, int f, int y, int x) {
     long block = ((long)(f / g->tf) * g->nby + (y / g->th)) * g->nbx + (x / g->tw);
+    if (g->order == 1) block = g->block_of_tile[block];
     long offset = ((long)(f % g->tf) * g->th + (y % g->th)) * g->tw + (x % g->tw);
     return block * g->bs + offset;
 }
@@ -85,6 +177,7 @@ static long og_tiled_pos(const og_geom *g, int f, int y, int x) {
 static int og_token_at(const og_geom *g, long pos, int *f, int *y, int *x) {
     long block = pos / g->bs;
     long offset = pos % g->bs;
+    if (g->order == 1) block = g->tile_of_block[block];   /* the block's raster tile */
     int bx = (int)(block % g->nbx);
     int by = (int)((block / g->nbx) % g->nby);
     int bf = (int)(block / ((long)g->nbx * g->nby));
@@ -123,10 +216,12 @@ void oracle_geometry(int B, int H, int D, int F, int Hs, int Ws, int tf, int th,
 }
 
 /* Exported: valid-token count of every block, int32[nb]. */
-void oracle_block_valid_counts(int F, int Hs, int Ws, int tf, int th, int tw, int *out) {
+void oracle_block_valid_counts(int F, int Hs, int Ws, int tf, int th, int tw, int order, int *out) {
     og_geom g;
     og_make(&g, 1, 1, 1, F, Hs, Ws, tf, th, tw);
+    og_set_order(&g, order);
     for (long b = 0; b < g.nb; ++b) out[b] = og_block_valid(&g, b);
+    og_free(&g);
 }
 
 /* ------------------------------------------------------------------ */
@@ -135,9 +230,10 @@ void oracle_block_valid_counts(int F, int Hs, int Ws, int tf, int th, int tw, in
 
 /* x: raster [B, N, H, D]  ->  out: tiled [B, H, Npad, D]; padding is zero. */
 void oracle_reorder(const uint16_t *x, uint16_t *out,
-                    int B, int H, int D, int F, int Hs, int Ws, int tf, int th, int tw) {
+                    int B, int H, int D, int F, int Hs, int Ws, int tf, int th, int tw, int order) {
     og_geom g;
     og_make(&g, B, H, D, F, Hs, Ws, tf, th, tw);
+    og_set_order(&g, order);
     memset(out, 0, sizeof(uint16_t) * (size_t)B * H * g.Npad * D);
     #pragma omp parallel for collapse(2) schedule(static)
     for (int b = 0; b < B; ++b)
@@ -152,13 +248,15 @@ void oracle_reorder(const uint16_t *x, uint16_t *out,
                         memcpy(dst, src, sizeof(uint16_t) * D);
                     }
                 }
+    og_free(&g);
 }
 
 /* t: tiled [B, H, Npad, D]  ->  x: raster [B, N, H, D]; padding is dropped. */
 void oracle_inverse_reorder(const uint16_t *t, uint16_t *x,
-                            int B, int H, int D, int F, int Hs, int Ws, int tf, int th, int tw) {
+                            int B, int H, int D, int F, int Hs, int Ws, int tf, int th, int tw, int order) {
     og_geom g;
     og_make(&g, B, H, D, F, Hs, Ws, tf, th, tw);
+    og_set_order(&g, order);
     #pragma omp parallel for collapse(2) schedule(static)
     for (int b = 0; b < B; ++b)
         for (int f = 0; f < F; ++f)
@@ -172,6 +270,7 @@ void oracle_inverse_reorder(const uint16_t *t, uint16_t *x,
                         memcpy(dst, src, sizeof(uint16_t) * D);
                     }
                 }
+    og_free(&g);
 }
 
 /* ------------------------------------------------------------------ */
@@ -183,9 +282,10 @@ void oracle_inverse_reorder(const uint16_t *t, uint16_t *x,
  * excluded from the mean).  t: tiled [B, H, Npad, D] bf16 bits;
  * out: [B, H, nb, D] double. */
 void oracle_pool(const uint16_t *t, double *out,
-                 int B, int H, int D, int F, int Hs, int Ws, int tf, int th, int tw) {
+                 int B, int H, int D, int F, int Hs, int Ws, int tf, int th, int tw, int order) {
     og_geom g;
     og_make(&g, B, H, D, F, Hs, Ws, tf, th, tw);
+    og_set_order(&g, order);
     #pragma omp parallel for collapse(2) schedule(static)
     for (int bh = 0; bh < B * H; ++bh)
         for (int blk = 0; blk < g.nb; ++blk) {
@@ -201,6 +301,7 @@ void oracle_pool(const uint16_t *t, double *out,
             }
             for (int d = 0; d < D; ++d) acc[d] /= (double)n_valid;
         }
+    og_free(&g);
 }
 
 /* Block scores: L[i][j] = scale * <qp_i, kp_j> per (b, h).  qp, kp: [BH, nb, D]
@@ -329,9 +430,10 @@ void oracle_select(const float *L, int rows, int nb, double p, int k, double tie
 void oracle_attention(const uint16_t *qt, const uint16_t *kt, const uint16_t *vt,
                       const int *kv_idx, const int *kv_cnt, const long *items, int n_items,
                       double scale, double *out,
-                      int B, int H, int D, int F, int Hs, int Ws, int tf, int th, int tw) {
+                      int B, int H, int D, int F, int Hs, int Ws, int tf, int th, int tw, int order) {
     og_geom g;
     og_make(&g, B, H, D, F, Hs, Ws, tf, th, tw);
+    og_set_order(&g, order);
     const int bs = g.bs;
     #pragma omp parallel
     {
@@ -385,6 +487,7 @@ void oracle_attention(const uint16_t *qt, const uint16_t *kt, const uint16_t *vt
         free(key_pos);
         free(qrow);
     }
+    og_free(&g);
 }
 
 /* Exported: number of OpenMP threads the oracle will use. */

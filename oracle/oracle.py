@@ -44,14 +44,15 @@ def lib():
         Dd = ctypes.c_double
         geo = [I] * 9
         L.oracle_geometry.argtypes = geo + [P]
-        L.oracle_block_valid_counts.argtypes = [I] * 6 + [P]
-        L.oracle_reorder.argtypes = [P, P] + geo
-        L.oracle_inverse_reorder.argtypes = [P, P] + geo
-        L.oracle_pool.argtypes = [P, P] + geo
+        L.oracle_block_valid_counts.argtypes = [I] * 7 + [P]
+        L.oracle_block_order.argtypes = [I, I, I, P]
+        L.oracle_reorder.argtypes = [P, P] + geo + [I]
+        L.oracle_inverse_reorder.argtypes = [P, P] + geo + [I]
+        L.oracle_pool.argtypes = [P, P] + geo + [I]
         L.oracle_logits.argtypes = [P, P, P, I, I, I, Dd]
         L.oracle_select.argtypes = [P, I, I, Dd, I, Dd, P, P, P, P]
         L.oracle_select_aug.argtypes = [P, I, I, Dd, I, I, Dd, P, P, P, P]
-        L.oracle_attention.argtypes = [P, P, P, P, P, P, I, Dd, P] + geo
+        L.oracle_attention.argtypes = [P, P, P, P, P, P, I, Dd, P] + geo + [I]
         L.oracle_num_threads.restype = I
         L.oracle_set_num_threads.argtypes = [I]
         _lib = L
@@ -65,6 +66,21 @@ def _ptr(a: np.ndarray):
 
 def _geo(w):
     return (w.B, w.H, w.D, w.F, w.Hs, w.Ws, w.tf, w.th, w.tw)
+
+
+def _order(w) -> int:
+    """Block order of a workload: 0 raster tile order, 1 Hilbert."""
+    order = getattr(w, "order", "raster")
+    assert order in ("raster", "hilbert"), order
+    return 1 if order == "hilbert" else 0
+
+
+def block_order(nbf: int, nby: int, nbx: int) -> np.ndarray:
+    """Hilbert block order of a tile grid: tile_of_block[nb], raster tile
+    index (frame-major, then row, then col) of each block."""
+    out = np.empty(nbf * nby * nbx, dtype=np.int32)
+    lib().oracle_block_order(int(nbf), int(nby), int(nbx), _ptr(out))
+    return out
 
 
 def num_threads() -> int:
@@ -85,7 +101,7 @@ def geometry(w) -> dict:
 def block_valid_counts(w) -> np.ndarray:
     g = geometry(w)
     out = np.zeros(g["nb"], dtype=np.int32)
-    lib().oracle_block_valid_counts(w.F, w.Hs, w.Ws, w.tf, w.th, w.tw, _ptr(out))
+    lib().oracle_block_valid_counts(w.F, w.Hs, w.Ws, w.tf, w.th, w.tw, _order(w), _ptr(out))
     return out
 
 
@@ -95,7 +111,7 @@ def reorder(x_bits: np.ndarray, w) -> np.ndarray:
     x = np.ascontiguousarray(x_bits, dtype=np.uint16)
     assert x.shape == (w.B, g["N"], w.H, w.D)
     out = np.empty((w.B, w.H, g["Npad"], w.D), dtype=np.uint16)
-    lib().oracle_reorder(_ptr(x), _ptr(out), *_geo(w))
+    lib().oracle_reorder(_ptr(x), _ptr(out), *_geo(w), _order(w))
     return out
 
 
@@ -105,7 +121,7 @@ def inverse_reorder(t_bits: np.ndarray, w) -> np.ndarray:
     t = np.ascontiguousarray(t_bits, dtype=np.uint16)
     assert t.shape == (w.B, w.H, g["Npad"], w.D)
     out = np.empty((w.B, g["N"], w.H, w.D), dtype=np.uint16)
-    lib().oracle_inverse_reorder(_ptr(t), _ptr(out), *_geo(w))
+    lib().oracle_inverse_reorder(_ptr(t), _ptr(out), *_geo(w), _order(w))
     return out
 
 
@@ -114,7 +130,7 @@ def pool(t_bits: np.ndarray, w) -> np.ndarray:
     g = geometry(w)
     t = np.ascontiguousarray(t_bits, dtype=np.uint16)
     out = np.empty((w.B, w.H, g["nb"], w.D), dtype=np.float64)
-    lib().oracle_pool(_ptr(t), _ptr(out), *_geo(w))
+    lib().oracle_pool(_ptr(t), _ptr(out), *_geo(w), _order(w))
     return out
 
 
@@ -166,7 +182,7 @@ def attention(qt_bits, kt_bits, vt_bits, kv_idx, kv_cnt, items, w, scale: float)
     it = np.ascontiguousarray(np.asarray(items, dtype=np.int64))
     out = np.empty((len(it), g["bs"], w.D), dtype=np.float64)
     lib().oracle_attention(_ptr(qt), _ptr(kt), _ptr(vt), _ptr(idx), _ptr(cnt), _ptr(it),
-                           len(it), float(scale), _ptr(out), *_geo(w))
+                           len(it), float(scale), _ptr(out), *_geo(w), _order(w))
     return out
 
 

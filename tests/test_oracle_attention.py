@@ -81,17 +81,23 @@ def test_full_mask_equals_dense_attention(orc, g):
             np.testing.assert_allclose(got[b, :, h], want, rtol=0, atol=1e-12)
 
 
+@pytest.mark.parametrize("order", ["raster", "hilbert"])
 @pytest.mark.parametrize("g", GEOMS)
-def test_block_mask_equals_token_mask(orc, g):
+def test_block_mask_equals_token_mask(orc, g, order):
     """A routed block mask, expanded to tokens by tile membership in raster
-    layout, gives the same attention as the oracle's block path."""
-    w, q, k, v = _setup(g, seed=7)
+    layout, gives the same attention as the oracle's block path (under either
+    block order: a token's block is its tile's index in that order)."""
+    w = synth.custom_workload(seed=7, order=order, **g)
+    q, k, v, _ = synth.make_qkv(w)
     geo = orc.geometry(w)
     nb = geo["nb"]
     qt, kt = (orc.reorder(synth.bf16_bits(t), w) for t in (q, k))
     _, _, _, kv_idx, kv_cnt, _, _ = orc.route(qt, kt, w, 0.6, 1, 1.0 / np.sqrt(w.D))
     got = _oracle_raster_output(orc, w, q, k, v, kv_idx, kv_cnt)
     tile = _tile_of_tokens(w, geo)
+    if order == "hilbert":
+        block_of_tile = np.argsort(orc.block_order(geo["nbf"], geo["nby"], geo["nbx"]))
+        tile = block_of_tile[tile]
     qd, kd, vd = (t.double().numpy() for t in (q, k, v))
     for b in range(w.B):
         for h in range(w.H):
