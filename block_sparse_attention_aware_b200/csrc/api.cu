@@ -29,7 +29,77 @@ extern "C" int fvattn_geom_init(fvattn_geom* g) {
     g->nb = static_cast<int>(nb);
     g->N = static_cast<long long>(g->F) * g->Hs * g->Ws;
     g->Npad = nb * bs;
+    g->order = nullptr;
     if (static_cast<long long>(g->B) * g->H * g->Npad >= (1ll << 31)) return FVATTN_ERR_UNSUPPORTED;
+    return FVATTN_OK;
+}
+
+namespace fv {
+
+// Curve index of tile (tf_, ty_, tx_) on the 3-D Hilbert curve of a 2^bits
+// cube (J. Skilling, "Programming the Hilbert curve", AIP Conf. Proc. 707,
+// 2004): undo the curve's rotations and reflections from the top bit down,
+// Gray-encode the result, then interleave its bits (frame axis first).
+__device__ unsigned long long hilbert_index3(unsigned tf_, unsigned ty_, unsigned tx_, int bits) {
+    unsigned a[3] = {tf_, ty_, tx_};
+    for (int level = bits - 1; level >= 1; --level) {
+        const unsigned q = 1u << level, mask = q - 1u;
+#pragma unroll
+        for (int i = 0; i < 3; ++i) {
+            if (a[i] & q) {
+                a[0] ^= mask;
+            } else {
+                const unsigned swap = (a[0] ^ a[i]) & mask;
+                a[0] ^= swap;
+                a[i] ^= swap;
+            }
+        }
+    }
+    a[1] ^= a[0];
+    a[2] ^= a[1];
+    unsigned flip = 0u;
+    for (int level = bits - 1; level >= 1; --level)
+        if (a[2] & (1u << level)) flip ^= (1u << level) - 1u;
+    unsigned long long key = 0ull;
+    for (int level = bits - 1; level >= 0; --level) {
+        key = (key << 3) | (static_cast<unsigned long long>(((a[0] ^ flip) >> level) & 1u) << 2) |
+              (static_cast<unsigned long long>(((a[1] ^ flip) >> level) & 1u) << 1) |
+              static_cast<unsigned long long>(((a[2] ^ flip) >> level) & 1u);
+    }
+    return key;
+}
+
+// One CTA: every tile's curve index into shared memory, then each tile's
+// block = its rank among them (indices are distinct).
+__global__ void __launch_bounds__(512) block_order_kernel(int nbf, int nby, int nbx, int bits,
+                                                          int32_t* __restrict__ table) {
+    extern __shared__ unsigned long long curve_key[];
+    const int nb = nbf * nby * nbx;
+    for (int t = threadIdx.x; t < nb; t += blockDim.x)
+        curve_key[t] = hilbert_index3(static_cast<unsigned>(t / (nby * nbx)), static_cast<unsigned>((t / nbx) % nby),
+                                      static_cast<unsigned>(t % nbx), bits);
+    __syncthreads();
+    for (int t = threadIdx.x; t < nb; t += blockDim.x) {
+        const unsigned long long k = curve_key[t];
+        int rank = 0;
+        for (int u = 0; u < nb; ++u) rank += curve_key[u] < k;
+        table[rank] = t;
+        table[nb + t] = rank;
+    }
+}
+
+}  // namespace fv
+
+extern "C" int fvattn_block_order(const fvattn_geom* g, int32_t* table, fvattn_stream_t stream) {
+    if (!g || !table || (reinterpret_cast<uintptr_t>(table) & 15u) != 0) return FVATTN_ERR_INVALID;
+    if (g->nb <= 0 || g->nb > 2560 || g->nbf * g->nby * g->nbx != g->nb) return FVATTN_ERR_INVALID;
+    int side = g->nbf > g->nby ? g->nbf : g->nby;
+    if (g->nbx > side) side = g->nbx;
+    int bits = 1;
+    while ((1 << bits) < side) ++bits;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    block_order_kernel<<<1, 512, sizeof(unsigned long long) * g->nb, s>>>(g->nbf, g->nby, g->nbx, bits, table);
+    FV_CHECK_LAUNCH();
     return FVATTN_OK;
 }
 

@@ -130,6 +130,7 @@ struct Smem {
 // Real extent of a tile: frames, rows and cols that hold tokens, packed as
 // nf | ny << 8 | nx << 16 (each <= 128).
 __device__ __forceinline__ int block_extent(const Geo& g, int block) {
+    block = tile_of_block(g, block);
     const int bx = block % g.nbx;
     const int rest = block / g.nbx;
     const int by = rest % g.nby;

@@ -14,6 +14,7 @@ struct Geo {
     int B, H, D, F, Hs, Ws, tf, th, tw;
     int nbf, nby, nbx, bs, nb;
     long long N, Npad;
+    const int32_t* order;   // block order table (2*nb), or null for raster tile order
 };
 
 inline Geo to_geo(const fvattn_geom& g) {
@@ -22,6 +23,7 @@ inline Geo to_geo(const fvattn_geom& g) {
     k.tf = g.tf; k.th = g.th; k.tw = g.tw;
     k.nbf = g.nbf; k.nby = g.nby; k.nbx = g.nbx; k.bs = g.bs; k.nb = g.nb;
     k.N = g.N; k.Npad = g.Npad;
+    k.order = g.order;
     return k;
 }
 
@@ -32,11 +34,22 @@ __device__ __forceinline__ void record_status(int code) {
     atomicCAS(&g_fvattn_status, 0, code);
 }
 
+// Raster tile index of a block, and block of a raster tile (identities in
+// raster tile order).
+__device__ __forceinline__ int tile_of_block(const Geo& g, int block) {
+    return g.order ? __ldg(g.order + block) : block;
+}
+
+__device__ __forceinline__ long long block_of_tile(const Geo& g, long long tile) {
+    return g.order ? static_cast<long long>(__ldg(g.order + g.nb + tile)) : tile;
+}
+
 // Raster token (f, y, x) of tile-layout position `pos` of a head, and
 // whether it is a real token.
 __device__ __forceinline__ bool token_of_pos(const Geo& g, long long pos, int& f, int& y, int& x) {
     int block = static_cast<int>(pos / g.bs);
     int off = static_cast<int>(pos - static_cast<long long>(block) * g.bs);
+    block = tile_of_block(g, block);
     int bx = block % g.nbx;
     int rest = block / g.nbx;
     int by = rest % g.nby;
@@ -53,6 +66,7 @@ __device__ __forceinline__ bool token_of_pos(const Geo& g, long long pos, int& f
 
 // Number of real tokens in block `block`.
 __device__ __forceinline__ int block_real_tokens(const Geo& g, int block) {
+    block = tile_of_block(g, block);
     int bx = block % g.nbx;
     int rest = block / g.nbx;
     int by = rest % g.nby;

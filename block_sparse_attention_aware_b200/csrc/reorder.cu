@@ -70,7 +70,7 @@ __global__ void __launch_bounds__(256) inverse_reorder_kernel(Geo g, const uint4
         long long fy = n / g.Ws;
         int y = static_cast<int>(fy % g.Hs);
         int f = static_cast<int>(fy / g.Hs);
-        long long block = (static_cast<long long>(f / g.tf) * g.nby + y / g.th) * g.nbx + xx / g.tw;
+        long long block = block_of_tile(g, (static_cast<long long>(f / g.tf) * g.nby + y / g.th) * g.nbx + xx / g.tw);
         long long off = (static_cast<long long>(f % g.tf) * g.th + y % g.th) * g.tw + xx % g.tw;
         src_row = (b * g.H + h) * g.Npad + block * g.bs + off;
     }

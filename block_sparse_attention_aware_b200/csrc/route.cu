@@ -65,7 +65,8 @@ __global__ void __launch_bounds__(256, 4) pool_kernel(Geo g, const __nv_bfloat16
     const long long dst_off = (bh * g.nb + blk) * D;
     const int vec = lane % VPR;
     const int r0 = lane / VPR;
-    const int bx = blk % g.nbx, by = (blk / g.nbx) % g.nby, bf = blk / (g.nbx * g.nby);
+    const int tile = tile_of_block(g, blk);
+    const int bx = tile % g.nbx, by = (tile / g.nbx) % g.nby, bf = tile / (g.nbx * g.nby);
     const int nf = min(g.tf, g.F - bf * g.tf);
     const int ny = min(g.th, g.Hs - by * g.th);
     const int nx = min(g.tw, g.Ws - bx * g.tw);

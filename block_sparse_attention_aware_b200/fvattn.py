@@ -20,7 +20,7 @@ LIB_PATH = os.path.join(_HERE, "libfvattn.so")
 _lib = None
 
 OK, ERR_INVALID, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_BOUNDS = range(6)
-EXPORTED = ("fvattn_geom_init", "fvattn_reorder", "fvattn_inverse_reorder",
+EXPORTED = ("fvattn_geom_init", "fvattn_block_order", "fvattn_reorder", "fvattn_inverse_reorder",
             "fvattn_route_workspace_size", "fvattn_route_kernel_launches", "fvattn_route", "fvattn_route_aug",
             "fvattn_attn_workspace_size",
             "fvattn_num_sms", "fvattn_sparse_attn", "fvattn_sparse_attn_raster", "fvattn_sparse_attn_noalloc",
@@ -39,7 +39,7 @@ class Geom(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int) for n in
                 ("B", "H", "D", "F", "Hs", "Ws", "tf", "th", "tw",
                  "Fp", "Hp", "Wp", "nbf", "nby", "nbx", "bs", "nb")] + \
-               [("N", ctypes.c_longlong), ("Npad", ctypes.c_longlong)]
+               [("N", ctypes.c_longlong), ("Npad", ctypes.c_longlong), ("order", ctypes.c_void_p)]
 
 
 def load(path: str = LIB_PATH):
@@ -55,6 +55,8 @@ def load(path: str = LIB_PATH):
     G = ctypes.POINTER(Geom)
     L.fvattn_geom_init.argtypes = [G]
     L.fvattn_geom_init.restype = I
+    L.fvattn_block_order.argtypes = [G, P, P]
+    L.fvattn_block_order.restype = I
     L.fvattn_reorder.argtypes = [G, P, P, P]
     L.fvattn_reorder.restype = I
     L.fvattn_inverse_reorder.argtypes = [G, P, P, P]
@@ -118,6 +120,22 @@ def geom(B, H, D, F, Hs, Ws, tf, th, tw) -> Geom:
 def geom_of(w) -> Geom:
     """Geometry of a synth.Workload."""
     return geom(w.B, w.H, w.D, w.F, w.Hs, w.Ws, w.tf, w.th, w.tw)
+
+
+def block_order(g: Geom, device="cuda", stream=None) -> torch.Tensor:
+    """fvattn_block_order: the Hilbert block-order table (int32 [2*nb]) of a
+    geometry.  Put it in a geometry with with_order(g, table)."""
+    table = torch.empty(2 * g.nb, dtype=torch.int32, device=device)
+    _check("fvattn_block_order", load().fvattn_block_order(ctypes.byref(g), _ptr(table), _stream(stream)))
+    return table
+
+
+def with_order(g: Geom, table: Optional[torch.Tensor]) -> Geom:
+    """A copy of g that numbers blocks by `table` (None: raster tile order).
+    The table must stay alive while the geometry is used."""
+    g2 = Geom.from_buffer_copy(g)
+    g2.order = None if table is None else table.data_ptr()
+    return g2
 
 
 def route_kernel_launches(g: Geom) -> int:
@@ -282,7 +300,11 @@ class Layer:
     inverse reorder)."""
 
     def __init__(self, g: Geom, p: float, k: int, scale: Optional[float] = None, device="cuda",
-                 debug: bool = False):
+                 debug: bool = False, order: str = "raster"):
+        if order not in ("raster", "hilbert"):
+            raise ValueError(f"block order {order!r}")
+        self.order_table = block_order(g, device) if order == "hilbert" else None
+        g = with_order(g, self.order_table)
         self.g, self.p, self.k = g, p, k
         self.scale = 1.0 / math.sqrt(g.D) if scale is None else scale
         self.qt = tiled_empty(g, device)

@@ -70,6 +70,10 @@ typedef struct {
     int nbf, nby, nbx;    /* tiles along frame, row, col */
     int bs, nb;           /* tokens per block, blocks per head (nb <= 2560) */
     long long N, Npad;    /* raster tokens, padded tokens (= nb*bs) */
+    /* optional, set by the caller after fvattn_geom_init: device table of
+     * 2*nb int32 written by fvattn_block_order; NULL numbers the tiles in
+     * raster tile order (fvattn_geom_init sets NULL) */
+    const int32_t *order;
 } fvattn_geom;
 
 /* Validate the caller-set fields and fill the derived ones.
@@ -77,11 +81,23 @@ typedef struct {
  * for D not in {64, 128}, bs not in {16, 32, 64, 128} or nb > 2560. */
 int fvattn_geom_init(fvattn_geom *g);
 
+/* Hilbert block order (paperlayer.ai summary, section 3, "Sparse-routing
+ * frontend": Hilbert-curve block reordering places spatially adjacent tokens
+ * in nearby blocks).  Writes into `table` (device, 2*nb int32, 16-byte
+ * aligned): [0, nb) the raster tile index ((f/tf)*nby + y/th)*nbx + x/tw of
+ * each block, [nb, 2nb) the block of each raster tile.  Blocks are numbered
+ * by increasing index of their tile along the 3-D Hilbert curve of the
+ * smallest cube of side 2^b holding the (nbf, nby, nbx) tile grid.  Set
+ * g->order = table afterwards to use it in every call; tokens inside a tile
+ * keep raster order.  Asynchronous on `stream`. */
+int fvattn_block_order(const fvattn_geom *g, int32_t *table, fvattn_stream_t stream);
+
 /* Video-aware block organisation (paperlayer.ai summary, section 3,
  * "Sparse-routing frontend": spatially adjacent tokens share a block).
  *   x       [B, N, H, D] bf16, raster token order (the DiT's layout)
  *   x_tiled [B, H, Npad, D] bf16; token (f, y, x) of head h goes to row
- *           block*bs + offset, block = ((f/tf)*nby + y/th)*nbx + x/tw,
+ *           block*bs + offset, block = ((f/tf)*nby + y/th)*nbx + x/tw
+ *           (or that tile's block in g->order when set),
  *           offset = ((f%tf)*th + y%th)*tw + x%tw; padding rows are zero.
  * Bit copy.  x and x_tiled must not overlap. */
 int fvattn_reorder(const fvattn_geom *g, const void *x, void *x_tiled, fvattn_stream_t stream);

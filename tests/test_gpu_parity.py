@@ -68,11 +68,12 @@ def _attn_check(orc, w, g, qt, kt, vt, ot, kv_idx, kv_cnt, items, scale):
     qb, kb, vb = _bits(qt), _bits(kt), _bits(vt)
     ref = orc.attention(qb, kb, vb, kv_idx.cpu().numpy(), kv_cnt.cpu().numpy(), items, w, scale)
     counts = orc.block_valid_counts(w)
+    tile_of = orc.block_order(g.nbf, g.nby, g.nbx) if getattr(w, "order", "raster") == "hilbert" else None
     got_all = ot.view(-1, g.bs, g.D)
     errs = []
     for n, it in enumerate(items):
         blk = it % g.nb
-        real = _real_rows(w, g, blk)
+        real = _real_rows(w, g, blk if tile_of is None else int(tile_of[blk]))
         got = got_all[it].float().cpu().numpy()[real]
         want = ref[n][real]
         assert len(real) == counts[blk]
@@ -85,6 +86,7 @@ _real_cache = {}
 
 
 def _real_rows(w, g, blk):
+    """Real token rows of raster tile `blk` (a block's tile in raster tile order)."""
     key = (w.F, w.Hs, w.Ws, w.tf, w.th, w.tw, blk)
     if key not in _real_cache:
         bx = blk % g.nbx
@@ -231,6 +233,59 @@ def test_fused_inverse_reorder_bit_exact(fv, name, w):
     torch.cuda.synchronize()
     assert fv.get_status() == 0
     assert torch.equal(got.view(torch.int16), want.view(torch.int16))
+
+
+@pytest.mark.parametrize("dims", [(11, 6, 10), (21, 6, 10), (3, 3, 3), (1, 1, 1), (2, 4, 4), (1, 2, 40)])
+def test_block_order_table_matches_oracle(fv, orc, dims):
+    nbf, nby, nbx = dims
+    g = fv.geom(1, 1, 64, nbf, nby * 4, nbx * 4, 1, 4, 4)
+    assert (g.nbf, g.nby, g.nbx) == dims
+    table = fv.block_order(g).cpu().numpy()
+    want = orc.block_order(nbf, nby, nbx)
+    assert np.array_equal(table[: g.nb], want)
+    assert np.array_equal(table[g.nb:], np.argsort(want))
+
+
+HILBERT = [
+    ("hilbert-bs128", synth.custom_workload(B=1, H=2, D=128, F=5, Hs=19, Ws=21, tf=2, th=8, tw=8, seed=6,
+                                            p=0.9, k=3, qscale="fixed", qscale_values=(1.0, 8.0), order="hilbert")),
+    ("hilbert-bs64", synth.custom_workload(B=2, H=2, D=128, F=3, Hs=16, Ws=24, tf=1, th=8, tw=8, seed=7,
+                                           p=0.95, k=4, qscale="fixed", qscale_values=(0.5, 4.0), order="hilbert")),
+    ("hilbert-bs16", synth.custom_workload(B=2, H=3, D=64, F=3, Hs=5, Ws=7, tf=2, th=2, tw=4, seed=5,
+                                           p=0.8, k=2, qscale="fixed", qscale_values=(0.3, 2.0, 6.0),
+                                           order="hilbert")),
+    ("hilbert-lowrank", synth.custom_workload(B=1, H=3, D=128, F=6, Hs=24, Ws=32, tf=2, th=8, tw=8, seed=9,
+                                              p=0.9, k=2, lowrank=True, order="hilbert")),
+]
+
+
+@pytest.mark.parametrize("name,w", HILBERT, ids=[s[0] for s in HILBERT])
+def test_hilbert_layer_parity(fv, orc, name, w):
+    """Hilbert block order through all four calls: reorder and inverse
+    bit-exact, masks (block indices in curve order) equal to the oracle's on
+    the GPU logits outside near ties, attention within the bar."""
+    g = fv.geom_of(w)
+    q, k, v = _gpu_inputs(w)
+    layer = fv.Layer(g, w.p, w.k, debug=True, order="hilbert")
+    out = layer(q, k, v, stats=True)
+    torch.cuda.synchronize()
+    assert fv.get_status() == 0
+    for x, xt in ((q, layer.qt), (k, layer.kt), (v, layer.vt)):
+        assert np.array_equal(_bits(xt), orc.reorder(_bits(x), w))
+    assert np.array_equal(_bits(out), orc.inverse_reorder(_bits(layer.ot), w))
+    # pooled means and logits against the oracle's own (Hilbert) pipeline
+    qp_o, kp_o = orc.pool(_bits(layer.qt), w), orc.pool(_bits(layer.kt), w)
+    L_o = orc.logits(qp_o, kp_o, layer.scale)
+    L_g = layer.routed.logits.cpu().numpy().astype(np.float64)
+    nq = np.linalg.norm(qp_o, axis=-1)[..., :, None]
+    nk = np.linalg.norm(kp_o, axis=-1)[..., None, :]
+    assert np.all(np.abs(L_g - L_o) <= 2e-5 * layer.scale * nq * nk + 1e-6)
+    bad, unexcused, _ = _check_mask(orc, layer.routed.logits, layer.routed.kv_idx, layer.routed.kv_cnt, w.p, w.k)
+    assert unexcused == []
+    items = list(range(w.B * w.H * g.nb))
+    mx, mean = _attn_check(orc, w, g, layer.qt, layer.kt, layer.vt, layer.ot, layer.routed.kv_idx,
+                           layer.routed.kv_cnt, items, layer.scale)
+    assert mx <= MAX_ABS and mean <= MEAN_ABS, (mx, mean)
 
 
 @pytest.mark.parametrize("p,k,k_extra", [(0.0, 3, 0), (0.0, 1, 2), (0.7, 2, 3), (0.9, 1, 10_000)])
