@@ -60,6 +60,7 @@ def workload_config(w, g):
                     f"p={w.p}, k={w.k}",
         "global_batch": w.B, "seq_len": w.N, "heads": w.H, "head_dim": w.D,
         "block": f"{w.tf}x{w.th}x{w.tw}", "nb": g.nb, "p": w.p, "k_floor": w.k,
+        "block_order": getattr(w, "order", "raster"),
         "l2": (f"no flush: every input tensor ({w.B * w.N * w.H * w.D * 2 / 1e6:.0f} MB raster) is larger "
                "than the 126 MB L2") if w.B * w.N * w.H * w.D * 2 > 126e6 else
               "small layer: inputs fit in L2 (no flush; not a bandwidth measurement)",
@@ -302,11 +303,14 @@ def run_fvattn(args):
     w = synth.WORKLOADS[args.workload]
     if args.heads:
         w = synth.custom_workload(**{**w.as_dict(), "H": args.heads, "name": f"{w.name}-h{args.heads}"})
+    if args.order != w.order:
+        w = synth.custom_workload(**{**w.as_dict(), "order": args.order})
     g = fvattn.geom_of(w)
     dev = torch.device("cuda", local)
     # each rank: its own seeded replica layer
     q, k, v, _ = synth.make_qkv(w, layer=rank, device=dev)
-    layer = fvattn.Layer(g, w.p, w.k, device=dev)
+    layer = fvattn.Layer(g, w.p, w.k, device=dev, order=args.order)
+    g = layer.g
     stream = torch.cuda.current_stream(dev)
     nsm = fvattn.num_sms()
 
@@ -478,6 +482,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--workload", default=WORKLOAD, help="named workload of synth.WORKLOADS")
+    ap.add_argument("--order", default="raster", choices=["raster", "hilbert"],
+                    help="block order of the tiles (raster tile order or the 3-D Hilbert curve)")
     ap.add_argument("--stack", action="store_true",
                     help="also time every seeded layer of a multi-layer workload once (cfg720p: 40 layers)")
     ap.add_argument("--heads", type=int, default=0,
