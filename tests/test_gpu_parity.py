@@ -113,6 +113,9 @@ SMALL = [
                                        p=0.7, k=2, qscale="fixed", qscale_values=(1.0, 10.0))),
     ("lowrank-bs128", synth.custom_workload(B=1, H=3, D=128, F=6, Hs=24, Ws=32, tf=2, th=8, tw=8, seed=9,
                                             p=0.9, k=2, lowrank=True)),
+    # head dim 64 with 128-token blocks, two batch entries, padding on the frame and row axes
+    ("bs128-d64-b2", synth.custom_workload(B=2, H=2, D=64, F=3, Hs=20, Ws=16, tf=2, th=8, tw=8, seed=12,
+                                           p=0.85, k=2, qscale="fixed", qscale_values=(0.7, 5.0))),
     # nb = 9 with two 64-token query blocks per tile: the last tile holds one block
     ("bs64-odd-nb", synth.custom_workload(B=1, H=2, D=128, F=3, Hs=8, Ws=24, tf=1, th=8, tw=8, seed=11,
                                           p=0.6, k=2, qscale="fixed", qscale_values=(0.5, 6.0))),
