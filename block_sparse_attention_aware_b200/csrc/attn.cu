@@ -633,24 +633,36 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                             const int q = q2 + hq;
                             const uint32_t mword = q == 0 ? mw0 : (q == 1 ? mw1 : (q == 2 ? mw2 : mw3));
                             uint32_t wv[16];
+                            if (mword == 0xFFFFFFFFu) {
+                                // every key of these 32 columns is visible
 #pragma unroll
-                            for (int i = 0; i < 32; i += 2) {
-                                const float s0 = __uint_as_float(v[hq][i]), s1 = __uint_as_float(v[hq][i + 1]);
-                                float x0, x1;
-                                f2_unpack(f2_fma(f2_pack(s0, s1), sl2x2, negx2), x0, x1);
-                                float p0 = ex2_approx(x0);
-                                float p1 = ex2_approx(x1);
-                                if (partial) {
+                                for (int i = 0; i < 32; i += 2) {
+                                    const float s0 = __uint_as_float(v[hq][i]), s1 = __uint_as_float(v[hq][i + 1]);
+                                    float x0, x1;
+                                    f2_unpack(f2_fma(f2_pack(s0, s1), sl2x2, negx2), x0, x1);
+                                    const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+                                    if (TRACK) mx[(i >> 1) & 7] = fmax3(mx[(i >> 1) & 7], s0, s1);
+                                    sm2[(i >> 1) & 3] = f2_add(sm2[(i >> 1) & 3], f2_pack(p0, p1));
+                                    wv[i >> 1] = pack_bf16x2(p0, p1);
+                                }
+                            } else if (mword == 0u) {
+                                // no visible key here: P = 0, nothing to the sum or the maximum
+#pragma unroll
+                                for (int i = 0; i < 16; ++i) wv[i] = 0u;
+                            } else {
+#pragma unroll
+                                for (int i = 0; i < 32; i += 2) {
+                                    const float s0 = __uint_as_float(v[hq][i]), s1 = __uint_as_float(v[hq][i + 1]);
+                                    float x0, x1;
+                                    f2_unpack(f2_fma(f2_pack(s0, s1), sl2x2, negx2), x0, x1);
                                     const bool k0 = (mword >> i) & 1u, k1 = (mword >> (i + 1)) & 1u;
-                                    p0 = k0 ? p0 : 0.f;
-                                    p1 = k1 ? p1 : 0.f;
+                                    const float p0 = k0 ? ex2_approx(x0) : 0.f;
+                                    const float p1 = k1 ? ex2_approx(x1) : 0.f;
                                     if (TRACK)
                                         mx[(i >> 1) & 7] = fmax3(mx[(i >> 1) & 7], k0 ? s0 : -INFINITY, k1 ? s1 : -INFINITY);
-                                } else if (TRACK) {
-                                    mx[(i >> 1) & 7] = fmax3(mx[(i >> 1) & 7], s0, s1);
+                                    sm2[(i >> 1) & 3] = f2_add(sm2[(i >> 1) & 3], f2_pack(p0, p1));
+                                    wv[i >> 1] = pack_bf16x2(p0, p1);
                                 }
-                                sm2[(i >> 1) & 3] = f2_add(sm2[(i >> 1) & 3], f2_pack(p0, p1));
-                                wv[i >> 1] = pack_bf16x2(p0, p1);
                             }
                             const int half = q >> 1;
 #pragma unroll
