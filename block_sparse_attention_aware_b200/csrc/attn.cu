@@ -40,8 +40,6 @@
 // always reaches the TMEM release.
 #include <cuda.h>
 
-#include <type_traits>
-
 #include "common.cuh"
 #include "ptx.cuh"
 #include "sync.cuh"
@@ -57,11 +55,13 @@ constexpr int V_STAGES = 2;             // V ring: a stage is free once its O +=
 constexpr uint32_t MAX_DYN_SMEM = 232448;   // sm_100 opt-in shared memory per block
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t O_COL = 256;          // S_w at columns 128*w, O_w at 256 + 128*w
-// Lazy rescaling: the running row maximum (log2 units) is only moved, and O
-// rescaled, when a new score exceeds it by more than this; until then
-// probabilities may reach 2^32, which bf16 P (8-bit exponent) and fp32 sums
-// and accumulators hold with their usual relative precision.
-constexpr float RESCALE_THRESHOLD = 32.0f;
+// Lazy rescaling: after an item's first chunk, a chunk's P is computed against
+// the running reference maximum without looking at the chunk's own maximum;
+// only when a row's chunk sum exceeds this (so some P may be large) is the
+// chunk redone against its exact maximum with O rescaled.  P below 2^30 is
+// held by bf16 P (8-bit exponent) and fp32 sums with their usual relative
+// precision.
+constexpr float RESCALE_SUM_LIMIT = 1073741824.0f;   // 2^30
 constexpr int MAX_GROUP = 8;             // query blocks per tile at bs = 16
 
 struct AttnArgs {
@@ -609,18 +609,12 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                 if (lane == 0) mbar_arrive(smem_u32(&ctl.k_empty[kst]));   // mask in registers: stage free
                 tc_fence_after();
                 // Exp pass: P = 2^(s*scale*log2e + negv), row sum on fp32 pairs, bf16 P row into P_w
-                // (128-byte swizzle, K-major operand), two TMEM loads in flight; with TRACK it also
-                // takes the row maximum of the (masked) raw scores.
+                // (128-byte swizzle, K-major operand), two TMEM loads in flight.
                 unsigned long long sm2[4];   // four chains of (even, odd) column sums
                 float mx[8];
-                auto exp_pass = [&](auto track, float negv) {
-                    constexpr bool TRACK = decltype(track)::value;
+                auto exp_pass = [&](float negv) {
 #pragma unroll
                     for (int i = 0; i < 4; ++i) sm2[i] = 0ull;
-                    if (TRACK) {
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) mx[i] = -INFINITY;
-                    }
                     const unsigned long long sl2x2 = f2_pack(sl2, sl2), negx2 = f2_pack(negv, negv);
 #pragma unroll 1
                     for (int q2 = 0; q2 < 4; q2 += 2) {
@@ -641,7 +635,6 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                                     float x0, x1;
                                     f2_unpack(f2_fma(f2_pack(s0, s1), sl2x2, negx2), x0, x1);
                                     const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
-                                    if (TRACK) mx[(i >> 1) & 7] = fmax3(mx[(i >> 1) & 7], s0, s1);
                                     sm2[(i >> 1) & 3] = f2_add(sm2[(i >> 1) & 3], f2_pack(p0, p1));
                                     wv[i >> 1] = pack_bf16x2(p0, p1);
                                 }
@@ -658,8 +651,6 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                                     const bool k0 = (mword >> i) & 1u, k1 = (mword >> (i + 1)) & 1u;
                                     const float p0 = k0 ? ex2_approx(x0) : 0.f;
                                     const float p1 = k1 ? ex2_approx(x1) : 0.f;
-                                    if (TRACK)
-                                        mx[(i >> 1) & 7] = fmax3(mx[(i >> 1) & 7], k0 ? s0 : -INFINITY, k1 ? s1 : -INFINITY);
                                     sm2[(i >> 1) & 3] = f2_add(sm2[(i >> 1) & 3], f2_pack(p0, p1));
                                     wv[i >> 1] = pack_bf16x2(p0, p1);
                                 }
@@ -689,9 +680,8 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                     }
                     tmem_wait_st();
                 };
-                float alpha = 1.0f;
-                if (!mine_any) {
-                    // the group's first chunk of the item: row maximum first, then P against it
+                // Row maximum of the visible raw scores of this chunk (scaled to log2 units).
+                auto max_pass = [&]() -> float {
 #pragma unroll
                     for (int i = 0; i < 8; ++i) mx[i] = -INFINITY;
 #pragma unroll
@@ -715,42 +705,54 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                                 mx[(i >> 1) & 7] = fmax3(mx[(i >> 1) & 7], __uint_as_float(sr[hq][i]),
                                                          __uint_as_float(sr[hq][i + 1]));
                     }
+                    return fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                                 fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * sl2;
+                };
+                auto chunk_sum = [&]() -> float {
+                    float sm[8];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) f2_unpack(sm2[i], sm[2 * i], sm[2 * i + 1]);
+                    return ((sm[0] + sm[1]) + (sm[2] + sm[3])) + ((sm[4] + sm[5]) + (sm[6] + sm[7]));
+                };
+                float alpha = 1.0f;
+                float sum;
+                if (!mine_any) {
+                    // the group's first chunk of the item: row maximum first, then P against it
                     // (a row may see no key of its block in a chunk: it keeps max -inf, P 0)
-                    m_ref = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                                  fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * sl2;
+                    m_ref = max_pass();
                     // P_w was last used by this group's previous PV
                     if (!wait_warp(smem_u32(&ctl.p_free[w]), (n & 1) ^ 1, abort_flag)) {
                         ok = false;
                         break;
                     }
-                    exp_pass(std::false_type{}, -m_ref);
+                    exp_pass(-m_ref);
+                    sum = chunk_sum();
                 } else {
-                    // later chunks: one pass against the running reference maximum, which is only
-                    // moved (and O rescaled, and the chunk redone) when a row maximum exceeds it by
-                    // more than 2^RESCALE_THRESHOLD; until then P stays below 2^RESCALE_THRESHOLD
+                    // later chunks: one pass against the running reference maximum.  While a row's sum
+                    // stays below 2^RESCALE_LOG2_SUM no P of it can overflow anything; otherwise (or for
+                    // a row that had seen no key yet) the chunk is redone: exact maximum, O rescaled,
+                    // P recomputed against it.
                     if (!wait_warp(smem_u32(&ctl.p_free[w]), (n & 1) ^ 1, abort_flag)) {
                         ok = false;
                         break;
                     }
-                    exp_pass(std::true_type{}, -m_ref);
-                    const float mxs = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                                            fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * sl2;
-                    const bool grow = mxs > m_ref + RESCALE_THRESHOLD;
-                    if (__any_sync(0xffffffffu, grow)) {
+                    exp_pass(-m_ref);
+                    sum = chunk_sum();
+                    const bool big = !(sum <= RESCALE_SUM_LIMIT);
+                    if (__any_sync(0xffffffffu, big)) {
+                        const float mxs = max_pass();
+                        const bool grow = big && mxs > m_ref;
                         const float m_new = grow ? mxs : m_ref;
                         alpha = grow ? ex2_approx(m_ref - m_new) : 1.0f;
                         m_ref = m_new;
                         rescale_o(alpha);
-                        exp_pass(std::false_type{}, -m_ref);
+                        exp_pass(-m_ref);
+                        sum = chunk_sum();
                     }
                 }
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(smem_u32(&ctl.s_free[w]));   // S_w consumed
-                float sm[8];
-#pragma unroll
-                for (int i = 0; i < 4; ++i) f2_unpack(sm2[i], sm[2 * i], sm[2 * i + 1]);
-                const float sum = ((sm[0] + sm[1]) + (sm[2] + sm[3])) + ((sm[4] + sm[5]) + (sm[6] + sm[7]));
                 l = l * alpha + sum;
                 fence_proxy_async_smem();
                 tc_fence_before();

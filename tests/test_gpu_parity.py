@@ -319,6 +319,26 @@ def test_route_variants(fv, orc, p, k, k_extra):
     assert mx <= MAX_ABS and mean <= MEAN_ABS, (mx, mean)
 
 
+@pytest.mark.parametrize("tw", [8, 4])
+def test_attention_with_extreme_score_range(fv, orc, tw):
+    """Scores spread over hundreds of log2 units (Q scaled by 40, every block
+    kept): later chunks of an item often exceed the running reference maximum,
+    so the one-pass softmax has to redo chunks with O rescaled."""
+    w = synth.custom_workload(B=1, H=2, D=128, F=4, Hs=16, Ws=32, tf=2, th=8, tw=tw, seed=41, p=1.0, k=1,
+                              qscale="fixed", qscale_values=(40.0, 25.0))
+    g = fv.geom_of(w)
+    q, kk, v = _gpu_inputs(w)
+    layer = fv.Layer(g, 1.0, 1)
+    layer(q, kk, v)
+    torch.cuda.synchronize()
+    assert fv.get_status() == 0
+    assert np.all(layer.routed.kv_cnt.cpu().numpy() == g.nb)
+    items = list(range(w.B * w.H * g.nb))
+    mx, mean = _attn_check(orc, w, g, layer.qt, layer.kt, layer.vt, layer.ot, layer.routed.kv_idx,
+                           layer.routed.kv_cnt, items, layer.scale)
+    assert mx <= MAX_ABS and mean <= MEAN_ABS, (mx, mean)
+
+
 def test_single_block_video(fv, orc):
     """nb = 1: one partial block per head (a 1 x 3 x 5 latent in a 2 x 8 x 8 tile)."""
     w = synth.custom_workload(B=1, H=2, D=128, F=1, Hs=3, Ws=5, tf=2, th=8, tw=8, seed=3, p=0.9, k=1)
