@@ -233,6 +233,18 @@ __host__ __device__ constexpr uint32_t idesc_tf32_f32(int M, int N) {
            (static_cast<uint32_t>(M >> 4) << 24);
 }
 
+// ---------------------------------------------------------------- programmatic dependent launch
+
+// Let the next kernel in the stream (launched with programmatic stream
+// serialisation) be scheduled once every CTA of this grid has passed here.
+__device__ __forceinline__ void pdl_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Wait until the preceding grid has completed and its memory is visible (a
+// no-op when this grid was launched without the programmatic attribute).
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ---------------------------------------------------------------- misc
 
 __device__ __forceinline__ float ex2_approx(float x) {

@@ -52,6 +52,7 @@ __global__ void __launch_bounds__(256, 4) pool_kernel(Geo g, const __nv_bfloat16
     constexpr int VPR = D / 8;             // 16-byte vectors per row
     constexpr int RPI = 32 / VPR;          // rows per warp instruction
     constexpr int UNR = 8;                 // loads in flight per lane
+    pdl_launch_dependents();   // the score kernel may be scheduled as this grid drains
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const long long unit = static_cast<long long>(blockIdx.x) * 8 + warp;   // (tensor, bh, blk) flattened
     const long long per_tensor = static_cast<long long>(g.B) * g.H * g.nb;
@@ -71,9 +72,9 @@ __global__ void __launch_bounds__(256, 4) pool_kernel(Geo g, const __nv_bfloat16
     const int ny = min(g.th, g.Hs - by * g.th);
     const int nx = min(g.tw, g.Ws - bx * g.tw);
     const bool full = nf == g.tf && ny == g.th && nx == g.tw;
-    float acc[8];
+    unsigned long long acc2[4];   // fp32 pairs (column 2e, 2e + 1) of this lane's slice
 #pragma unroll
-    for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+    for (int e = 0; e < 4; ++e) acc2[e] = 0ull;
     const int steps = g.bs / RPI;          // warp instructions per tile
     for (int s0 = 0; s0 < steps; s0 += UNR) {
         uint4 u[UNR];
@@ -94,15 +95,18 @@ __global__ void __launch_bounds__(256, 4) pool_kernel(Geo g, const __nv_bfloat16
         }
 #pragma unroll
         for (int i = 0; i < UNR; ++i) {
-            const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&u[i]);
+            const uint32_t wds[4] = {u[i].x, u[i].y, u[i].z, u[i].w};
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-                const float2 f = __bfloat1622float2(p2[e]);
-                acc[2 * e] += f.x;
-                acc[2 * e + 1] += f.y;
+                // a bf16 is the top half of the fp32 with the same value
+                const float lo = __uint_as_float(wds[e] << 16), hi = __uint_as_float(wds[e] & 0xffff0000u);
+                acc2[e] = f2_add(acc2[e], f2_pack(lo, hi));
             }
         }
     }
+    float acc[8];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) f2_unpack(acc2[e], acc[2 * e], acc[2 * e + 1]);
     // lanes with the same column slice hold partial sums of different rows
 #pragma unroll
     for (int o = VPR; o < 32; o <<= 1)
@@ -223,6 +227,8 @@ __global__ void __launch_bounds__(SC_THREADS, 1) score_kernel(const __grid_const
     tc_fence_after();
     const uint32_t tmem = ctl.tmem_base;
     const int per_head = a.m_tiles * a.n_tiles;
+    pdl_launch_dependents();   // the select kernel may be scheduled as this grid drains
+    pdl_wait();                // pooled Q/K of the previous kernel complete and visible
 
     if (warp == 0) {
         // ---- TMA producer
@@ -543,6 +549,7 @@ __global__ void __launch_bounds__(32 * SEL_WARPS, NPL <= 24 ? 4 : 1) select_kern
                                                                 int32_t* __restrict__ kv_idx,
                                                                 int32_t* __restrict__ kv_cnt) {
     __shared__ unsigned long long cand_keys[SEL_WARPS][32];
+    pdl_wait();                // logits of the score kernel complete and visible
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const long long row = static_cast<long long>(blockIdx.x) * SEL_WARPS + warp;
     if (row >= rows) return;
@@ -609,8 +616,19 @@ template <int NPL, bool KEEP_E>
 static int launch_select(long long rows, int nb, const float* L, double p, int kfloor, int kextra, int32_t* kv_idx,
                          int32_t* kv_cnt, cudaStream_t s) {
     const long long blocks = (rows + SEL_WARPS - 1) / SEL_WARPS;
-    select_kernel<NPL, KEEP_E><<<static_cast<unsigned>(blocks), 32 * SEL_WARPS, 0, s>>>(nb, rows, L, p, kfloor, kextra,
-                                                                                      kv_idx, kv_cnt);
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.gridDim = dim3(static_cast<unsigned>(blocks));
+    cfg.blockDim = dim3(32 * SEL_WARPS);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, select_kernel<NPL, KEEP_E>, nb, rows, L, p, kfloor, kextra, kv_idx, kv_cnt) !=
+        cudaSuccess)
+        return FVATTN_ERR_CUDA;
     FV_CHECK_LAUNCH();
     return FVATTN_OK;
 }
@@ -722,7 +740,20 @@ static int route_impl(const fvattn_geom* gp, const void* q_tiled, const void* k_
         cudaSuccess)
         return FVATTN_ERR_CUDA;
     const unsigned sgrid = static_cast<unsigned>(sa.tiles < nsm ? sa.tiles : nsm);
-    score_kernel<<<sgrid, SC_THREADS, SC_SMEM, s>>>(tqh, tql, tkh, tkl, tout, sa);
+    {
+        // programmatic serialisation: the kernel is scheduled while pooling drains and waits in-kernel
+        cudaLaunchConfig_t cfg = {};
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.gridDim = dim3(sgrid);
+        cfg.blockDim = dim3(SC_THREADS);
+        cfg.dynamicSmemBytes = SC_SMEM;
+        cfg.stream = s;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        if (cudaLaunchKernelEx(&cfg, score_kernel, tqh, tql, tkh, tkl, tout, sa) != cudaSuccess) return FVATTN_ERR_CUDA;
+    }
     FV_CHECK_LAUNCH();
     const long long rows = static_cast<long long>(g.B) * g.H * g.nb;
     // entries per lane: the smallest instantiated count that covers a row
