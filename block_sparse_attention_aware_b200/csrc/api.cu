@@ -124,3 +124,20 @@ extern "C" const char* fvattn_status_string(int code) {
         default: return "unknown status";
     }
 }
+
+extern "C" int fvattn_copy_heads(const fvattn_geom* g, int h0, int nh, const void* src, void* dst, int to_device,
+                                 fvattn_stream_t stream) {
+    if (!g || !src || !dst || h0 < 0 || nh < 1 || h0 + nh > g->H) return FVATTN_ERR_INVALID;
+    const size_t row = static_cast<size_t>(g->D) * 2;   // one head of one token, bf16
+    const size_t full = row * g->H, part = row * nh;
+    const size_t rows = static_cast<size_t>(g->B) * static_cast<size_t>(g->N);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e;
+    if (to_device)
+        e = cudaMemcpy2DAsync(dst, part, static_cast<const char*>(src) + row * h0, full, part, rows,
+                              cudaMemcpyHostToDevice, s);
+    else
+        e = cudaMemcpy2DAsync(static_cast<char*>(dst) + row * h0, full, src, part, part, rows,
+                              cudaMemcpyDeviceToHost, s);
+    return e == cudaSuccess ? FVATTN_OK : FVATTN_ERR_CUDA;
+}

@@ -20,7 +20,7 @@ LIB_PATH = os.path.join(_HERE, "libfvattn.so")
 _lib = None
 
 OK, ERR_INVALID, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_BOUNDS = range(6)
-EXPORTED = ("fvattn_geom_init", "fvattn_block_order", "fvattn_reorder", "fvattn_inverse_reorder",
+EXPORTED = ("fvattn_geom_init", "fvattn_block_order", "fvattn_copy_heads", "fvattn_reorder", "fvattn_inverse_reorder",
             "fvattn_route_workspace_size", "fvattn_route_kernel_launches", "fvattn_route", "fvattn_route_aug",
             "fvattn_attn_workspace_size",
             "fvattn_num_sms", "fvattn_sparse_attn", "fvattn_sparse_attn_raster", "fvattn_sparse_attn_noalloc",
@@ -57,6 +57,8 @@ def load(path: str = LIB_PATH):
     L.fvattn_geom_init.restype = I
     L.fvattn_block_order.argtypes = [G, P, P]
     L.fvattn_block_order.restype = I
+    L.fvattn_copy_heads.argtypes = [G, I, I, P, P, I, P]
+    L.fvattn_copy_heads.restype = I
     L.fvattn_reorder.argtypes = [G, P, P, P]
     L.fvattn_reorder.restype = I
     L.fvattn_inverse_reorder.argtypes = [G, P, P, P]
@@ -350,6 +352,63 @@ class Layer:
             return self.attend_raster(stats, stream)
         self.attend(stats, stream)
         return self.restore(stream)
+
+
+class HostPipeline:
+    """End to end from page-locked host buffers, pipelined by head groups.
+
+    Heads are independent through every step, so the layer is run as
+    `groups` head slices on two rotating sets of device buffers: the upload
+    of slice i+1 (one copy stream), the four library calls on slice i (the
+    compute stream) and the download of slice i-1 (another copy stream)
+    overlap.  The output equals one whole-layer call bit for bit."""
+
+    def __init__(self, g: Geom, p: float, k: int, groups: int = 4, device="cuda", order: str = "raster"):
+        if g.H % groups:
+            raise ValueError(f"{g.H} heads do not split into {groups} equal groups")
+        self.g, self.groups, self.nh = g, groups, g.H // groups
+        gs = geom(g.B, self.nh, g.D, g.F, g.Hs, g.Ws, g.tf, g.th, g.tw)
+        self.layers = [Layer(gs, p, k, device=device, order=order) for _ in range(min(2, groups))]
+        shape = (g.B, g.N, self.nh, g.D)
+        self.inputs = [[torch.empty(shape, dtype=torch.bfloat16, device=device) for _ in range(3)]
+                       for _ in self.layers]
+        self.up = torch.cuda.Stream(device=device)
+        self.down = torch.cuda.Stream(device=device)
+
+    def __call__(self, q_host, k_host, v_host, o_host, stream=None):
+        L = load()
+        s = stream if stream is not None else torch.cuda.current_stream()
+        g = self.g
+        start = torch.cuda.Event()
+        start.record(s)
+        self.up.wait_event(start)
+        self.down.wait_event(start)
+        freed = [None] * len(self.layers)     # download of the slice that last used a buffer set
+        done = None
+        for i in range(self.groups):
+            b = i % len(self.layers)
+            lay, (qd, kd, vd) = self.layers[b], self.inputs[b]
+            if freed[b] is not None:
+                self.up.wait_event(freed[b])
+            for src, dst in ((q_host, qd), (k_host, kd), (v_host, vd)):
+                _check("fvattn_copy_heads", L.fvattn_copy_heads(ctypes.byref(g), i * self.nh, self.nh,
+                                                                ctypes.c_void_p(src.data_ptr()), _ptr(dst), 1,
+                                                                _stream(self.up)))
+            uploaded = torch.cuda.Event()
+            uploaded.record(self.up)
+            s.wait_event(uploaded)
+            out = lay(qd, kd, vd, stream=s)
+            computed = torch.cuda.Event()
+            computed.record(s)
+            self.down.wait_event(computed)
+            _check("fvattn_copy_heads", L.fvattn_copy_heads(ctypes.byref(g), i * self.nh, self.nh, _ptr(out),
+                                                            ctypes.c_void_p(o_host.data_ptr()), 0,
+                                                            _stream(self.down)))
+            done = torch.cuda.Event()
+            done.record(self.down)
+            freed[b] = done
+        s.wait_event(done)
+        return o_host
 
 
 def attention_from_host(layer: Layer, q_host, k_host, v_host, o_host, stream=None):

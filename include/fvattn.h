@@ -162,6 +162,16 @@ int fvattn_route_aug(const fvattn_geom *g, const void *q_tiled, const void *k_ti
                      float *q_pool, float *k_pool, float *logits,
                      void *workspace, size_t ws_bytes, fvattn_stream_t stream);
 
+/* Host <-> device copy of a head slice of a raster tensor, for pipelining a
+ * layer by head groups (plumbing; no part of the method).  Heads
+ * [h0, h0 + nh) of a raster [B, N, H, D] bf16 tensor in host memory (page
+ * locked for asynchrony) go to / come from a device [B, N, nh, D] bf16
+ * buffer; g gives B, N, H, D of the full tensor.  to_device = 1: src is the
+ * host tensor, dst the device slice; 0: src is the device slice, dst the
+ * host tensor.  One 2-D asynchronous copy on `stream`. */
+int fvattn_copy_heads(const fvattn_geom *g, int h0, int nh, const void *src, void *dst, int to_device,
+                      fvattn_stream_t stream);
+
 /* Number of kernel launches one fvattn_route call makes for this geometry
  * (pooling, scoring, selection); 0 for a null pointer. */
 int fvattn_route_kernel_launches(const fvattn_geom *g);

@@ -27,7 +27,7 @@ def _declared():
 def test_exports_every_declared_symbol(fv):
     lib = fv.load()
     names = _declared()
-    assert len(names) == 15
+    assert len(names) == 16
     assert sorted(fv.EXPORTED) == names
     for n in names:
         assert hasattr(lib, n), n

@@ -291,6 +291,24 @@ def test_hilbert_layer_parity(fv, orc, name, w):
     assert mx <= MAX_ABS and mean <= MEAN_ABS, (mx, mean)
 
 
+@pytest.mark.parametrize("groups", [2, 4])
+def test_host_pipeline_matches_whole_layer(fv, groups):
+    """The head-group pipeline from page-locked host buffers writes the same
+    bits as one whole-layer call."""
+    w = synth.custom_workload(B=2, H=4, D=128, F=3, Hs=16, Ws=24, tf=2, th=8, tw=8, seed=51, p=0.8, k=2,
+                              qscale="fixed", qscale_values=(0.5, 2.0, 6.0, 1.0))
+    g = fv.geom_of(w)
+    q, k, v = _gpu_inputs(w)
+    want = fv.Layer(g, w.p, w.k)(q, k, v).cpu()
+    qh, kh, vh = (t.cpu().pin_memory() for t in (q, k, v))
+    oh = torch.full_like(qh, float("nan")).pin_memory()
+    pipe = fv.HostPipeline(g, w.p, w.k, groups=groups)
+    pipe(qh, kh, vh, oh)
+    torch.cuda.synchronize()
+    assert fv.get_status() == 0
+    assert torch.equal(oh.view(torch.int16), want.view(torch.int16))
+
+
 @pytest.mark.parametrize("p,k,k_extra", [(0.0, 3, 0), (0.0, 1, 2), (0.7, 2, 3), (0.9, 1, 10_000)])
 def test_route_variants(fv, orc, p, k, k_extra):
     """Fixed Top-k mode (p = 0) and importance-order augmentation (k_extra):
