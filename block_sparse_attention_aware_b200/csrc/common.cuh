@@ -64,19 +64,6 @@ __device__ __forceinline__ bool token_of_pos(const Geo& g, long long pos, int& f
     return f < g.F && y < g.Hs && x < g.Ws;
 }
 
-// Number of real tokens in block `block`.
-__device__ __forceinline__ int block_real_tokens(const Geo& g, int block) {
-    block = tile_of_block(g, block);
-    int bx = block % g.nbx;
-    int rest = block / g.nbx;
-    int by = rest % g.nby;
-    int bf = rest / g.nby;
-    int nf = min(g.tf, g.F - bf * g.tf);
-    int ny = min(g.th, g.Hs - by * g.th);
-    int nx = min(g.tw, g.Ws - bx * g.tw);
-    return nf * ny * nx;
-}
-
 }  // namespace fv
 
 #define FV_CHECK_LAUNCH()                                      \

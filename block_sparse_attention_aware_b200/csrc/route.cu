@@ -445,14 +445,13 @@ __device__ __forceinline__ void sel_eval(const float (&v)[NPL], const float (&e)
 // or a single logit value remains (ties resolved by ascending index).
 // Returns the crossing's order key and its 1-based rank.
 template <int NPL, bool KEEP_E>
-__device__ unsigned long long sel_boundary(const float (&v)[NPL], const float (&e)[NPL], int nb, float lmax, float lmin,
+__device__ unsigned long long sel_boundary(const float (&v)[NPL], const float (&e)[NPL], float lmax, float lmin,
                                            bool mass, int c_all, double target,
                                            unsigned long long* ck, int* rank) {
     const int lane = threadIdx.x & 31;
     uint32_t lo_k = fkey(lmin), hi_k = fkey(lmax) + 1u;
     unsigned long long s_hi = 0ull;
     int c_lo = c_all, c_hi = 0;
-    (void)nb;
 #pragma unroll 1
     for (int it = 0; c_lo - c_hi > 32 && hi_k - lo_k > 1u; ++it) {
         uint32_t mk;
@@ -582,7 +581,7 @@ __global__ void __launch_bounds__(32 * SEL_WARPS, NPL <= 24 ? 4 : 1) select_kern
         if (p > 0.0) {
             sel_eval<NPL, KEEP_E>(v, e, lmax, lmin, true, s_all, c_all);
             const double target = p * static_cast<double>(s_all);
-            thr = sel_boundary<NPL, KEEP_E>(v, e, nb, lmax, lmin, true, c_all, target, cand_keys[warp], &rank);
+            thr = sel_boundary<NPL, KEEP_E>(v, e, lmax, lmin, true, c_all, target, cand_keys[warp], &rank);
         } else {
             sel_eval<NPL, KEEP_E>(v, e, lmax, lmin, false, s_all, c_all);
         }
@@ -591,7 +590,7 @@ __global__ void __launch_bounds__(32 * SEL_WARPS, NPL <= 24 ? 4 : 1) select_kern
         if (want >= c_all) {
             thr = ~0ull;
         } else if (want > rank) {
-            thr = sel_boundary<NPL, KEEP_E>(v, e, nb, lmax, lmin, false, c_all, static_cast<double>(want),
+            thr = sel_boundary<NPL, KEEP_E>(v, e, lmax, lmin, false, c_all, static_cast<double>(want),
                                             cand_keys[warp], &rank);
         }
     }
