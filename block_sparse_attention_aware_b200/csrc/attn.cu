@@ -377,17 +377,23 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                     break;
                 }
                 if (GRP) {
-                    // per query block t of the tile: key column real and its block in t's list
+                    // per query block t of the tile: key column real and its block in t's list.
+                    // Real-token bits once per 32-column word; a word lies in one slot when
+                    // bs >= 32, so its membership bits are warp-uniform there.
+                    uint32_t pad[4], mq[4];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const int e = __shfl_sync(0xffffffffu, ext, c_slot[q]);
+                        mq[q] = __shfl_sync(0xffffffffu, mem, c_slot[q]);
+                        pad[q] = __ballot_sync(0xffffffffu, (c_of[q] < (e & 255)) && (c_oy[q] < ((e >> 8) & 255)) &&
+                                                                (c_ox[q] < (e >> 16)));
+                    }
                     for (int tq = 0; tq < G; ++tq) {
                         uint32_t words[4];
 #pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            const int e = __shfl_sync(0xffffffffu, ext, c_slot[q]);
-                            const uint32_t mm = __shfl_sync(0xffffffffu, mem, c_slot[q]);
-                            const bool valid = (c_of[q] < (e & 255)) && (c_oy[q] < ((e >> 8) & 255)) &&
-                                               (c_ox[q] < (e >> 16)) && ((mm >> tq) & 1u);
-                            words[q] = __ballot_sync(0xffffffffu, valid);
-                        }
+                        for (int q = 0; q < 4; ++q)
+                            words[q] = bs >= 32 ? (((mq[q] >> tq) & 1u) ? pad[q] : 0u)
+                                                : (pad[q] & __ballot_sync(0xffffffffu, (mq[q] >> tq) & 1u));
                         if (lane == 0) {
 #pragma unroll
                             for (int q = 0; q < 4; ++q) ctl.mask[stage][tq][q] = words[q];
