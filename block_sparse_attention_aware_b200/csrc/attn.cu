@@ -76,6 +76,7 @@ struct AttnArgs {
     int nwords;                  // 32-bit words per bitmap, ceil(nb / 32)
     const uint32_t* gbits;       // [B*H][ngroups][G][nwords] (G > 1)
     const int32_t* gcnt;         // [B*H][ngroups] union sizes (G > 1)
+    const int32_t* ext;          // [nb] real extent of each block, packed as block_extent
     const int32_t* head_order;   // [B*H] heads, heaviest first
     const int32_t* item_order;   // [B*H][nb] query blocks of each head, longest first
     int* counter;                // next item to hand out
@@ -171,8 +172,9 @@ struct UnionWalk {
         rem = 0u;
         ahead = lane < G ? __ldg(maps + lane * nwords) : 0u;
     }
-    // Next union block j and its membership bits (bit t: in block t's list);
-    // false once the union is exhausted.  Warp-uniform.
+    // Next union block j and (when WANT_MEM) its membership bits (bit t: in
+    // block t's list); false once the union is exhausted.  Warp-uniform.
+    template <bool WANT_MEM>
     __device__ __forceinline__ bool next(int lane, int& j, uint32_t& mem) {
         while (rem == 0u) {
             if (++wi >= nwords) return false;
@@ -183,13 +185,14 @@ struct UnionWalk {
         const int bit = __ffs(static_cast<int>(rem)) - 1;
         rem &= rem - 1u;
         j = wi * 32 + bit;
-        mem = __ballot_sync(0xffffffffu, (word >> bit) & 1u);
+        if (WANT_MEM) mem = __ballot_sync(0xffffffffu, (word >> bit) & 1u);
         return true;
     }
 };
 
 // Slots of the next chunk of a group walk: lane s < (returned count) gets
-// slot s's block and membership bits.
+// slot s's block and (when WANT_MEM) membership bits.
+template <bool WANT_MEM>
 __device__ __forceinline__ int union_chunk(UnionWalk& u, int bpc, int lane, int& j, uint32_t& mem) {
     int n = 0;
     j = 0;
@@ -197,7 +200,8 @@ __device__ __forceinline__ int union_chunk(UnionWalk& u, int bpc, int lane, int&
     for (int s2 = 0; s2 < bpc; ++s2) {
         int jj;
         uint32_t mm;
-        if (!u.next(lane, jj, mm)) break;
+        mm = 0u;
+        if (!u.template next<WANT_MEM>(lane, jj, mm)) break;
         if (lane == s2) {
             j = jj;
             mem = mm;
@@ -352,7 +356,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
             int j_next = 0, n_next = 0;
             uint32_t m_next = 0u;
             if (GRP) {
-                n_next = union_chunk(uw, bpc, lane, j_next, m_next);
+                n_next = union_chunk<true>(uw, bpc, lane, j_next, m_next);
             } else {
                 n_next = min(bpc, cnt);
                 j_next = chunk_block(list, 0, bpc, n_next, lane, g.nb);
@@ -365,13 +369,13 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                 const uint32_t mem = m_next;
                 if (cl + 1 < nc) {
                     if (GRP) {
-                        n_next = union_chunk(uw, bpc, lane, j_next, m_next);
+                        n_next = union_chunk<true>(uw, bpc, lane, j_next, m_next);
                     } else {
                         n_next = min(bpc, cnt - (cl + 1) * bpc);
                         j_next = chunk_block(list, cl + 1, bpc, n_next, lane, g.nb);
                     }
                 }
-                const int ext = lane < nblk ? block_extent(g, j) : 0;
+                const int ext = lane < nblk ? __ldg(a.ext + j) : 0;
                 if (!wait_warp(smem_u32(&ctl.k_empty[stage]), ((c_seq / KS) & 1) ^ 1, abort_flag)) {
                     ok = false;
                     break;
@@ -449,7 +453,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
             int j_next = 0, n_next = 0;
             uint32_t m_unused = 0u;
             if (GRP) {
-                n_next = union_chunk(uw, bpc, lane, j_next, m_unused);
+                n_next = union_chunk<false>(uw, bpc, lane, j_next, m_unused);
             } else {
                 n_next = min(bpc, cnt);
                 j_next = chunk_block(list, 0, bpc, n_next, lane, g.nb);
@@ -460,7 +464,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                 const int j = j_next;
                 if (cl + 1 < nc) {
                     if (GRP) {
-                        n_next = union_chunk(uw, bpc, lane, j_next, m_unused);
+                        n_next = union_chunk<false>(uw, bpc, lane, j_next, m_unused);
                     } else {
                         n_next = min(bpc, cnt - (cl + 1) * bpc);
                         j_next = chunk_block(list, cl + 1, bpc, n_next, lane, g.nb);
@@ -956,9 +960,11 @@ __global__ void __launch_bounds__(256) worklist_head_kernel(Geo g, int units, co
 }
 
 // Single CTA: heads by total cost, heaviest first (ties by lower index);
-// resets the item counter.
-__global__ void __launch_bounds__(256) worklist_heads_kernel(int BH, const long long* __restrict__ head_cost,
-                                                             int32_t* __restrict__ head_order, int* counter) {
+// resets the item counter; writes every block's real extent.
+__global__ void __launch_bounds__(256) worklist_heads_kernel(Geo g, int BH, const long long* __restrict__ head_cost,
+                                                             int32_t* __restrict__ head_order, int* counter,
+                                                             int32_t* __restrict__ ext) {
+    for (int b = threadIdx.x; b < g.nb; b += blockDim.x) ext[b] = block_extent(g, b);
     for (int h = threadIdx.x; h < BH; h += blockDim.x) {
         const long long ch = head_cost[h];
         int rank = 0;
@@ -983,7 +989,7 @@ static bool make_tmap(CUtensorMap* m, const void* base, long long rows, int D, i
 // Workspace: work list (item order, head cost and order, counter) and, when
 // G = 128 / bs > 1, the query groups' membership bitmaps and union sizes.
 struct WsLayout {
-    size_t item_order, head_cost, head_order, counter, gbits, gcnt, total;
+    size_t item_order, head_cost, head_order, counter, ext, gbits, gcnt, total;
     int G, ngroups, nwords;
 };
 
@@ -999,7 +1005,8 @@ static WsLayout ws_layout(const fvattn_geom& g) {
     w.head_cost = al256(sizeof(int32_t) * BH * g.nb);
     w.head_order = w.head_cost + al256(sizeof(long long) * BH);
     w.counter = w.head_order + al256(sizeof(int32_t) * BH);
-    w.gbits = w.counter + 256;
+    w.ext = w.counter + 256;
+    w.gbits = w.ext + al256(sizeof(int32_t) * g.nb);
     w.gcnt = w.gbits;
     w.total = w.gbits;
     if (w.G > 1) {
@@ -1077,7 +1084,8 @@ static int attn_impl(const fvattn_geom* gp, const void* q_t, const void* k_t, co
     worklist_head_kernel<<<BH, 256, sizeof(int) * (g.nb + 2), s>>>(g, units, wl.G > 1 ? gcnt : kv_cnt, item_order,
                                                                    head_cost);
     FV_CHECK_LAUNCH();
-    worklist_heads_kernel<<<1, 256, 0, s>>>(BH, head_cost, head_order, counter);
+    int32_t* ext = reinterpret_cast<int32_t*>(ws + wl.ext);
+    worklist_heads_kernel<<<1, 256, 0, s>>>(g, BH, head_cost, head_order, counter, ext);
     FV_CHECK_LAUNCH();
 
     CUtensorMap tq, tk, tv;
@@ -1100,6 +1108,7 @@ static int attn_impl(const fvattn_geom* gp, const void* q_t, const void* k_t, co
     args.nwords = wl.nwords;
     args.gbits = gbits;
     args.gcnt = gcnt;
+    args.ext = ext;
     args.total_items = BH * units;
     int nsm = cached_num_sms();
     if (nsm <= 0) return FVATTN_ERR_CUDA;
