@@ -37,9 +37,9 @@ WORKLOAD = "720p"
 OTHER_KERNELS_PER_STEP = 7
 
 # DRAM bytes (read + write) of one sparse_attn_kernel<128, 0> launch on the 720p layer: an ncu capture
-# of the same layer restricted to 4 heads read 347.0 MB and wrote 74.4 MB; K/V reuse stays inside a
+# of the same layer restricted to 4 heads read 372.6 MB and wrote 74.3 MB; K/V reuse stays inside a
 # head, so traffic scales with the head count (x10 for 40 heads).
-ATTN_TRAFFIC_720P = {"bytes": (347.001088e6 + 74.445312e6) * 10,
+ATTN_TRAFFIC_720P = {"bytes": (372.626688e6 + 74.264064e6) * 10,
                      "how": "ncu dram__bytes_read.sum + dram__bytes_write.sum of the 4-head 720p layer, x10 heads"}
 
 
