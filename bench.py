@@ -33,8 +33,6 @@ if ROOT not in sys.path:
 METRIC = "sparse-attn TFLOPS on executed blocks (% of bf16 peak) + end-to-end ms per layer"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 WORKLOAD = "720p"
-# kernels per step besides routing's: reorder x3, 2 work-list kernels, attention, inverse reorder
-OTHER_KERNELS_PER_STEP = 7
 
 # DRAM bytes (read + write) of one sparse_attn_kernel<128, 0> launch on the 720p layer: an ncu capture
 # of the same layer restricted to 4 heads read 372.6 MB and wrote 74.3 MB; K/V reuse stays inside a
@@ -309,7 +307,8 @@ def run_fvattn(args):
     dev = torch.device("cuda", local)
     # each rank: its own seeded replica layer
     q, k, v, _ = synth.make_qkv(w, layer=rank, device=dev)
-    layer = fvattn.Layer(g, w.p, w.k, device=dev, order=args.order)
+    fused = not args.unfused_route
+    layer = fvattn.Layer(g, w.p, w.k, device=dev, order=args.order, fused_route=fused)
     g = layer.g
     stream = torch.cuda.current_stream(dev)
     nsm = fvattn.num_sms()
@@ -336,9 +335,14 @@ def run_fvattn(args):
     for i in range(args.steps):
         e = ev[i]
         e[0].record(stream)
-        layer.reorder_qkv(q, k, v)
-        e[1].record(stream)
-        layer.route()
+        if fused:
+            layer.reorder_route(q, k)
+            e[1].record(stream)
+            layer.reorder_v(v)
+        else:
+            layer.reorder_qkv(q, k, v)
+            e[1].record(stream)
+            layer.route()
         e[2].record(stream)
         layer.attend(stats=True)
         e[3].record(stream)
@@ -356,22 +360,43 @@ def run_fvattn(args):
     flops = 4.0 * g.bs * g.bs * g.D * pairs
     t_max, flops_all = aggregate_over_ranks(t_total, flops, world, dev)
 
-    stage = {n: [] for n in ("reorder_qkv", "route", "attention", "inverse_reorder")}
+    names = (("reorder_route_qk", "reorder_v") if fused else ("reorder_qkv", "route")) + \
+        ("attention", "inverse_reorder")
+    stage = {n: [] for n in names}
     for e in ev:
-        stage["reorder_qkv"].append(e[0].elapsed_time(e[1]))
-        stage["route"].append(e[1].elapsed_time(e[2]))
-        stage["attention"].append(e[2].elapsed_time(e[3]))
-        stage["inverse_reorder"].append(e[3].elapsed_time(e[4]))
+        for j, n in enumerate(names):
+            stage[n].append(e[j].elapsed_time(e[j + 1]))
     ms = {kk: statistics.mean(vv) for kk, vv in stage.items()}
+    if fused:
+        # routing alone (pooling from the tiles, scoring, selection) on the tiles the step wrote,
+        # for its own bandwidth figure; the same kv lists come out
+        r0, r1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        layer.route()
+        r0.record(stream)
+        for _ in range(args.steps):
+            layer.route()
+        r1.record(stream)
+        torch.cuda.synchronize()
+        ms["route_alone"] = r0.elapsed_time(r1) / args.steps
     peaks, peak_src = load_peaks()
     raster_bytes = g.B * g.N * g.H * g.D * 2
     tiled_bytes = g.B * g.H * g.Npad * g.D * 2
     attn_s = ms["attention"] / 1e3
     attn_tflops = flops / attn_s / 1e12
-    route_bytes = 2 * tiled_bytes * (g.N / g.Npad) + 4 * pairs + 4 * cnt.numel()
-    route_gbs = route_bytes / (ms["route"] / 1e3) / 1e9
-    reorder_gbs = 3 * (raster_bytes + tiled_bytes) / (ms["reorder_qkv"] / 1e3) / 1e9
+    kv_bytes = 4 * pairs + 4 * cnt.numel()
+    route_bytes = 2 * tiled_bytes * (g.N / g.Npad) + kv_bytes
+    route_gbs = route_bytes / (ms["route_alone" if fused else "route"] / 1e3) / 1e9
     inverse_gbs = (raster_bytes + tiled_bytes) / (ms["inverse_reorder"] / 1e3) / 1e9
+    gbs = {"route": route_gbs, "inverse_reorder": inverse_gbs,
+           "route_pct_of_hbm": 100.0 * route_gbs / peaks["hbm_gbs"]}
+    if fused:
+        # fused stage: raster Q, K read once, their tiles and the kv lists written
+        fr_bytes = 2 * (raster_bytes + tiled_bytes) + kv_bytes
+        gbs["reorder_route_qk"] = fr_bytes / (ms["reorder_route_qk"] / 1e3) / 1e9
+        gbs["reorder_route_qk_pct_of_hbm"] = 100.0 * gbs["reorder_route_qk"] / peaks["hbm_gbs"]
+        gbs["reorder_v"] = (raster_bytes + tiled_bytes) / (ms["reorder_v"] / 1e3) / 1e9
+    else:
+        gbs["reorder_qkv"] = 3 * (raster_bytes + tiled_bytes) / (ms["reorder_qkv"] / 1e3) / 1e9
     st = layer.sm_stats.cpu().numpy().astype(np.float64)
     busy, blocks = st[:nsm], st[nsm:2 * nsm]
     used = busy > 0
@@ -395,7 +420,8 @@ def run_fvattn(args):
                  + (", shared rank-8 spatio-temporal component" if w.lowrank else "")),
         "config": workload_config(w, g),
         "value_note": "executed-block attention FLOPs of all ranks / (max-over-ranks time of one whole "
-                      "layer step: reorder x3 + route + attention + inverse reorder)",
+                      "layer step: " + ("reorder+route of Q/K in one pass + reorder V" if fused else
+                                        "reorder x3 + route") + " + attention + inverse reorder)",
         "attention": {
             "tflops_executed_blocks": attn_tflops,
             "pct_of_bf16_peak_burst": 100.0 * attn_tflops / peaks["bf16_tflops"],
@@ -406,8 +432,7 @@ def run_fvattn(args):
             "head_blocks_max_over_mean": float(per_head.max() / per_head.mean()),
         },
         "stages_ms": ms,
-        "stages_gbs": {"reorder_qkv": reorder_gbs, "route": route_gbs, "inverse_reorder": inverse_gbs,
-                       "route_pct_of_hbm": 100.0 * route_gbs / peaks["hbm_gbs"]},
+        "stages_gbs": gbs,
         "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": sustained, "unit": "TFLOP/s",
                      "frac": attn_tflops / sustained,
                      "traffic": ATTN_TRAFFIC_720P["bytes"] if (w.name == "720p" and not args.heads) else None,
@@ -416,7 +441,7 @@ def run_fvattn(args):
                      "kernel": f"sparse_attn_kernel<{g.D}, {int(g.bs < 128)}>",
                      "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside back-to-back steps)",
                      "algorithmic_flops_per_launch": flops},
-        "gpu_launches": (OTHER_KERNELS_PER_STEP + fvattn.route_kernel_launches(g)) * args.steps,
+        "gpu_launches": layer.kernel_launches() * args.steps,
         "clocks": clock_info,
     }
 
@@ -429,6 +454,17 @@ def run_fvattn(args):
     ef1.record(stream)
     torch.cuda.synchronize()
     line["fused_inverse_step_ms"] = ef0.elapsed_time(ef1) / args.steps
+
+    # the step with the other routing path (separate reorders and routing, or the fused call)
+    layer.fused_route = not fused
+    layer(q, k, v)
+    ef0.record(stream)
+    for _ in range(args.steps):
+        layer(q, k, v)
+    ef1.record(stream)
+    torch.cuda.synchronize()
+    line["unfused_route_step_ms" if fused else "fused_route_step_ms"] = ef0.elapsed_time(ef1) / args.steps
+    layer.fused_route = fused
 
     # p sweep (load-skew workload): per p, one routed + attended step after one warm-up
     if w.p_sweep:
@@ -447,7 +483,8 @@ def run_fvattn(args):
         vh = v.cpu().pin_memory()
         oh = torch.empty_like(qh).pin_memory()
         groups = 4 if (g.H % 4 == 0 and g.H >= 8) else 1
-        pipe = fvattn.HostPipeline(fvattn.geom_of(w), w.p, w.k, groups=groups, device=dev, order=args.order)
+        pipe = fvattn.HostPipeline(fvattn.geom_of(w), w.p, w.k, groups=groups, device=dev, order=args.order,
+                                   fused_route=fused)
         pipe(qh, kh, vh, oh)
         torch.cuda.synchronize()
         barrier()
@@ -491,6 +528,8 @@ def main():
                     help="block order of the tiles (raster tile order or the 3-D Hilbert curve)")
     ap.add_argument("--stack", action="store_true",
                     help="also time every seeded layer of a multi-layer workload once (cfg720p: 40 layers)")
+    ap.add_argument("--unfused-route", action="store_true",
+                    help="time the step with separate reorders and routing instead of the fused call")
     ap.add_argument("--heads", type=int, default=0,
                     help="profiling-size variant: the same layer with fewer heads (0 = all)")
     args = ap.parse_args()

@@ -25,6 +25,11 @@
 //                  floor) is found the same way with counts when the Top-p
 //                  prefix is shorter.  No shared-memory atomics.  The kept
 //                  indices are written in ascending order with ballots.
+//
+// fvattn_reorder_route replaces the pooling kernel by reorder_pool_kernel,
+// which reads raster Q and K once, writes their tiles and pools the same rows
+// on the way (the reorder and pooling steps of the pages' pipeline in one
+// pass).
 #include <cstring>
 
 #include "common.cuh"
@@ -46,6 +51,58 @@ struct PoolOut {
     float* mean[2];   // [q, k]: the fp32 mean itself, or null
 };
 
+// Mean of a block's rows from the lanes' fp32 pair sums (lane l holds column
+// slice l % (D/8) of every (32 / (D/8))-th row): reduce across the lanes of a
+// slice, divide by the real-row count, write the tf32 part, the exact
+// remainder and, if asked, the mean.
+template <int D>
+__device__ __forceinline__ void pool_write(const unsigned long long (&acc2)[4], int lane, int real_rows,
+                                           long long dst_off, bool is_k, const PoolOut& out) {
+    constexpr int VPR = D / 8;
+    float acc[8];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) f2_unpack(acc2[e], acc[2 * e], acc[2 * e + 1]);
+    // lanes with the same column slice hold partial sums of different rows
+#pragma unroll
+    for (int o = VPR; o < 32; o <<= 1)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], o);
+    if (lane < VPR) {
+        const float inv = 1.0f / static_cast<float>(real_rows);
+        float m[8], h[8], l[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            m[e] = acc[e] * inv;
+            h[e] = __uint_as_float(__float_as_uint(m[e]) & 0xffffe000u);
+            l[e] = m[e] - h[e];
+        }
+        const long long o = dst_off + lane * 8;
+        float* mp = is_k ? out.mean[1] : out.mean[0];
+        float4* dh = reinterpret_cast<float4*>((is_k ? out.hi[1] : out.hi[0]) + o);
+        float4* dl = reinterpret_cast<float4*>((is_k ? out.lo[1] : out.lo[0]) + o);
+        dh[0] = make_float4(h[0], h[1], h[2], h[3]);
+        dh[1] = make_float4(h[4], h[5], h[6], h[7]);
+        dl[0] = make_float4(l[0], l[1], l[2], l[3]);
+        dl[1] = make_float4(l[4], l[5], l[6], l[7]);
+        if (mp) {
+            float4* dm = reinterpret_cast<float4*>(mp + o);
+            dm[0] = make_float4(m[0], m[1], m[2], m[3]);
+            dm[1] = make_float4(m[4], m[5], m[6], m[7]);
+        }
+    }
+}
+
+// Adds the 8 bf16 of a 16-byte vector to the lane's fp32 pair sums.
+__device__ __forceinline__ void pool_add(unsigned long long (&acc2)[4], const uint4& u) {
+    const uint32_t wds[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        // a bf16 is the top half of the fp32 with the same value
+        const float lo = __uint_as_float(wds[e] << 16), hi = __uint_as_float(wds[e] & 0xffff0000u);
+        acc2[e] = f2_add(acc2[e], f2_pack(lo, hi));
+    }
+}
+
 template <int D>
 __global__ void __launch_bounds__(256, 4) pool_kernel(Geo g, const __nv_bfloat16* __restrict__ qt,
                                                    const __nv_bfloat16* __restrict__ kt, PoolOut out) {
@@ -63,7 +120,6 @@ __global__ void __launch_bounds__(256, 4) pool_kernel(Geo g, const __nv_bfloat16
     const int blk = static_cast<int>(ub - bh * g.nb);
     const uint4* src = reinterpret_cast<const uint4*>((is_k ? kt : qt) +
                                                       (bh * g.Npad + static_cast<long long>(blk) * g.bs) * D);
-    const long long dst_off = (bh * g.nb + blk) * D;
     const int vec = lane % VPR;
     const int r0 = lane / VPR;
     const int tile = tile_of_block(g, blk);
@@ -94,47 +150,77 @@ __global__ void __launch_bounds__(256, 4) pool_kernel(Geo g, const __nv_bfloat16
             }
         }
 #pragma unroll
-        for (int i = 0; i < UNR; ++i) {
-            const uint32_t wds[4] = {u[i].x, u[i].y, u[i].z, u[i].w};
+        for (int i = 0; i < UNR; ++i) pool_add(acc2, u[i]);
+    }
+    pool_write<D>(acc2, lane, nf * ny * nx, (bh * g.nb + blk) * D, is_k, out);
+}
+
+// Reorder and pooling in one pass over raster Q and K.  One warp per (tensor,
+// b, block, h) unit, h fastest, so the warps running at one time read every
+// head of the same raster tokens (contiguous H * D runs) instead of one
+// 2*D-byte row every H * 2*D bytes.  The warp copies the block's bs raster rows into
+// its tile, 32 tile rows a round (padding rows written as zeros), and adds
+// each loaded vector to its pair sums.  Lane l always holds column slice
+// l % (D/8) and meets its rows in increasing order, exactly as in
+// pool_kernel, so the means are bit-identical to pooling the tiles after a
+// separate reorder.  Two CTAs per SM (at most 128 registers a thread) keep
+// 16 warps x 8 KB of loads in flight per SM; one CTA (the unbounded
+// allocation) halves that and the bandwidth with it.
+template <int D>
+__global__ void __launch_bounds__(256, 2) reorder_pool_kernel(Geo g, const uint4* __restrict__ q,
+                                                           const uint4* __restrict__ k, uint4* __restrict__ qt,
+                                                           uint4* __restrict__ kt, PoolOut out) {
+    constexpr int VPR = D / 8;             // 16-byte vectors per row
+    constexpr int RPI = 32 / VPR;          // rows per warp instruction
+    pdl_launch_dependents();   // the score kernel may be scheduled as this grid drains
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const long long unit = static_cast<long long>(blockIdx.x) * 8 + warp;
+    const long long per_tensor = static_cast<long long>(g.B) * g.H * g.nb;
+    if (unit >= 2 * per_tensor) return;
+    const bool is_k = unit >= per_tensor;
+    const long long ub = is_k ? unit - per_tensor : unit;
+    const int h = static_cast<int>(ub % g.H);
+    const long long bblk = ub / g.H;                       // b * nb + block
+    const int blk = static_cast<int>(bblk % g.nb);
+    const int b = static_cast<int>(bblk / g.nb);
+    const long long bh = static_cast<long long>(b) * g.H + h;
+    const uint4* src = is_k ? k : q;
+    uint4* dst = (is_k ? kt : qt) + (bh * g.Npad + static_cast<long long>(blk) * g.bs) * VPR;
+    const int tile = tile_of_block(g, blk);
+    const int bx = tile % g.nbx, by = (tile / g.nbx) % g.nby, bf = tile / (g.nbx * g.nby);
+    const int nf = min(g.tf, g.F - bf * g.tf);
+    const int ny = min(g.th, g.Hs - by * g.th);
+    const int nx = min(g.tw, g.Ws - bx * g.tw);
+    const int vec = lane % VPR;
+    unsigned long long acc2[4];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                // a bf16 is the top half of the fp32 with the same value
-                const float lo = __uint_as_float(wds[e] << 16), hi = __uint_as_float(wds[e] & 0xffff0000u);
-                acc2[e] = f2_add(acc2[e], f2_pack(lo, hi));
+    for (int e = 0; e < 4; ++e) acc2[e] = 0ull;
+    for (int r32 = 0; r32 < g.bs; r32 += 32) {
+        // raster row of tile row r32 + lane, or -1 (padding, or past the tile when bs = 16)
+        long long s_row = -1;
+        const int o = r32 + lane;
+        if (o < g.bs) {
+            const int ox = o % g.tw, oy = (o / g.tw) % g.th, of = o / (g.tw * g.th);
+            if (of < nf && oy < ny && ox < nx) {
+                const long long n =
+                    (static_cast<long long>(bf * g.tf + of) * g.Hs + by * g.th + oy) * g.Ws + bx * g.tw + ox;
+                s_row = (static_cast<long long>(b) * g.N + n) * g.H + h;
             }
         }
-    }
-    float acc[8];
+        uint4 v[VPR];   // 32 rows x VPR vectors over 32 lanes, all in flight
 #pragma unroll
-    for (int e = 0; e < 4; ++e) f2_unpack(acc2[e], acc[2 * e], acc[2 * e + 1]);
-    // lanes with the same column slice hold partial sums of different rows
-#pragma unroll
-    for (int o = VPR; o < 32; o <<= 1)
-#pragma unroll
-        for (int e = 0; e < 8; ++e) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], o);
-    if (lane < VPR) {
-        const float inv = 1.0f / static_cast<float>(nf * ny * nx);
-        float m[8], h[8], l[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            m[e] = acc[e] * inv;
-            h[e] = __uint_as_float(__float_as_uint(m[e]) & 0xffffe000u);
-            l[e] = m[e] - h[e];
+        for (int it = 0; it < VPR; ++it) {
+            const long long sr = __shfl_sync(0xffffffffu, s_row, it * RPI + lane / VPR);
+            v[it] = sr >= 0 ? __ldg(src + sr * VPR + vec) : make_uint4(0, 0, 0, 0);
         }
-        const long long o = dst_off + lane * 8;
-        float* mp = is_k ? out.mean[1] : out.mean[0];
-        float4* dh = reinterpret_cast<float4*>((is_k ? out.hi[1] : out.hi[0]) + o);
-        float4* dl = reinterpret_cast<float4*>((is_k ? out.lo[1] : out.lo[0]) + o);
-        dh[0] = make_float4(h[0], h[1], h[2], h[3]);
-        dh[1] = make_float4(h[4], h[5], h[6], h[7]);
-        dl[0] = make_float4(l[0], l[1], l[2], l[3]);
-        dl[1] = make_float4(l[4], l[5], l[6], l[7]);
-        if (mp) {
-            float4* dm = reinterpret_cast<float4*>(mp + o);
-            dm[0] = make_float4(m[0], m[1], m[2], m[3]);
-            dm[1] = make_float4(m[4], m[5], m[6], m[7]);
+#pragma unroll
+        for (int it = 0; it < VPR; ++it) {
+            const int r = r32 + it * RPI + lane / VPR;
+            if (r < g.bs) dst[static_cast<long long>(r) * VPR + vec] = v[it];
+            pool_add(acc2, v[it]);
         }
     }
+    pool_write<D>(acc2, lane, nf * ny * nx, (bh * g.nb + blk) * D, is_k, out);
 }
 
 // ------------------------------------------------------------------ scoring
@@ -676,11 +762,17 @@ extern "C" int fvattn_route_kernel_launches(const fvattn_geom* gp) {
     return 3;   // pool, score, select
 }
 
-static int route_impl(const fvattn_geom* gp, const void* q_tiled, const void* k_tiled, double p, int k_floor,
-                      int k_extra, float scale, int32_t* kv_idx, int32_t* kv_cnt, float* q_pool, float* k_pool,
-                      float* logits, void* workspace, size_t ws_bytes, fvattn_stream_t stream) {
+// Pooling (from the tiles, or fused with the reorder when raster Q and K are
+// given, which then writes the tiles), scoring and selection.
+static int route_impl(const fvattn_geom* gp, const void* q_raster, const void* k_raster, const void* q_tiled,
+                      const void* k_tiled, double p, int k_floor, int k_extra, float scale, int32_t* kv_idx,
+                      int32_t* kv_cnt, float* q_pool, float* k_pool, float* logits, void* workspace,
+                      size_t ws_bytes, fvattn_stream_t stream) {
     if (!gp || !q_tiled || !k_tiled || !kv_idx || !kv_cnt) return FVATTN_ERR_INVALID;
     if (!aligned16(q_tiled) || !aligned16(k_tiled) || !aligned16(kv_idx) || !aligned16(kv_cnt))
+        return FVATTN_ERR_INVALID;
+    const bool fused = q_raster != nullptr || k_raster != nullptr;
+    if (fused && (!q_raster || !k_raster || !aligned16(q_raster) || !aligned16(k_raster) || q_tiled == k_tiled))
         return FVATTN_ERR_INVALID;
     if (!(p >= 0.0 && p <= 1.0) || k_floor < 1 || k_extra < 0 || !isfinite(scale)) return FVATTN_ERR_INVALID;
     if (gp->nb <= 0 || gp->nb > 2560) return FVATTN_ERR_UNSUPPORTED;
@@ -703,12 +795,20 @@ static int route_impl(const fvattn_geom* gp, const void* q_tiled, const void* k_
     po.mean[1] = k_pool;
     const long long units = 2ll * g.B * g.H * g.nb;
     const unsigned pblocks = static_cast<unsigned>((units + 7) / 8);
-    if (g.D == 128)
+    if (fused) {
+        const uint4 *qr = static_cast<const uint4*>(q_raster), *kr = static_cast<const uint4*>(k_raster);
+        uint4 *qw = static_cast<uint4*>(const_cast<void*>(q_tiled)), *kw = static_cast<uint4*>(const_cast<void*>(k_tiled));
+        if (g.D == 128)
+            reorder_pool_kernel<128><<<pblocks, 256, 0, s>>>(g, qr, kr, qw, kw, po);
+        else
+            reorder_pool_kernel<64><<<pblocks, 256, 0, s>>>(g, qr, kr, qw, kw, po);
+    } else if (g.D == 128) {
         pool_kernel<128><<<pblocks, 256, 0, s>>>(g, static_cast<const __nv_bfloat16*>(q_tiled),
                                                  static_cast<const __nv_bfloat16*>(k_tiled), po);
-    else
+    } else {
         pool_kernel<64><<<pblocks, 256, 0, s>>>(g, static_cast<const __nv_bfloat16*>(q_tiled),
                                                 static_cast<const __nv_bfloat16*>(k_tiled), po);
+    }
     FV_CHECK_LAUNCH();
 
     const unsigned long long prow = static_cast<unsigned long long>(g.B) * g.H * g.nb;
@@ -774,14 +874,23 @@ extern "C" int fvattn_route(const fvattn_geom* gp, const void* q_tiled, const vo
                             float scale, int32_t* kv_idx, int32_t* kv_cnt, float* q_pool, float* k_pool,
                             float* logits, void* workspace, size_t ws_bytes, fvattn_stream_t stream) {
     if (!(p > 0.0)) return FVATTN_ERR_INVALID;
-    return route_impl(gp, q_tiled, k_tiled, p, k_floor, 0, scale, kv_idx, kv_cnt, q_pool, k_pool, logits, workspace,
-                      ws_bytes, stream);
+    return route_impl(gp, nullptr, nullptr, q_tiled, k_tiled, p, k_floor, 0, scale, kv_idx, kv_cnt, q_pool, k_pool,
+                      logits, workspace, ws_bytes, stream);
 }
 
 extern "C" int fvattn_route_aug(const fvattn_geom* gp, const void* q_tiled, const void* k_tiled, double p,
                                 int k_floor, int k_extra, float scale, int32_t* kv_idx, int32_t* kv_cnt,
                                 float* q_pool, float* k_pool, float* logits, void* workspace, size_t ws_bytes,
                                 fvattn_stream_t stream) {
-    return route_impl(gp, q_tiled, k_tiled, p, k_floor, k_extra, scale, kv_idx, kv_cnt, q_pool, k_pool, logits,
+    return route_impl(gp, nullptr, nullptr, q_tiled, k_tiled, p, k_floor, k_extra, scale, kv_idx, kv_cnt, q_pool,
+                      k_pool, logits, workspace, ws_bytes, stream);
+}
+
+extern "C" int fvattn_reorder_route(const fvattn_geom* gp, const void* q, const void* k, void* q_tiled,
+                                    void* k_tiled, double p, int k_floor, int k_extra, float scale, int32_t* kv_idx,
+                                    int32_t* kv_cnt, float* q_pool, float* k_pool, float* logits, void* workspace,
+                                    size_t ws_bytes, fvattn_stream_t stream) {
+    if (!q || !k) return FVATTN_ERR_INVALID;
+    return route_impl(gp, q, k, q_tiled, k_tiled, p, k_floor, k_extra, scale, kv_idx, kv_cnt, q_pool, k_pool, logits,
                       workspace, ws_bytes, stream);
 }

@@ -22,6 +22,7 @@ _lib = None
 OK, ERR_INVALID, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_BOUNDS = range(6)
 EXPORTED = ("fvattn_geom_init", "fvattn_block_order", "fvattn_copy_heads", "fvattn_reorder", "fvattn_inverse_reorder",
             "fvattn_route_workspace_size", "fvattn_route_kernel_launches", "fvattn_route", "fvattn_route_aug",
+            "fvattn_reorder_route",
             "fvattn_attn_workspace_size",
             "fvattn_num_sms", "fvattn_sparse_attn", "fvattn_sparse_attn_raster", "fvattn_sparse_attn_noalloc",
             "fvattn_get_status",
@@ -71,6 +72,9 @@ def load(path: str = LIB_PATH):
     L.fvattn_route.restype = I
     L.fvattn_route_aug.argtypes = [G, P, P, ctypes.c_double, I, I, ctypes.c_float, P, P, P, P, P, P, S, P]
     L.fvattn_route_aug.restype = I
+    L.fvattn_reorder_route.argtypes = [G, P, P, P, P, ctypes.c_double, I, I, ctypes.c_float, P, P, P, P, P, P, S,
+                                       P]
+    L.fvattn_reorder_route.restype = I
     L.fvattn_attn_workspace_size.argtypes = [G]
     L.fvattn_attn_workspace_size.restype = S
     L.fvattn_num_sms.argtypes = []
@@ -193,6 +197,16 @@ def attn_workspace(g: Geom, device="cuda") -> torch.Tensor:
     return torch.empty(max(n, 256), dtype=torch.uint8, device=device)
 
 
+def _route_out(g: Geom, dev, debug: bool) -> RouteOut:
+    out = RouteOut(kv_idx=torch.empty((g.B, g.H, g.nb, g.nb), dtype=torch.int32, device=dev),
+                   kv_cnt=torch.empty((g.B, g.H, g.nb), dtype=torch.int32, device=dev))
+    if debug:
+        out.q_pool = torch.empty((g.B, g.H, g.nb, g.D), dtype=torch.float32, device=dev)
+        out.k_pool = torch.empty_like(out.q_pool)
+        out.logits = torch.empty((g.B, g.H, g.nb, g.nb), dtype=torch.float32, device=dev)
+    return out
+
+
 def route(g: Geom, qt: torch.Tensor, kt: torch.Tensor, p: float, k: int,
           scale: Optional[float] = None, debug: bool = False, out: Optional[RouteOut] = None,
           workspace: Optional[torch.Tensor] = None, stream=None, k_extra: int = 0) -> RouteOut:
@@ -204,12 +218,7 @@ def route(g: Geom, qt: torch.Tensor, kt: torch.Tensor, p: float, k: int,
     if scale is None:
         scale = 1.0 / math.sqrt(g.D)
     if out is None:
-        out = RouteOut(kv_idx=torch.empty((g.B, g.H, g.nb, g.nb), dtype=torch.int32, device=dev),
-                       kv_cnt=torch.empty((g.B, g.H, g.nb), dtype=torch.int32, device=dev))
-        if debug:
-            out.q_pool = torch.empty((g.B, g.H, g.nb, g.D), dtype=torch.float32, device=dev)
-            out.k_pool = torch.empty_like(out.q_pool)
-            out.logits = torch.empty((g.B, g.H, g.nb, g.nb), dtype=torch.float32, device=dev)
+        out = _route_out(g, dev, debug)
     if workspace is None:
         workspace = route_workspace(g, dev)
     if k_extra or p == 0:
@@ -225,6 +234,32 @@ def route(g: Geom, qt: torch.Tensor, kt: torch.Tensor, p: float, k: int,
                                  0 if workspace is None else workspace.numel(), _stream(stream))
         _check("fvattn_route", rc)
     return out
+
+
+def reorder_route(g: Geom, q: torch.Tensor, k: torch.Tensor, p: float, kf: int,
+                  scale: Optional[float] = None, debug: bool = False, out: Optional[RouteOut] = None,
+                  qt: Optional[torch.Tensor] = None, kt: Optional[torch.Tensor] = None,
+                  workspace: Optional[torch.Tensor] = None, stream=None, k_extra: int = 0):
+    """fvattn_reorder_route: raster Q, K -> their tiles and the kv lists in
+    one pass over Q and K.  Returns (qt, kt, RouteOut)."""
+    _need_cuda(q, k, qt, kt)
+    for x in (q, k):
+        assert x.dtype == torch.bfloat16 and tuple(x.shape) == (g.B, g.N, g.H, g.D)
+    dev = q.device
+    if scale is None:
+        scale = 1.0 / math.sqrt(g.D)
+    if out is None:
+        out = _route_out(g, dev, debug)
+    qt = tiled_empty(g, dev) if qt is None else qt
+    kt = tiled_empty(g, dev) if kt is None else kt
+    if workspace is None:
+        workspace = route_workspace(g, dev)
+    rc = load().fvattn_reorder_route(ctypes.byref(g), _ptr(q), _ptr(k), _ptr(qt), _ptr(kt), float(p), int(kf),
+                                     int(k_extra), float(scale), _ptr(out.kv_idx), _ptr(out.kv_cnt),
+                                     _ptr(out.q_pool), _ptr(out.k_pool), _ptr(out.logits), _ptr(workspace),
+                                     workspace.numel(), _stream(stream))
+    _check("fvattn_reorder_route", rc)
+    return qt, kt, out
 
 
 def sparse_attn(g: Geom, qt, kt, vt, kv_idx, kv_cnt, scale: Optional[float] = None,
@@ -299,15 +334,18 @@ def get_status(stream=None) -> int:
 class Layer:
     """One attention layer's buffers, allocated once and reused: the four C
     ABI calls in order (reorder Q, K, V -> route -> sparse attention ->
-    inverse reorder)."""
+    inverse reorder).  With fused_route (the default) the reorder of Q and K
+    and the routing are one call, fvattn_reorder_route, which reads Q and K
+    once; the results are the same bits as the separate calls."""
 
     def __init__(self, g: Geom, p: float, k: int, scale: Optional[float] = None, device="cuda",
-                 debug: bool = False, order: str = "raster"):
+                 debug: bool = False, order: str = "raster", fused_route: bool = True):
         if order not in ("raster", "hilbert"):
             raise ValueError(f"block order {order!r}")
         self.order_table = block_order(g, device) if order == "hilbert" else None
         g = with_order(g, self.order_table)
         self.g, self.p, self.k = g, p, k
+        self.fused_route = fused_route
         self.scale = 1.0 / math.sqrt(g.D) if scale is None else scale
         self.qt = tiled_empty(g, device)
         self.kt = tiled_empty(g, device)
@@ -331,6 +369,23 @@ class Layer:
         return route(self.g, self.qt, self.kt, self.p, self.k, self.scale, out=self.routed,
                      workspace=self.route_ws, stream=stream)
 
+    def reorder_route(self, q, k, stream=None):
+        """Q and K reordered and routed in one pass (fvattn_reorder_route)."""
+        reorder_route(self.g, q, k, self.p, self.k, self.scale, out=self.routed, qt=self.qt, kt=self.kt,
+                      workspace=self.route_ws, stream=stream)
+        return self.routed
+
+    def reorder_v(self, v, stream=None):
+        reorder(self.g, v, self.vt, stream)
+
+    def kernel_launches(self) -> int:
+        """Kernels one __call__ (unfused inverse) launches: reorders, routing,
+        the work list (plus the query-group bitmaps for bs < 128), attention,
+        inverse reorder."""
+        reorders = 1 if self.fused_route else 3
+        worklist = 2 + (1 if self.g.bs < 128 else 0)
+        return reorders + route_kernel_launches(self.g) + worklist + 1 + 1
+
     def attend(self, stats: bool = False, stream=None):
         return sparse_attn(self.g, self.qt, self.kt, self.vt, self.routed.kv_idx, self.routed.kv_cnt,
                            self.scale, out=self.ot, sm_stats=self.sm_stats if stats else None,
@@ -346,8 +401,12 @@ class Layer:
                                   workspace=self.attn_ws, stream=stream)
 
     def __call__(self, q, k, v, stats: bool = False, stream=None, fused_inverse: bool = False):
-        self.reorder_qkv(q, k, v, stream)
-        self.route(stream)
+        if self.fused_route:
+            self.reorder_route(q, k, stream)
+            self.reorder_v(v, stream)
+        else:
+            self.reorder_qkv(q, k, v, stream)
+            self.route(stream)
         if fused_inverse:
             return self.attend_raster(stats, stream)
         self.attend(stats, stream)
@@ -363,12 +422,14 @@ class HostPipeline:
     compute stream) and the download of slice i-1 (another copy stream)
     overlap.  The output equals one whole-layer call bit for bit."""
 
-    def __init__(self, g: Geom, p: float, k: int, groups: int = 4, device="cuda", order: str = "raster"):
+    def __init__(self, g: Geom, p: float, k: int, groups: int = 4, device="cuda", order: str = "raster",
+                 fused_route: bool = True):
         if g.H % groups:
             raise ValueError(f"{g.H} heads do not split into {groups} equal groups")
         self.g, self.groups, self.nh = g, groups, g.H // groups
         gs = geom(g.B, self.nh, g.D, g.F, g.Hs, g.Ws, g.tf, g.th, g.tw)
-        self.layers = [Layer(gs, p, k, device=device, order=order) for _ in range(min(2, groups))]
+        self.layers = [Layer(gs, p, k, device=device, order=order, fused_route=fused_route)
+                       for _ in range(min(2, groups))]
         shape = (g.B, g.N, self.nh, g.D)
         self.inputs = [[torch.empty(shape, dtype=torch.bfloat16, device=device) for _ in range(3)]
                        for _ in self.layers]

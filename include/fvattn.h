@@ -162,6 +162,26 @@ int fvattn_route_aug(const fvattn_geom *g, const void *q_tiled, const void *k_ti
                      float *q_pool, float *k_pool, float *logits,
                      void *workspace, size_t ws_bytes, fvattn_stream_t stream);
 
+/* Reorder of Q and K fused with routing (paperlayer.ai summary, section 3,
+ * "Pipeline": the video-aware reorder comes first and the sparse-routing
+ * frontend pools the reordered blocks; here both happen in one pass over
+ * the raster tensors, which are read once).
+ *   q, k              raster [B, N, H, D] bf16 device tensors (as for
+ *                     fvattn_reorder), 16-byte aligned, read only
+ *   q_tiled, k_tiled  tiled [B, H, Npad, D] bf16 outputs, two distinct
+ *                     buffers: bit for bit what fvattn_reorder writes
+ *   the rest          as fvattn_route_aug.
+ * The pooled means are bit-identical to pooling the tiles afterwards, so
+ * kv_idx / kv_cnt equal those of fvattn_reorder x 2 + fvattn_route_aug on
+ * the same inputs.  Launches fvattn_route_kernel_launches kernels.  Null or
+ * misaligned pointers, q_tiled == k_tiled, and the parameter errors of
+ * fvattn_route_aug return FVATTN_ERR_INVALID before any launch. */
+int fvattn_reorder_route(const fvattn_geom *g, const void *q, const void *k, void *q_tiled, void *k_tiled,
+                         double p, int k_floor, int k_extra, float scale,
+                         int32_t *kv_idx, int32_t *kv_cnt,
+                         float *q_pool, float *k_pool, float *logits,
+                         void *workspace, size_t ws_bytes, fvattn_stream_t stream);
+
 /* Host <-> device copy of a head slice of a raster tensor, for pipelining a
  * layer by head groups (plumbing; no part of the method).  Heads
  * [h0, h0 + nh) of a raster [B, N, H, D] bf16 tensor in host memory (page

@@ -27,7 +27,7 @@ def _declared():
 def test_exports_every_declared_symbol(fv):
     lib = fv.load()
     names = _declared()
-    assert len(names) == 16
+    assert len(names) == 17
     assert sorted(fv.EXPORTED) == names
     for n in names:
         assert hasattr(lib, n), n
@@ -76,6 +76,20 @@ def test_null_and_misaligned_pointers_rejected(fv):
     assert lib.fvattn_route_aug(gp, ctypes.c_void_p(16), ctypes.c_void_p(32), 1.5, 1, 0, 0.125, ctypes.c_void_p(48),
                                 ctypes.c_void_p(64), None, None, None, ctypes.c_void_p(256), 1 << 30,
                                 None) == fv.ERR_INVALID
+    # fused reorder + routing: raster pointers, two distinct tile buffers, the route_aug parameter checks
+    V = ctypes.c_void_p
+    assert lib.fvattn_reorder_route(gp, None, V(16), V(32), V(48), 0.9, 1, 0, 0.125, V(64), V(80), None, None,
+                                    None, V(256), 1 << 30, None) == fv.ERR_INVALID
+    assert lib.fvattn_reorder_route(gp, V(16), V(24), V(32), V(48), 0.9, 1, 0, 0.125, V(64), V(80), None, None,
+                                    None, V(256), 1 << 30, None) == fv.ERR_INVALID
+    assert lib.fvattn_reorder_route(gp, V(16), V(32), V(48), V(48), 0.9, 1, 0, 0.125, V(64), V(80), None, None,
+                                    None, V(256), 1 << 30, None) == fv.ERR_INVALID
+    assert lib.fvattn_reorder_route(gp, V(16), V(32), V(48), V(64), 1.5, 1, 0, 0.125, V(80), V(96), None, None,
+                                    None, V(256), 1 << 30, None) == fv.ERR_INVALID
+    assert lib.fvattn_reorder_route(gp, V(16), V(32), V(48), V(64), 0.9, 1, -2, 0.125, V(80), V(96), None, None,
+                                    None, V(256), 1 << 30, None) == fv.ERR_INVALID
+    assert lib.fvattn_reorder_route(gp, V(16), V(32), V(48), V(64), 0.9, 1, 0, 0.125, V(80), V(96), None, None,
+                                    None, V(256), 16, None) == fv.ERR_INVALID
     # workspace too small
     assert lib.fvattn_route(gp, ctypes.c_void_p(16), ctypes.c_void_p(32), 0.9, 1, 0.125, ctypes.c_void_p(48),
                             ctypes.c_void_p(64), None, None, None, ctypes.c_void_p(256), 16, None) == fv.ERR_INVALID

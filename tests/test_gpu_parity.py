@@ -197,6 +197,10 @@ def test_sparse_attention_parity(fv, orc, name, w):
     st = layer.sm_stats.cpu().numpy()
     n = fv.num_sms()
     assert st[n:2 * n].sum() == _walked_blocks(g, layer.routed.kv_idx, layer.routed.kv_cnt)
+    # the layer with separate reorders and routing writes the same bits
+    out2 = fv.Layer(g, w.p, w.k, fused_route=False)(q, k, v)
+    torch.cuda.synchronize()
+    assert torch.equal(out2.view(torch.int16), out.view(torch.int16))
 
 
 @pytest.mark.parametrize("p,k", [(1.0, 1), (0.3, 1), (0.9, 10_000), (0.5, 3)])
@@ -307,6 +311,46 @@ def test_host_pipeline_matches_whole_layer(fv, groups):
     torch.cuda.synchronize()
     assert fv.get_status() == 0
     assert torch.equal(oh.view(torch.int16), want.view(torch.int16))
+
+
+FUSED = SMALL + HILBERT[:3]
+
+
+@pytest.mark.parametrize("name,w", FUSED, ids=[s[0] for s in FUSED])
+def test_reorder_route_matches_separate_calls(fv, orc, name, w):
+    """fvattn_reorder_route (reorder of Q and K fused with pooling, then
+    scoring and selection) against fvattn_reorder x 2 + fvattn_route: tiles,
+    pooled means, logits and kv lists are the same bits, and the tiles equal
+    the oracle's reorder."""
+    g = fv.geom_of(w)
+    table = fv.block_order(g) if w.order == "hilbert" else None
+    g = fv.with_order(g, table)
+    q, k, _ = _gpu_inputs(w)
+    for k_extra in (0, 2):
+        qt, kt = fv.reorder(g, q), fv.reorder(g, k)
+        sep = fv.route(g, qt, kt, w.p, w.k, debug=True, k_extra=k_extra)
+        qt2 = torch.full_like(qt, float("nan"))
+        kt2 = torch.full_like(kt, float("nan"))
+        qt2, kt2, fus = fv.reorder_route(g, q, k, w.p, w.k, debug=True, qt=qt2, kt=kt2, k_extra=k_extra)
+        torch.cuda.synchronize()
+        assert fv.get_status() == 0
+        assert torch.equal(qt2.view(torch.int16), qt.view(torch.int16))
+        assert torch.equal(kt2.view(torch.int16), kt.view(torch.int16))
+        for a, b in ((fus.q_pool, sep.q_pool), (fus.k_pool, sep.k_pool), (fus.logits, sep.logits)):
+            assert torch.equal(a.view(torch.int32), b.view(torch.int32))
+        assert torch.equal(fus.kv_cnt, sep.kv_cnt)
+        cnt = fus.kv_cnt.cpu().numpy().reshape(-1)
+        used = np.arange(g.nb)[None, :] < cnt[:, None]
+        a = fus.kv_idx.cpu().numpy().reshape(-1, g.nb)
+        b = sep.kv_idx.cpu().numpy().reshape(-1, g.nb)
+        assert np.array_equal(a[used], b[used])
+    assert np.array_equal(_bits(qt2), orc.reorder(_bits(q), w))
+    assert np.array_equal(_bits(kt2), orc.reorder(_bits(k), w))
+    kp_o = orc.pool(_bits(kt2), w)
+    got = fus.k_pool.cpu().numpy().astype(np.float64)
+    assert np.max(np.abs(got - kp_o)) <= 1e-5 * np.sqrt(np.mean(kp_o ** 2)) + 1e-6
+    bad, unexcused, _ = _check_mask(orc, fus.logits, fus.kv_idx, fus.kv_cnt, w.p, w.k, 2)
+    assert unexcused == []
 
 
 @pytest.mark.parametrize("p,k,k_extra", [(0.0, 3, 0), (0.0, 1, 2), (0.7, 2, 3), (0.9, 1, 10_000)])
