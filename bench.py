@@ -35,9 +35,9 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 WORKLOAD = "720p"
 
 # DRAM bytes (read + write) of one sparse_attn_kernel<128, 0> launch on the 720p layer: an ncu capture
-# of the same layer restricted to 4 heads read 372.6 MB and wrote 74.3 MB; K/V reuse stays inside a
+# of the same layer restricted to 4 heads read 338.6 MB and wrote 74.8 MB; K/V reuse stays inside a
 # head, so traffic scales with the head count (x10 for 40 heads).
-ATTN_TRAFFIC_720P = {"bytes": (372.626688e6 + 74.264064e6) * 10,
+ATTN_TRAFFIC_720P = {"bytes": (338.585856e6 + 74.816256e6) * 10,
                      "how": "ncu dram__bytes_read.sum + dram__bytes_write.sum of the 4-head 720p layer, x10 heads"}
 
 
@@ -482,7 +482,7 @@ def run_fvattn(args):
         kh = k.cpu().pin_memory()
         vh = v.cpu().pin_memory()
         oh = torch.empty_like(qh).pin_memory()
-        groups = 4 if (g.H % 4 == 0 and g.H >= 8) else 1
+        groups = args.e2e_groups if (g.H % args.e2e_groups == 0 and g.H >= 2 * args.e2e_groups) else 1
         pipe = fvattn.HostPipeline(fvattn.geom_of(w), w.p, w.k, groups=groups, device=dev, order=args.order,
                                    fused_route=fused)
         pipe(qh, kh, vh, oh)
@@ -528,6 +528,8 @@ def main():
                     help="block order of the tiles (raster tile order or the 3-D Hilbert curve)")
     ap.add_argument("--stack", action="store_true",
                     help="also time every seeded layer of a multi-layer workload once (cfg720p: 40 layers)")
+    ap.add_argument("--e2e-groups", type=int, default=20,
+                    help="head groups of the end-to-end pipeline (uploads, compute and downloads overlap)")
     ap.add_argument("--unfused-route", action="store_true",
                     help="time the step with separate reorders and routing instead of the fused call")
     ap.add_argument("--heads", type=int, default=0,

@@ -788,7 +788,10 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
             // a group with no chunk in this item has l = 0 and m = -inf: weight 0
             const float a0 = l0 > 0.f ? ex2_approx(m0 - mm) : 0.f;
             const float a1 = l1 > 0.f ? ex2_approx(m1 - mm) : 0.f;
-            const float inv = 1.0f / (l0 * a0 + l1 * a1);
+            // Which group holds which half of an item's chunks follows the CTA's chunk count, so the
+            // merge is written symmetric in the two groups (products rounded separately, one add;
+            // no contraction into an fma): the output bits do not depend on the schedule.
+            const float inv = 1.0f / __fadd_rn(__fmul_rn(l0, a0), __fmul_rn(l1, a1));
             const float f0 = a0 * inv, f1 = a1 * inv;
             const bool use0 = __any_sync(0xffffffffu, l0 > 0.f), use1 = __any_sync(0xffffffffu, l1 > 0.f);
             tc_fence_after();
@@ -811,16 +814,16 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
 #pragma unroll 1
             for (int q = 0; q < D / 64; ++q) {
                 const uint32_t col = static_cast<uint32_t>(w * (D / 2) + q * 32);
-                float r[32];
+                float r[32], r1[32];
 #pragma unroll
-                for (int i = 0; i < 32; ++i) r[i] = 0.f;
+                for (int i = 0; i < 32; ++i) r[i] = r1[i] = 0.f;
                 if (use0) {
                     uint32_t o0[32];
                     tmem_ld32(trow + O_COL + col, o0);
                     tmem_wait_ld();
                     if (l0 > 0.f) {
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) r[i] = __uint_as_float(o0[i]) * f0;
+                        for (int i = 0; i < 32; ++i) r[i] = __fmul_rn(__uint_as_float(o0[i]), f0);
                     }
                 }
                 if (use1) {
@@ -829,9 +832,11 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                     tmem_wait_ld();
                     if (l1 > 0.f) {
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) r[i] = fmaf(__uint_as_float(o1[i]), f1, r[i]);
+                        for (int i = 0; i < 32; ++i) r1[i] = __fmul_rn(__uint_as_float(o1[i]), f1);
                     }
                 }
+#pragma unroll
+                for (int i = 0; i < 32; ++i) r[i] = __fadd_rn(r[i], r1[i]);
                 if (store) {
 #pragma unroll
                     for (int v8 = 0; v8 < 4; ++v8) {

@@ -378,6 +378,15 @@ class Layer:
     def reorder_v(self, v, stream=None):
         reorder(self.g, v, self.vt, stream)
 
+    def route_qk(self, q, k, stream=None):
+        """Q and K to tiles and kv lists: the fused call, or two reorders and
+        routing (same bits)."""
+        if self.fused_route:
+            return self.reorder_route(q, k, stream)
+        reorder(self.g, q, self.qt, stream)
+        reorder(self.g, k, self.kt, stream)
+        return self.route(stream)
+
     def kernel_launches(self) -> int:
         """Kernels one __call__ (unfused inverse) launches: reorders, routing,
         the work list (plus the query-group bitmaps for bs < 128), attention,
@@ -401,12 +410,8 @@ class Layer:
                                   workspace=self.attn_ws, stream=stream)
 
     def __call__(self, q, k, v, stats: bool = False, stream=None, fused_inverse: bool = False):
-        if self.fused_route:
-            self.reorder_route(q, k, stream)
-            self.reorder_v(v, stream)
-        else:
-            self.reorder_qkv(q, k, v, stream)
-            self.route(stream)
+        self.route_qk(q, k, stream)
+        self.reorder_v(v, stream)
         if fused_inverse:
             return self.attend_raster(stats, stream)
         self.attend(stats, stream)
@@ -418,9 +423,11 @@ class HostPipeline:
 
     Heads are independent through every step, so the layer is run as
     `groups` head slices on two rotating sets of device buffers: the upload
-    of slice i+1 (one copy stream), the four library calls on slice i (the
+    of slice i+1 (one copy stream), the library calls on slice i (the
     compute stream) and the download of slice i-1 (another copy stream)
-    overlap.  The output equals one whole-layer call bit for bit."""
+    overlap.  Within a slice, Q and K are uploaded first and routed while V
+    is still on its way.  The output equals one whole-layer call bit for
+    bit."""
 
     def __init__(self, g: Geom, p: float, k: int, groups: int = 4, device="cuda", order: str = "raster",
                  fused_route: bool = True):
@@ -451,14 +458,20 @@ class HostPipeline:
             lay, (qd, kd, vd) = self.layers[b], self.inputs[b]
             if freed[b] is not None:
                 self.up.wait_event(freed[b])
-            for src, dst in ((q_host, qd), (k_host, kd), (v_host, vd)):
-                _check("fvattn_copy_heads", L.fvattn_copy_heads(ctypes.byref(g), i * self.nh, self.nh,
-                                                                ctypes.c_void_p(src.data_ptr()), _ptr(dst), 1,
-                                                                _stream(self.up)))
-            uploaded = torch.cuda.Event()
-            uploaded.record(self.up)
-            s.wait_event(uploaded)
-            out = lay(qd, kd, vd, stream=s)
+            uploaded = []
+            for pair in (((q_host, qd), (k_host, kd)), ((v_host, vd),)):
+                for src, dst in pair:
+                    _check("fvattn_copy_heads", L.fvattn_copy_heads(ctypes.byref(g), i * self.nh, self.nh,
+                                                                    ctypes.c_void_p(src.data_ptr()), _ptr(dst), 1,
+                                                                    _stream(self.up)))
+                uploaded.append(torch.cuda.Event())
+                uploaded[-1].record(self.up)
+            s.wait_event(uploaded[0])
+            lay.route_qk(qd, kd, stream=s)
+            s.wait_event(uploaded[1])
+            lay.reorder_v(vd, stream=s)
+            lay.attend(stream=s)
+            out = lay.restore(stream=s)
             computed = torch.cuda.Event()
             computed.record(s)
             self.down.wait_event(computed)

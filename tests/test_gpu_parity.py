@@ -401,6 +401,29 @@ def test_attention_with_extreme_score_range(fv, orc, tw):
     assert mx <= MAX_ABS and mean <= MEAN_ABS, (mx, mean)
 
 
+@pytest.mark.parametrize("name", ["720p", "cfg720p"])
+def test_attention_output_is_schedule_independent(fv, name):
+    """Four heads of a full-size layer: CTAs take thousands of items in a
+    timing-dependent order, and which softmax group owns which half of an
+    item's chunks follows that order.  Two runs, and the heads run as two
+    separate two-head layers, give the same output bits."""
+    w = synth.custom_workload(**{**synth.WORKLOADS[name].as_dict(), "H": 4})
+    g = fv.geom_of(w)
+    q, k, v = _gpu_inputs(w)
+    layer = fv.Layer(g, w.p, w.k)
+    first = layer(q, k, v).clone()
+    second = layer(q, k, v)
+    torch.cuda.synchronize()
+    assert fv.get_status() == 0
+    assert torch.equal(first.view(torch.int16), second.view(torch.int16))
+    gh = fv.geom(w.B, 2, w.D, w.F, w.Hs, w.Ws, w.tf, w.th, w.tw)
+    half = fv.Layer(gh, w.p, w.k)
+    for h0 in (0, 2):
+        part = half(*(t[:, :, h0:h0 + 2].contiguous() for t in (q, k, v)))
+        torch.cuda.synchronize()
+        assert torch.equal(part.view(torch.int16), first[:, :, h0:h0 + 2].contiguous().view(torch.int16))
+
+
 def test_single_block_video(fv, orc):
     """nb = 1: one partial block per head (a 1 x 3 x 5 latent in a 2 x 8 x 8 tile)."""
     w = synth.custom_workload(B=1, H=2, D=128, F=1, Hs=3, Ws=5, tf=2, th=8, tw=8, seed=3, p=0.9, k=1)
@@ -481,6 +504,19 @@ def test_full_size_sampled_parity(fv, orc, name):
     qb = _bits(q)
     assert np.array_equal(_bits(layer.qt), orc.reorder(qb, w))
     del qb
+    # logits against the oracle's pooling and scoring on sampled heads (the persistent score kernel
+    # runs several tiles per CTA at these sizes)
+    BH = w.B * w.H
+    heads = sorted({0, BH - 1, *synth.sample_items(BH, 2, seed=7)})
+    w1 = synth.custom_workload(**{**w.as_dict(), "B": 1, "H": len(heads)})
+    sel = torch.tensor(heads, device=layer.qt.device)
+    qp_o = orc.pool(_bits(layer.qt.view(BH, g.Npad, g.D)[sel].unsqueeze(0)), w1)
+    kp_o = orc.pool(_bits(layer.kt.view(BH, g.Npad, g.D)[sel].unsqueeze(0)), w1)
+    L_o = orc.logits(qp_o, kp_o, layer.scale)[0]
+    L_g = layer.routed.logits.view(BH, g.nb, g.nb)[sel].cpu().numpy().astype(np.float64)
+    nq = np.linalg.norm(qp_o[0], axis=-1)[:, :, None]
+    nk = np.linalg.norm(kp_o[0], axis=-1)[:, None, :]
+    assert np.all(np.abs(L_g - L_o) <= 2e-5 * layer.scale * nq * nk + 1e-6)
     bad, unexcused, ties = _check_mask(orc, layer.routed.logits, layer.routed.kv_idx, layer.routed.kv_cnt,
                                        w.p, w.k)
     assert unexcused == [], unexcused[:10]
