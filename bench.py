@@ -482,7 +482,7 @@ def run_fvattn(args):
         kh = k.cpu().pin_memory()
         vh = v.cpu().pin_memory()
         oh = torch.empty_like(qh).pin_memory()
-        groups = args.e2e_groups if (g.H % args.e2e_groups == 0 and g.H >= 2 * args.e2e_groups) else 1
+        groups = args.e2e_groups or fvattn.default_head_groups(g.H)
         pipe = fvattn.HostPipeline(fvattn.geom_of(w), w.p, w.k, groups=groups, device=dev, order=args.order,
                                    fused_route=fused)
         pipe(qh, kh, vh, oh)
@@ -528,8 +528,9 @@ def main():
                     help="block order of the tiles (raster tile order or the 3-D Hilbert curve)")
     ap.add_argument("--stack", action="store_true",
                     help="also time every seeded layer of a multi-layer workload once (cfg720p: 40 layers)")
-    ap.add_argument("--e2e-groups", type=int, default=20,
-                    help="head groups of the end-to-end pipeline (uploads, compute and downloads overlap)")
+    ap.add_argument("--e2e-groups", type=int, default=0,
+                    help="head groups of the end-to-end pipeline (uploads, compute and downloads overlap); "
+                         "0: fvattn.default_head_groups (two heads a group: 20 for 40 heads)")
     ap.add_argument("--unfused-route", action="store_true",
                     help="time the step with separate reorders and routing instead of the fused call")
     ap.add_argument("--heads", type=int, default=0,

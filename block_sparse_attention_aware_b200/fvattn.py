@@ -418,6 +418,18 @@ class Layer:
         return self.restore(stream)
 
 
+def default_head_groups(H: int) -> int:
+    """Head groups for HostPipeline: two heads per group when H is even,
+    otherwise the most groups with at least two heads each (one group when
+    no divisor of H allows that).  Smaller groups leave less of the first
+    upload and the last download outside the overlap."""
+    best = 1
+    for groups in range(1, H + 1):
+        if H % groups == 0 and H // groups >= 2:
+            best = groups
+    return best
+
+
 class HostPipeline:
     """End to end from page-locked host buffers, pipelined by head groups.
 
@@ -429,9 +441,11 @@ class HostPipeline:
     is still on its way.  The output equals one whole-layer call bit for
     bit."""
 
-    def __init__(self, g: Geom, p: float, k: int, groups: int = 4, device="cuda", order: str = "raster",
-                 fused_route: bool = True):
-        if g.H % groups:
+    def __init__(self, g: Geom, p: float, k: int, groups: Optional[int] = None, device="cuda",
+                 order: str = "raster", fused_route: bool = True):
+        if groups is None:
+            groups = default_head_groups(g.H)
+        if groups < 1 or g.H % groups:
             raise ValueError(f"{g.H} heads do not split into {groups} equal groups")
         self.g, self.groups, self.nh = g, groups, g.H // groups
         gs = geom(g.B, self.nh, g.D, g.F, g.Hs, g.Ws, g.tf, g.th, g.tw)
