@@ -117,6 +117,45 @@ def _need_cuda(*ts):
             raise ValueError("tensors must be contiguous CUDA tensors")
 
 
+def _expect(name: str, t: Optional[torch.Tensor], shape, dtype):
+    """The kernels read and write dense buffers of exactly this shape."""
+    if t is None:
+        return
+    if t.dtype != dtype or tuple(t.shape) != tuple(shape) or not t.is_contiguous() or not t.is_cuda:
+        raise ValueError(f"{name}: expected a contiguous CUDA {dtype} tensor of shape {tuple(shape)}, "
+                         f"got {t.dtype} {tuple(t.shape)} (contiguous={t.is_contiguous()}, cuda={t.is_cuda})")
+
+
+def _raster(g: Geom):
+    return (g.B, g.N, g.H, g.D)
+
+
+def _tiled(g: Geom):
+    return (g.B, g.H, g.Npad, g.D)
+
+
+def _expect_attn(g: Geom, qt, kt, vt, kv_idx, kv_cnt, out, out_shape, sm_stats):
+    for name, t in (("qt", qt), ("kt", kt), ("vt", vt)):
+        if t is None:
+            raise ValueError(f"{name} is required")
+        _expect(name, t, _tiled(g), torch.bfloat16)
+    _expect("kv_idx", kv_idx, (g.B, g.H, g.nb, g.nb), torch.int32)
+    _expect("kv_cnt", kv_cnt, (g.B, g.H, g.nb), torch.int32)
+    _expect("out", out, out_shape, torch.bfloat16)
+    if sm_stats is not None:
+        _need_cuda(sm_stats)
+        if sm_stats.dtype != torch.int64 or sm_stats.numel() < 2 * num_sms():
+            raise ValueError(f"sm_stats: expected int64 with at least {2 * num_sms()} elements")
+
+
+def _expect_routed(g: Geom, out: "RouteOut"):
+    _expect("kv_idx", out.kv_idx, (g.B, g.H, g.nb, g.nb), torch.int32)
+    _expect("kv_cnt", out.kv_cnt, (g.B, g.H, g.nb), torch.int32)
+    _expect("q_pool", out.q_pool, (g.B, g.H, g.nb, g.D), torch.float32)
+    _expect("k_pool", out.k_pool, (g.B, g.H, g.nb, g.D), torch.float32)
+    _expect("logits", out.logits, (g.B, g.H, g.nb, g.nb), torch.float32)
+
+
 def geom(B, H, D, F, Hs, Ws, tf, th, tw) -> Geom:
     g = Geom(B=B, H=H, D=D, F=F, Hs=Hs, Ws=Ws, tf=tf, th=th, tw=tw)
     _check("fvattn_geom_init", load().fvattn_geom_init(ctypes.byref(g)))
@@ -159,8 +198,8 @@ def tiled_empty(g: Geom, device="cuda") -> torch.Tensor:
 
 def reorder(g: Geom, x: torch.Tensor, out: Optional[torch.Tensor] = None, stream=None):
     """fvattn_reorder: raster [B, N, H, D] bf16 -> tiled [B, H, Npad, D]."""
-    _need_cuda(x, out)
-    assert x.dtype == torch.bfloat16 and tuple(x.shape) == (g.B, g.N, g.H, g.D)
+    _expect("x", x, _raster(g), torch.bfloat16)
+    _expect("out", out, _tiled(g), torch.bfloat16)
     if out is None:
         out = tiled_empty(g, x.device)
     _check("fvattn_reorder", load().fvattn_reorder(ctypes.byref(g), _ptr(x), _ptr(out), _stream(stream)))
@@ -169,8 +208,8 @@ def reorder(g: Geom, x: torch.Tensor, out: Optional[torch.Tensor] = None, stream
 
 def inverse_reorder(g: Geom, ot: torch.Tensor, out: Optional[torch.Tensor] = None, stream=None):
     """fvattn_inverse_reorder: tiled [B, H, Npad, D] -> raster [B, N, H, D]."""
-    _need_cuda(ot, out)
-    assert ot.dtype == torch.bfloat16 and tuple(ot.shape) == (g.B, g.H, g.Npad, g.D)
+    _expect("ot", ot, _tiled(g), torch.bfloat16)
+    _expect("out", out, _raster(g), torch.bfloat16)
     if out is None:
         out = torch.empty((g.B, g.N, g.H, g.D), dtype=torch.bfloat16, device=ot.device)
     _check("fvattn_inverse_reorder",
@@ -213,14 +252,17 @@ def route(g: Geom, qt: torch.Tensor, kt: torch.Tensor, p: float, k: int,
     """fvattn_route: pooled block scores -> Top-p (+ Top-k floor) kv lists.
     p = 0 (fixed Top-k mode) or k_extra > 0 (augmentation) go through
     fvattn_route_aug."""
-    _need_cuda(qt, kt)
+    _expect("qt", qt, _tiled(g), torch.bfloat16)
+    _expect("kt", kt, _tiled(g), torch.bfloat16)
     dev = qt.device
     if scale is None:
         scale = 1.0 / math.sqrt(g.D)
     if out is None:
         out = _route_out(g, dev, debug)
+    _expect_routed(g, out)
     if workspace is None:
         workspace = route_workspace(g, dev)
+    _need_cuda(workspace)
     if k_extra or p == 0:
         rc = load().fvattn_route_aug(ctypes.byref(g), _ptr(qt), _ptr(kt), float(p), int(k), int(k_extra),
                                      float(scale), _ptr(out.kv_idx), _ptr(out.kv_cnt), _ptr(out.q_pool),
@@ -242,18 +284,23 @@ def reorder_route(g: Geom, q: torch.Tensor, k: torch.Tensor, p: float, kf: int,
                   workspace: Optional[torch.Tensor] = None, stream=None, k_extra: int = 0):
     """fvattn_reorder_route: raster Q, K -> their tiles and the kv lists in
     one pass over Q and K.  Returns (qt, kt, RouteOut)."""
-    _need_cuda(q, k, qt, kt)
-    for x in (q, k):
-        assert x.dtype == torch.bfloat16 and tuple(x.shape) == (g.B, g.N, g.H, g.D)
+    _expect("q", q, _raster(g), torch.bfloat16)
+    _expect("k", k, _raster(g), torch.bfloat16)
     dev = q.device
     if scale is None:
         scale = 1.0 / math.sqrt(g.D)
     if out is None:
         out = _route_out(g, dev, debug)
+    _expect_routed(g, out)
     qt = tiled_empty(g, dev) if qt is None else qt
     kt = tiled_empty(g, dev) if kt is None else kt
+    _expect("qt", qt, _tiled(g), torch.bfloat16)
+    _expect("kt", kt, _tiled(g), torch.bfloat16)
+    if qt.data_ptr() == kt.data_ptr():
+        raise ValueError("qt and kt must be distinct buffers")
     if workspace is None:
         workspace = route_workspace(g, dev)
+    _need_cuda(workspace)
     rc = load().fvattn_reorder_route(ctypes.byref(g), _ptr(q), _ptr(k), _ptr(qt), _ptr(kt), float(p), int(kf),
                                      int(k_extra), float(scale), _ptr(out.kv_idx), _ptr(out.kv_cnt),
                                      _ptr(out.q_pool), _ptr(out.k_pool), _ptr(out.logits), _ptr(workspace),
@@ -266,15 +313,14 @@ def sparse_attn(g: Geom, qt, kt, vt, kv_idx, kv_cnt, scale: Optional[float] = No
                 out: Optional[torch.Tensor] = None, sm_stats: Optional[torch.Tensor] = None,
                 workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
     """fvattn_sparse_attn: block-sparse attention on the kept blocks -> tiled O."""
-    _need_cuda(qt, kt, vt, kv_idx, kv_cnt, out, sm_stats)
+    _expect_attn(g, qt, kt, vt, kv_idx, kv_cnt, out, _tiled(g), sm_stats)
     if scale is None:
         scale = 1.0 / math.sqrt(g.D)
     if out is None:
         out = tiled_empty(g, qt.device)
     if workspace is None:
         workspace = attn_workspace(g, qt.device)
-    if sm_stats is not None:
-        assert sm_stats.dtype == torch.int64 and sm_stats.numel() >= 2 * num_sms()
+    _need_cuda(workspace)
     rc = load().fvattn_sparse_attn(ctypes.byref(g), _ptr(qt), _ptr(kt), _ptr(vt), _ptr(kv_idx),
                                    _ptr(kv_cnt), float(scale), _ptr(out), _ptr(sm_stats),
                                    _ptr(workspace), workspace.numel(), _stream(stream))
@@ -292,15 +338,14 @@ def sparse_attn_raster(g: Geom, qt, kt, vt, kv_idx, kv_cnt, scale: Optional[floa
                        workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
     """fvattn_sparse_attn_raster: sparse attention writing O in the raster
     [B, N, H, D] layout (the inverse reorder fused into the epilogue)."""
-    _need_cuda(qt, kt, vt, kv_idx, kv_cnt, out, sm_stats)
+    _expect_attn(g, qt, kt, vt, kv_idx, kv_cnt, out, _raster(g), sm_stats)
     if scale is None:
         scale = 1.0 / math.sqrt(g.D)
     if out is None:
-        out = torch.empty((g.B, g.N, g.H, g.D), dtype=torch.bfloat16, device=qt.device)
+        out = torch.empty(_raster(g), dtype=torch.bfloat16, device=qt.device)
     if workspace is None:
         workspace = attn_workspace(g, qt.device)
-    if sm_stats is not None:
-        assert sm_stats.dtype == torch.int64 and sm_stats.numel() >= 2 * num_sms()
+    _need_cuda(workspace)
     rc = load().fvattn_sparse_attn_raster(ctypes.byref(g), _ptr(qt), _ptr(kt), _ptr(vt), _ptr(kv_idx),
                                           _ptr(kv_cnt), float(scale), _ptr(out), _ptr(sm_stats),
                                           _ptr(workspace), workspace.numel(), _stream(stream))
@@ -314,7 +359,7 @@ def sparse_attn_noalloc(g: Geom, qt, kt, vt, kv_idx, kv_cnt, scale: Optional[flo
     scratch array instead of a caller workspace (for callers that cannot
     allocate device memory).  Calls that overlap on the GPU share that
     scratch and must be serialised by the caller."""
-    _need_cuda(qt, kt, vt, kv_idx, kv_cnt, out, sm_stats)
+    _expect_attn(g, qt, kt, vt, kv_idx, kv_cnt, out, _tiled(g), sm_stats)
     if scale is None:
         scale = 1.0 / math.sqrt(g.D)
     if out is None:
