@@ -216,7 +216,9 @@ int fvattn_num_sms(void);
  * are taken longest-first by a persistent kernel with one CTA per SM.  For
  * bs < 128 an item is a 128-row tile of 128 / bs consecutive query blocks
  * that walks the union of their kv lists, each row masked to its own
- * block's list (the order of a list does not matter).
+ * block's list (the order of a list does not matter).  The output bits
+ * depend only on the inputs: not on which CTA takes an item, nor on how the
+ * heads of a layer are split across calls.
  *   q_t, k_t, v_t  [B, H, Npad, D] bf16 from fvattn_reorder (padding zero)
  *   kv_idx, kv_cnt as written by fvattn_route (each row: cnt in [1, nb],
  *                  distinct indices in [0, nb)); out-of-range entries set
