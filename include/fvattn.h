@@ -15,6 +15,11 @@
  *   fvattn_sparse_attn      block-sparse flash attention on the kept blocks
  *   fvattn_inverse_reorder  tiles -> raster tokens
  *
+ * and fused forms of the first two and last two steps
+ * (fvattn_reorder_route: reorder of Q and K and routing in one pass over
+ * them; fvattn_sparse_attn_raster: attention writing raster rows), with the
+ * same results bit for bit.
+ *
  * Conventions for every call:
  *   - All tensor pointers are DEVICE pointers, 16-byte aligned, contiguous.
  *     bf16 tensors are passed as void* holding IEEE bfloat16 values.
