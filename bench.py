@@ -223,6 +223,38 @@ def aggregate_over_ranks(t_local: float, work_local: float, world: int, device):
 
 # ---------------------------------------------------------------- GPU arm
 
+NOMINAL_DENSE_BF16_TFLOPS = 2250.0   # NVIDIA's B200 dense bf16 figure (context only)
+
+
+def block_real_counts(g, tile_of_block=None):
+    """Real (non-padding) tokens of each block: the tile's clipped extent.
+    tile_of_block: the block -> raster tile table (Hilbert order), or None."""
+    counts = []
+    for blk in range(g.nb):
+        t = blk if tile_of_block is None else int(tile_of_block[blk])
+        bx, by, bf = t % g.nbx, (t // g.nbx) % g.nby, t // (g.nbx * g.nby)
+        counts.append(min(g.tf, g.F - bf * g.tf) * min(g.th, g.Hs - by * g.th) * min(g.tw, g.Ws - bx * g.tw))
+    return counts
+
+
+def valid_token_flops(g, kv_idx, kv_cnt, counts, rows_per_chunk=64):
+    """Attention FLOPs over real tokens only: 4 * D * sum over (b, h, i) of
+    n_i * sum of n_j over the kept blocks j (entries past kv_cnt ignored)."""
+    import torch
+    nb = g.nb
+    n = torch.as_tensor(counts, dtype=torch.float64, device=kv_idx.device)
+    idx = kv_idx.reshape(-1, nb, nb)
+    cnt = kv_cnt.reshape(-1, nb)
+    pos = torch.arange(nb, device=kv_idx.device)
+    total = 0.0
+    for r0 in range(0, idx.shape[0], rows_per_chunk):
+        i = idx[r0:r0 + rows_per_chunk].long().clamp(0, nb - 1)
+        used = pos[None, None, :] < cnt[r0:r0 + rows_per_chunk, :, None]
+        kept = torch.where(used, n[i], torch.zeros((), dtype=torch.float64, device=n.device)).sum(dim=-1)
+        total += float((kept * n[None, :]).sum())
+    return 4.0 * g.D * total
+
+
 def _imbalance(layer, nsm):
     import numpy as np
     st = layer.sm_stats.cpu().numpy().astype(np.float64)
@@ -404,6 +436,8 @@ def run_fvattn(args):
     imb_pred = float(blocks[used].max() / blocks[used].mean()) if used.any() else None
     per_head = cnt.view(g.B * g.H, g.nb).sum(dim=1).double().cpu().numpy()
     sustained = peaks["bf16_tflops_sustained"]
+    table = layer.order_table[: g.nb].cpu().tolist() if layer.order_table is not None else None
+    vflops = valid_token_flops(g, layer.routed.kv_idx, cnt, block_real_counts(g, table))
 
     line = {
         "metric": METRIC,
@@ -426,6 +460,9 @@ def run_fvattn(args):
             "tflops_executed_blocks": attn_tflops,
             "pct_of_bf16_peak_burst": 100.0 * attn_tflops / peaks["bf16_tflops"],
             "pct_of_bf16_peak_sustained": 100.0 * attn_tflops / sustained,
+            "pct_of_nominal_dense_bf16": 100.0 * attn_tflops / NOMINAL_DENSE_BF16_TFLOPS,
+            "tflops_valid_tokens": vflops / attn_s / 1e12,
+            "valid_token_flop_fraction": vflops / flops,
             "ms": ms["attention"], "density": pairs / float(g.B * g.H * g.nb * g.nb),
             "executed_block_pairs": pairs,
             "sm_imbalance_max_over_mean": imb, "sm_imbalance_predicted_from_blocks": imb_pred,

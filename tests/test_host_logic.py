@@ -46,3 +46,37 @@ def test_binding_rejects_bad_buffers_before_any_launch(fv):
     for call in (fv.sparse_attn, fv.sparse_attn_raster, fv.sparse_attn_noalloc):
         with pytest.raises(ValueError):
             call(g, t, t, t, idx, cnt)
+
+
+def test_valid_token_flops_against_brute_force():
+    """bench's real-token FLOP count: padding rows and columns of partial
+    blocks excluded, entries past kv_cnt ignored (here filled with junk)."""
+    import torch
+    import bench
+    g = fvattn.Geom(B=2, H=3, D=64, F=3, Hs=5, Ws=7, tf=2, th=2, tw=4)
+    g.nbf, g.nby, g.nbx = 2, 3, 2
+    g.nb, g.bs = 12, 16
+    counts = bench.block_real_counts(g)
+    # brute force over the token grid
+    want = [0] * g.nb
+    for f in range(g.F):
+        for y in range(g.Hs):
+            for x in range(g.Ws):
+                want[((f // g.tf) * g.nby + y // g.th) * g.nbx + x // g.tw] += 1
+    assert counts == want and sum(counts) == g.F * g.Hs * g.Ws
+    gen = torch.Generator().manual_seed(3)
+    kv_cnt = torch.randint(1, g.nb + 1, (g.B, g.H, g.nb), generator=gen, dtype=torch.int32)
+    kv_idx = torch.randint(-50, 50, (g.B, g.H, g.nb, g.nb), generator=gen, dtype=torch.int32)
+    ref = 0
+    for b in range(g.B):
+        for h in range(g.H):
+            for i in range(g.nb):
+                c = int(kv_cnt[b, h, i])
+                kept = torch.randperm(g.nb, generator=gen)[:c]
+                kv_idx[b, h, i, :c] = kept.to(torch.int32)
+                ref += counts[i] * sum(counts[j] for j in kept.tolist())
+    got = bench.valid_token_flops(g, kv_idx, kv_cnt, counts, rows_per_chunk=4)
+    assert got == 4.0 * g.D * ref
+    # Hilbert-style table: counts follow each block's tile
+    table = list(reversed(range(g.nb)))
+    assert bench.block_real_counts(g, table) == list(reversed(counts))
