@@ -537,7 +537,8 @@ def run_fvattn(args):
         line["e2e"] = {"value": flops_all / te / 1e12, "unit": "TFLOP/s", "ms_per_step": te * 1e3,
                        "h2d_bytes_per_step": 3 * raster_bytes, "d2h_bytes_per_step": raster_bytes,
                        "steps": args.e2e_steps, "head_groups": groups,
-                       "how": "fvattn.HostPipeline: per head group, 2-D H2D copies of Q/K/V, the four calls, "
+                       "how": "fvattn.HostPipeline: per head group, 2-D H2D copies of Q/K/V, the layer's calls "
+                              "(Q/K reorder + routing in one pass, V reorder, attention, inverse reorder), "
                               "2-D D2H copy of O; groups overlap on two copy streams and the compute stream"}
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

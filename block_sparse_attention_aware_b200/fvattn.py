@@ -546,7 +546,8 @@ class HostPipeline:
 
 def attention_from_host(layer: Layer, q_host, k_host, v_host, o_host, stream=None):
     """End to end from pinned host buffers: H2D copies of raster Q, K, V, the
-    four library calls, and a D2H copy of the raster output, all on one stream."""
+    layer's library calls, and a D2H copy of the raster output, all on one
+    stream (HostPipeline overlaps them instead)."""
     s = stream if stream is not None else torch.cuda.current_stream()
     with torch.cuda.stream(s):
         qd = torch.empty_like(q_host, device="cuda")

@@ -268,7 +268,7 @@ HILBERT = [
 
 @pytest.mark.parametrize("name,w", HILBERT, ids=[s[0] for s in HILBERT])
 def test_hilbert_layer_parity(fv, orc, name, w):
-    """Hilbert block order through all four calls: reorder and inverse
+    """Hilbert block order through every call of a layer: reorder and inverse
     bit-exact, masks (block indices in curve order) equal to the oracle's on
     the GPU logits outside near ties, attention within the bar."""
     g = fv.geom_of(w)
