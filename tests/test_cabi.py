@@ -99,6 +99,32 @@ def test_null_and_misaligned_pointers_rejected(fv):
                                   ctypes.c_void_p(256), 0, None) == fv.ERR_INVALID
 
 
+def test_copy_heads_rejects_bad_slices(fv):
+    """fvattn_copy_heads checks the head slice before any copy is queued."""
+    lib = fv.load()
+    g = fv.geom(1, 4, 64, 2, 8, 8, 2, 2, 4)
+    gp, V = ctypes.byref(g), ctypes.c_void_p
+    for h0, nh in ((-1, 2), (0, 0), (3, 2), (0, 5)):
+        assert lib.fvattn_copy_heads(gp, h0, nh, V(16), V(32), 1, None) == fv.ERR_INVALID
+    assert lib.fvattn_copy_heads(gp, 0, 2, None, V(32), 1, None) == fv.ERR_INVALID
+    assert lib.fvattn_copy_heads(gp, 0, 2, V(16), None, 0, None) == fv.ERR_INVALID
+    assert lib.fvattn_copy_heads(None, 0, 2, V(16), V(32), 0, None) == fv.ERR_INVALID
+
+
+def test_block_order_rejects_bad_arguments(fv):
+    """fvattn_block_order: null or misaligned table, or a geometry whose tile
+    counts do not multiply to nb, is refused before the launch."""
+    lib = fv.load()
+    g = fv.geom(1, 1, 64, 4, 8, 8, 1, 4, 4)
+    V = ctypes.c_void_p
+    assert lib.fvattn_block_order(ctypes.byref(g), None, None) == fv.ERR_INVALID
+    assert lib.fvattn_block_order(ctypes.byref(g), V(20), None) == fv.ERR_INVALID
+    assert lib.fvattn_block_order(None, V(32), None) == fv.ERR_INVALID
+    bad = fv.Geom.from_buffer_copy(g)
+    bad.nb = g.nb + 1
+    assert lib.fvattn_block_order(ctypes.byref(bad), V(32), None) == fv.ERR_INVALID
+
+
 def test_workspace_sizes(fv):
     lib = fv.load()
     g = fv.geom(1, 40, 128, 21, 45, 80, 2, 8, 8)
