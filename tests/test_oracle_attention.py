@@ -149,3 +149,36 @@ def test_single_kept_block_is_local_softmax(orc):
     e = np.exp(s - s.max(axis=1, keepdims=True))
     want = (e / e.sum(axis=1, keepdims=True)) @ vd[0, keys, 0]
     np.testing.assert_allclose(got[0, :, 0], want, rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("g", GEOMS)
+def test_equal_scores_average_the_kept_values(orc, g):
+    """Closed form: with every key zero all scores are equal, so each output
+    row is the plain mean of V over the real tokens of its row's kept blocks
+    (padding excluded, each kept block counted once).  No exponential is
+    involved, so this pins the masking, the kept-set gather and the
+    normalisation independently of any softmax implementation."""
+    w, q, k, v = _setup(g, seed=11)
+    k = torch.zeros_like(k)
+    geo = orc.geometry(w)
+    nb = geo["nb"]
+    rng = np.random.default_rng(5)
+    kv_idx = np.zeros((w.B, w.H, nb, nb), dtype=np.int32)
+    kv_cnt = np.zeros((w.B, w.H, nb), dtype=np.int32)
+    for b in range(w.B):
+        for h in range(w.H):
+            for i in range(nb):
+                c = int(rng.integers(1, nb + 1))
+                kv_idx[b, h, i, :c] = np.sort(rng.choice(nb, size=c, replace=False))
+                kv_cnt[b, h, i] = c
+    got = _oracle_raster_output(orc, w, q, k, v, kv_idx, kv_cnt)
+    tile = _tile_of_tokens(w, geo)
+    vd = v.double().numpy()
+    for b in range(w.B):
+        for h in range(w.H):
+            for n in range(w.N):
+                i = tile[n]
+                kept = kv_idx[b, h, i, :kv_cnt[b, h, i]]
+                keys = np.nonzero(np.isin(tile, kept))[0]
+                want = vd[b, keys, h].mean(axis=0)
+                np.testing.assert_allclose(got[b, n, h], want, rtol=0, atol=1e-12)
