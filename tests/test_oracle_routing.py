@@ -96,6 +96,26 @@ def test_logits_vs_numpy_matmul(orc):
     np.testing.assert_allclose(L, want, rtol=1e-13, atol=1e-13)
 
 
+def test_logits_closed_forms(orc):
+    """Scores of structured pooled vectors, known without any product:
+    unit vectors give scale on the diagonal and 0 elsewhere; constant rows
+    give scale * D * a * b; a transposed operand or a dropped scale fails."""
+    nb, D, scale = 6, 8, 0.5
+    eye = np.zeros((1, 1, nb, D))
+    for i in range(nb):
+        eye[0, 0, i, i % D] = 1.0
+    L = orc.logits(eye, eye, scale)[0, 0]
+    np.testing.assert_array_equal(L, scale * np.eye(nb))
+    a = np.arange(1, nb + 1, dtype=np.float64)          # row i of Qp is all a_i
+    b = np.arange(nb, 0, -1, dtype=np.float64) * 0.25   # row j of Kp is all b_j
+    qp = np.repeat(a[:, None], D, axis=1)[None, None]
+    kp = np.repeat(b[:, None], D, axis=1)[None, None]
+    L = orc.logits(qp, kp, scale)[0, 0]
+    for i in range(nb):
+        for j in range(nb):
+            assert L[i, j] == scale * D * a[i] * b[j]
+
+
 # ---------------------------------------------------------------- select
 
 def _probs_in_order(L):
