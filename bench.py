@@ -164,6 +164,68 @@ def oracle_sample_time(w, qt, kt, vt, q_raster, kv_idx_full, kv_cnt_full, heads=
     return full, desc, threads, t_reorder + t_route + t_attn
 
 
+def oracle_mask_parity(w, g, layer, q, k, e2e_heads=4):
+    """Mask parity of the benchmarked step, checked by the oracle after the
+    timed region (same leg as the CPU baseline, rank 0 only).
+
+    One more pass of the step's routing call, with its debug logits output,
+    gives the kv lists and the fp32 logits they were selected from.  The
+    oracle's selection on those logits must give the same kept set in every
+    row except rows it flags as near ties (cumulative mass within 1e-5 of p);
+    all three counts are returned.  End-to-end mode: on `e2e_heads` heads the
+    oracle also pools and scores the tiles itself and selects on its own
+    logits; the rows whose kept set then differs are counted (not graded:
+    logit rounding can move rows that sit near the p boundary)."""
+    import numpy as np
+    import torch
+    from oracle import oracle as orc
+    from block_sparse_attention_aware_b200 import fvattn, synth
+    dev = q.device
+    routed = fvattn.RouteOut(kv_idx=torch.empty_like(layer.routed.kv_idx),
+                             kv_cnt=torch.empty_like(layer.routed.kv_cnt),
+                             logits=torch.empty((g.B, g.H, g.nb, g.nb), dtype=torch.float32, device=dev))
+    if layer.fused_route:
+        fvattn.reorder_route(layer.g, q, k, layer.p, layer.k, layer.scale, out=routed, qt=layer.qt, kt=layer.kt,
+                             workspace=layer.route_ws)
+    else:
+        fvattn.route(layer.g, layer.qt, layer.kt, layer.p, layer.k, layer.scale, out=routed,
+                     workspace=layer.route_ws)
+    torch.cuda.synchronize()
+    same_as_step = bool(torch.equal(routed.kv_cnt, layer.routed.kv_cnt))
+    nb = g.nb
+    cnt_g = routed.kv_cnt.cpu().numpy().reshape(-1)
+    idx_g = routed.kv_idx.cpu().numpy().reshape(-1, nb)
+    t0 = time.perf_counter()
+    idx_o, cnt_o, _, tie = orc.select(routed.logits.cpu().numpy().reshape(-1, nb), w.p, w.k)
+
+    def differing(ig, cg, io, co):
+        bad = set(np.nonzero(cg != co)[0].tolist())
+        for r in np.nonzero(cg == co)[0]:
+            if not np.array_equal(ig[r, :cg[r]], io[r, :co[r]]):
+                bad.add(int(r))
+        return sorted(bad)
+
+    bad = differing(idx_g, cnt_g, idx_o, cnt_o)
+    unexcused = [r for r in bad if not tie[r]]
+    BH = g.B * g.H
+    heads = sorted({0, BH // 2, BH - 1} | set(synth.sample_items(BH, max(e2e_heads - 3, 0), seed=11)))
+    sub = synth.custom_workload(**{**w.as_dict(), "B": 1, "H": len(heads), "name": "sample"})
+    sel = torch.tensor(heads, device=dev)
+    qb = synth.bf16_bits(layer.qt.view(BH, g.Npad, g.D)[sel].unsqueeze(0))
+    kb = synth.bf16_bits(layer.kt.view(BH, g.Npad, g.D)[sel].unsqueeze(0))
+    _, _, _, idx_e, cnt_e, _, _ = orc.route(qb, kb, sub, w.p, w.k, layer.scale)
+    hs = np.array(heads)
+    e2e_bad = differing(idx_g.reshape(BH, nb, nb)[hs].reshape(-1, nb), cnt_g.reshape(BH, nb)[hs].reshape(-1),
+                        idx_e.reshape(-1, nb), cnt_e.reshape(-1))
+    return {"rows": int(len(cnt_g)), "near_tie_rows": int(tie.sum()), "mismatched_rows": len(bad),
+            "unexcused": len(unexcused), "near_tie_band": orc.TIE_BAND,
+            "kv_lists_equal_timed_step": same_as_step,
+            "how": "oracle selection on the GPU's own fp32 logits, every row of the layer",
+            "e2e": {"heads": heads, "rows": int(len(hs) * nb), "mismatched_rows": len(e2e_bad),
+                    "how": "oracle pools, scores and selects the tiles of these heads by itself"},
+            "oracle_seconds": time.perf_counter() - t0}
+
+
 def run_reference(args):
     """The oracle timed as the reference arm (rank 0; other ranks exit)."""
     rank = int(os.environ.get("RANK", "0"))
@@ -541,7 +603,9 @@ def run_fvattn(args):
                               "(Q/K reorder + routing in one pass, V reorder, attention, inverse reorder), "
                               "2-D D2H copy of O; groups overlap on two copy streams and the compute stream"}
 
+    # oracle leg (rank 0, one GPU, after every timed region): the CPU baseline and the mask parity
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["mask_parity"] = oracle_mask_parity(w, g, layer, q, k)
         full, desc, threads, spent = oracle_sample_time(
             w, layer.qt.cpu(), layer.kt.cpu(), layer.vt.cpu(), q.cpu(), None, cnt.cpu().numpy())
         line["cpu_baseline"] = {"value": flops / full / 1e12, "unit": "TFLOP/s", "cores": threads,
@@ -559,8 +623,9 @@ def main():
     ap.add_argument("--steps", type=int, default=5)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="fvattn", choices=["fvattn", "reference"])
-    ap.add_argument("--e2e-steps", type=int, default=3)
-    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--no-cpu-baseline", action="store_true",
+                    help="skip the oracle leg (CPU baseline timing and mask parity)")
     ap.add_argument("--workload", default=WORKLOAD, help="named workload of synth.WORKLOADS")
     ap.add_argument("--order", default="raster", choices=["raster", "hilbert"],
                     help="block order of the tiles (raster tile order or the 3-D Hilbert curve)")

@@ -3,8 +3,10 @@
     python -m block_sparse_attention_aware_b200.build [--force]
 
 Each .cu under csrc/ is compiled to an object with
-`-gencode arch=compute_100a,code=sm_100a -lineinfo -O3`, then linked into
-block_sparse_attention_aware_b200/libfvattn.so.  Needs only nvcc (no GPU).
+`-gencode arch=compute_100a,code=sm_100a -lineinfo -O3` as a whole program
+(no relocatable device code: ptxas honours per-warpgroup register budgets
+only then), then linked into block_sparse_attention_aware_b200/libfvattn.so.
+Needs only nvcc (no GPU).
 """
 from __future__ import annotations
 
@@ -21,7 +23,7 @@ LIB = os.path.join(HERE, "libfvattn.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
 SOURCES = ["api.cu", "reorder.cu", "route.cu", "attn.cu", "noalloc.cu"]
-FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3", "-std=c++17", "-rdc=true",
+FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3", "-std=c++17",
          "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr", "-I", INCLUDE, "-I", CSRC]
 
 
@@ -44,7 +46,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
         subprocess.check_call(cmd)
         objs.append(obj)
     tmp = LIB + f".tmp{os.getpid()}"
-    subprocess.check_call([NVCC, "-shared", "-rdc=true", "-gencode", "arch=compute_100a,code=sm_100a",
+    subprocess.check_call([NVCC, "-shared", "-gencode", "arch=compute_100a,code=sm_100a",
                            "-o", tmp, *objs, "-lcudart"])
     os.replace(tmp, LIB)
     return LIB

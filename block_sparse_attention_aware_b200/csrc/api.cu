@@ -1,10 +1,6 @@
 // Geometry set-up and the device status word of the FVAttn C ABI.
 #include "common.cuh"
 
-namespace fv {
-__device__ int g_fvattn_status = 0;
-}
-
 using namespace fv;
 
 static int ceil_div_i(int a, int b) { return (a + b - 1) / b; }
@@ -106,11 +102,10 @@ extern "C" int fvattn_block_order(const fvattn_geom* g, int32_t* table, fvattn_s
 extern "C" int fvattn_get_status(fvattn_stream_t stream) {
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (cudaStreamSynchronize(s) != cudaSuccess) return FVATTN_ERR_CUDA;
-    int v = 0;
-    if (cudaMemcpyFromSymbol(&v, g_fvattn_status, sizeof(int)) != cudaSuccess) return FVATTN_ERR_CUDA;
-    const int zero = 0;
-    if (cudaMemcpyToSymbol(g_fvattn_status, &zero, sizeof(int)) != cudaSuccess) return FVATTN_ERR_CUDA;
-    return v;
+    // both words are read and cleared; the attention kernels' error is reported first
+    const int va = take_status_attn();
+    const int vr = take_status_route();
+    return va != FVATTN_OK ? va : vr;
 }
 
 extern "C" const char* fvattn_status_string(int code) {

@@ -40,6 +40,8 @@
 // always reaches the TMEM release.
 #include <cuda.h>
 
+#include <atomic>
+
 #include "common.cuh"
 #include "ptx.cuh"
 #include "sync.cuh"
@@ -63,6 +65,15 @@ constexpr uint32_t O_COL = 256;          // S_w at columns 128*w, O_w at 256 + 1
 // precision.
 constexpr float RESCALE_SUM_LIMIT = 1073741824.0f;   // 2^30
 constexpr int MAX_GROUP = 8;             // query blocks per tile at bs = 16
+// Register split: the launch gives every thread LAUNCH_REGS; the producer and
+// issuer warpgroup drops to REGS_LOW and the two softmax warpgroups (which
+// hold a whole 128-column S row) rise to REGS_HIGH.  One warpgroup at
+// REGS_LOW plus two at REGS_HIGH must fit in what the CTA was launched with;
+// the host checks the compiled register count before every launch.
+constexpr int LAUNCH_REGS = 168;          // 65536 / 384 rounded down to a multiple of 8
+constexpr int REGS_LOW = 88;
+constexpr int REGS_HIGH = 208;
+static_assert(128 * REGS_LOW + 256 * REGS_HIGH <= ATT_THREADS * LAUNCH_REGS, "register split");
 
 struct AttnArgs {
     Geo g;
@@ -85,6 +96,8 @@ struct AttnArgs {
     unsigned long long* sm_stats;
     float scale_log2;            // scale * log2(e), > 0
     int total_items;
+    unsigned long long wait_limit_ns;   // bound of every wait (fault-injection tests shorten it)
+    int hooks;                   // FVATTN_HOOK_* fault injection (0 in normal use)
 };
 
 struct __align__(16) Ctrl {
@@ -97,6 +110,7 @@ struct __align__(16) Ctrl {
     unsigned long long mrg_full, mrg_empty;    // end-of-item exchange of (m, l)
     unsigned long long item_full[2], item_empty[2];
     unsigned long long blocks_done;
+    unsigned long long drain[2];               // issuers' final commit: their MMAs have completed
     int item[2][4];              // bh, first query block, cnt (kv blocks to walk), valid
     uint32_t mask[MAX_K_STAGES][MAX_GROUP][4];  // per query block of the tile: its valid keys of a K stage's chunk
     uint32_t tmem_base;
@@ -238,6 +252,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     const int bs = g.bs;
     const int bpc = 128 / bs;   // key blocks per 128-key chunk
     volatile int* abort_flag = &ctl.abort_flag;
+    const unsigned long long wlim = a.wait_limit_ns;
     const unsigned long long t_start = global_timer_ns();
 
     // ---- set-up: zero the operand tiles (stale rows must be finite), barriers, TMEM
@@ -267,6 +282,8 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
             mbar_init(smem_u32(&ctl.item_empty[w]), 3 + SOFTMAX_WARPS);  // two issuers, V producer, softmax
         }
         mbar_init(smem_u32(&ctl.o_free), SOFTMAX_WARPS);
+        mbar_init(smem_u32(&ctl.drain[0]), 1);
+        mbar_init(smem_u32(&ctl.drain[1]), 1);
         mbar_init(smem_u32(&ctl.mrg_full), SOFTMAX_WARPS);
         mbar_init(smem_u32(&ctl.mrg_empty), SOFTMAX_WARPS);
         ctl.abort_flag = 0;
@@ -287,295 +304,16 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     tc_fence_after();
     const uint32_t tmem = ctl.tmem_base;
 
-    if (warp == 0) {
-        // =========================== K producer: items, Q tile, K blocks, masks
-        // Column col = q*32 + lane of a chunk is token `off` of slot `slot`;
-        // its frame / row / col offsets inside the tile never change.
-        int c_slot[4], c_of[4], c_oy[4], c_ox[4];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const int col = q * 32 + lane;
-            c_slot[q] = col / bs;
-            const int off = col - c_slot[q] * bs;
-            c_ox[q] = off % g.tw;
-            c_oy[q] = (off / g.tw) % g.th;
-            c_of[q] = off / (g.tw * g.th);
-        }
-        int item_seq = 0;
-        uint32_t c_seq = 0;
-        bool ok = true;
-        while (ok) {
-            const int slot = item_seq & 1;
-            if (!wait_warp(smem_u32(&ctl.item_empty[slot]), ((item_seq >> 1) & 1) ^ 1, abort_flag)) break;
-            int t = 0;
-            if (lane == 0) t = atomicAdd(a.counter, 1);
-            t = __shfl_sync(0xffffffffu, t, 0);
-            if (t >= a.total_items) {
-                if (lane == 0) {
-                    ctl.item[slot][3] = 0;
-                    mbar_arrive(smem_u32(&ctl.item_full[slot]));
-                }
-                break;
-            }
-            const int G = GRP ? a.G : 1;
-            const int units = GRP ? a.ngroups : g.nb;
-            const int hs = t / units;
-            const int r = t - hs * units;
-            const int bh = __ldg(a.head_order + hs);
-            const int u = __ldg(a.item_order + static_cast<long long>(bh) * units + r);
-            const int qb = u * G;                     // first query block of the tile
-            const int nq = min(G, g.nb - qb);         // query blocks in the tile
-            int cnt = GRP ? __ldg(a.gcnt + static_cast<long long>(bh) * a.ngroups + u)
-                          : __ldg(a.kv_cnt + static_cast<long long>(bh) * g.nb + qb);
-            if (cnt < 1 || cnt > g.nb) {
-                if (lane == 0) record_status(FVATTN_ERR_BOUNDS);
-                cnt = cnt < 1 ? 1 : g.nb;
-            }
-            if (lane == 0) {
-                ctl.item[slot][0] = bh;
-                ctl.item[slot][1] = qb;
-                ctl.item[slot][2] = cnt;
-                ctl.item[slot][3] = 1;
-                mbar_arrive(smem_u32(&ctl.item_full[slot]));
-            }
-            if (!wait_warp(smem_u32(&ctl.q_empty), (item_seq & 1) ^ 1, abort_flag)) break;
-            const int row_base = bh * static_cast<int>(g.Npad);
-            if (lane == 0) {
-                mbar_arrive_expect_tx(smem_u32(&ctl.q_full), static_cast<uint32_t>(nq * bs * D * 2));
-                for (int tq = 0; tq < (GRP ? nq : 1); ++tq)
-#pragma unroll
-                    for (int h = 0; h < D / 64; ++h)
-                        tma_load_2d(sQ + h * 16384u + static_cast<uint32_t>(tq * bs) * 128u, &tmQ, h * 64,
-                                    row_base + (qb + tq) * bs, smem_u32(&ctl.q_full));
-            }
-            const int32_t* list = a.kv_idx + (static_cast<long long>(bh) * g.nb + qb) * g.nb;
-            UnionWalk uw;
-            if (GRP) uw.init(a.gbits + (static_cast<long long>(bh) * a.ngroups + u) * G * a.nwords, G, a.nwords, lane);
-            const int nc = (cnt + bpc - 1) / bpc;
-            // chunk cl's blocks (lane s < nblk: slot s) and membership bits, one chunk ahead
-            int j_next = 0, n_next = 0;
-            uint32_t m_next = 0u;
-            if (GRP) {
-                n_next = union_chunk<true>(uw, bpc, lane, j_next, m_next);
-            } else {
-                n_next = min(bpc, cnt);
-                j_next = chunk_block(list, 0, bpc, n_next, lane, g.nb);
-                m_next = 1u;
-            }
-            for (int cl = 0; cl < nc; ++cl, ++c_seq) {
-                const int stage = c_seq % KS;
-                const int nblk = n_next;
-                const int j = j_next;
-                const uint32_t mem = m_next;
-                if (cl + 1 < nc) {
-                    if (GRP) {
-                        n_next = union_chunk<true>(uw, bpc, lane, j_next, m_next);
-                    } else {
-                        n_next = min(bpc, cnt - (cl + 1) * bpc);
-                        j_next = chunk_block(list, cl + 1, bpc, n_next, lane, g.nb);
-                    }
-                }
-                const int ext = lane < nblk ? __ldg(a.ext + j) : 0;
-                if (!wait_warp(smem_u32(&ctl.k_empty[stage]), ((c_seq / KS) & 1) ^ 1, abort_flag)) {
-                    ok = false;
-                    break;
-                }
-                if (GRP) {
-                    // per query block t of the tile: key column real and its block in t's list.
-                    // Real-token bits once per 32-column word; a word lies in one slot when
-                    // bs >= 32, so its membership bits are warp-uniform there.
-                    uint32_t pad[4], mq[4];
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const int e = __shfl_sync(0xffffffffu, ext, c_slot[q]);
-                        mq[q] = __shfl_sync(0xffffffffu, mem, c_slot[q]);
-                        pad[q] = __ballot_sync(0xffffffffu, (c_of[q] < (e & 255)) && (c_oy[q] < ((e >> 8) & 255)) &&
-                                                                (c_ox[q] < (e >> 16)));
-                    }
-                    for (int tq = 0; tq < G; ++tq) {
-                        uint32_t words[4];
-#pragma unroll
-                        for (int q = 0; q < 4; ++q)
-                            words[q] = bs >= 32 ? (((mq[q] >> tq) & 1u) ? pad[q] : 0u)
-                                                : (pad[q] & __ballot_sync(0xffffffffu, (mq[q] >> tq) & 1u));
-                        if (lane == 0) {
-#pragma unroll
-                            for (int q = 0; q < 4; ++q) ctl.mask[stage][tq][q] = words[q];
-                        }
-                    }
-                } else {
-                    (void)mem;
-                    uint32_t words[4];
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const int e = __shfl_sync(0xffffffffu, ext, c_slot[q]);
-                        const bool valid = (c_of[q] < (e & 255)) && (c_oy[q] < ((e >> 8) & 255)) && (c_ox[q] < (e >> 16));
-                        words[q] = __ballot_sync(0xffffffffu, valid);
-                    }
-                    if (lane == 0) {
-#pragma unroll
-                        for (int q = 0; q < 4; ++q) ctl.mask[stage][0][q] = words[q];
-                    }
-                }
-                const uint32_t bar = smem_u32(&ctl.k_full[stage]);
-                if (lane == 0) mbar_arrive_expect_tx(bar, static_cast<uint32_t>(nblk * bs * D * 2));
-                __syncwarp();
-                if (lane < nblk) {
-                    const uint32_t kb = sK + stage * L::KV_BYTES + lane * bs * 128u;
-#pragma unroll
-                    for (int h = 0; h < D / 64; ++h) tma_load_2d(kb + h * 16384u, &tmK, h * 64, row_base + j * bs, bar);
-                }
-            }
-            ++item_seq;
-        }
-    } else if (warp == 2) {
-        // =========================== V producer
-        int item_seq = 0;
-        uint32_t c_seq = 0;
-        bool ok = true;
-        while (ok) {
-            const int slot = item_seq & 1;
-            if (!wait_warp(smem_u32(&ctl.item_full[slot]), (item_seq >> 1) & 1, abort_flag)) break;
-            const int bh = ctl.item[slot][0];
-            const int qb = ctl.item[slot][1];
-            const int cnt = ctl.item[slot][2];
-            const int valid = ctl.item[slot][3];
-            __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(&ctl.item_empty[slot]));
-            if (!valid) break;
-            const int row_base = bh * static_cast<int>(g.Npad);
-            const int G = GRP ? a.G : 1;
-            const int32_t* list = a.kv_idx + (static_cast<long long>(bh) * g.nb + qb) * g.nb;
-            UnionWalk uw;
-            if (GRP) uw.init(a.gbits + (static_cast<long long>(bh) * a.ngroups + qb / G) * G * a.nwords, G, a.nwords,
-                             lane);
-            const int nc = (cnt + bpc - 1) / bpc;
-            int j_next = 0, n_next = 0;
-            uint32_t m_unused = 0u;
-            if (GRP) {
-                n_next = union_chunk<false>(uw, bpc, lane, j_next, m_unused);
-            } else {
-                n_next = min(bpc, cnt);
-                j_next = chunk_block(list, 0, bpc, n_next, lane, g.nb);
-            }
-            for (int cl = 0; cl < nc; ++cl, ++c_seq) {
-                const int stage = c_seq % V_STAGES;
-                const int nblk = n_next;
-                const int j = j_next;
-                if (cl + 1 < nc) {
-                    if (GRP) {
-                        n_next = union_chunk<false>(uw, bpc, lane, j_next, m_unused);
-                    } else {
-                        n_next = min(bpc, cnt - (cl + 1) * bpc);
-                        j_next = chunk_block(list, cl + 1, bpc, n_next, lane, g.nb);
-                    }
-                }
-                if (!wait_warp(smem_u32(&ctl.v_empty[stage]), ((c_seq / V_STAGES) & 1) ^ 1, abort_flag)) {
-                    ok = false;
-                    break;
-                }
-                const uint32_t bar = smem_u32(&ctl.v_full[stage]);
-                if (lane == 0) mbar_arrive_expect_tx(bar, static_cast<uint32_t>(nblk * bs * D * 2));
-                __syncwarp();
-                if (lane < nblk) {
-                    const uint32_t vb = sV + stage * L::KV_BYTES + lane * bs * 128u;
-#pragma unroll
-                    for (int h = 0; h < D / 64; ++h) tma_load_2d(vb + h * 16384u, &tmV, h * 64, row_base + j * bs, bar);
-                }
-            }
-            ++item_seq;
-        }
-    } else if (warp == 1 || warp == 3) {
-        // =========================== tensor-core issuers (one lane each)
-        // Chunk c of the CTA's stream goes to softmax group w = c & 1 (S_w,
-        // P_w, O_w).  Warp 1 issues S_w = Q K^T for every chunk, warp 3
-        // issues O_w += P_w V.  Two issuing threads keep the tensor pipe fed:
-        // while one waits on its barriers (a memory operation by the issuing
-        // thread stalls until its own MMAs drain) the other's MMAs run.
-        if (lane == 0) {
-            const bool qk_role = warp == 1;
-            constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, 128, false);
-            constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, D, true);
-            int item_seq = 0;
-            uint32_t c_seq = 0;
-            uint32_t n0 = 0u, n1 = 0u;   // chunks handled per group
-            unsigned long long blocks = 0;
-            bool ok = true;
-            while (ok) {
-                const int slot = item_seq & 1;
-                if (!wait_bar(smem_u32(&ctl.item_full[slot]), (item_seq >> 1) & 1, abort_flag)) break;
-                const int valid = ctl.item[slot][3];
-                const int cnt = ctl.item[slot][2];
-                mbar_arrive(smem_u32(&ctl.item_empty[slot]));
-                if (!valid) break;
-                const int nc = (cnt + bpc - 1) / bpc;
-                if (qk_role) {
-                    blocks += static_cast<unsigned long long>(cnt);
-                    if (!wait_bar(smem_u32(&ctl.q_full), item_seq & 1, abort_flag)) break;
-                } else {
-                    // the item's first PV waits until the previous item's
-                    // epilogue has read both accumulators
-                    if (!wait_bar(smem_u32(&ctl.o_free), (item_seq & 1) ^ 1, abort_flag)) break;
-                }
-                for (int cl = 0; cl < nc; ++cl) {
-                    const uint32_t c = c_seq + cl;
-                    const int w = c & 1;
-                    const uint32_t n = w ? n1 : n0;
-                    if (qk_role) {
-                        const int stage = c % KS;
-                        if (!wait_bar(smem_u32(&ctl.k_full[stage]), (c / KS) & 1, abort_flag) ||
-                            !wait_bar(smem_u32(&ctl.s_free[w]), (n & 1) ^ 1, abort_flag)) {
-                            ok = false;
-                            break;
-                        }
-                        tc_fence_after();
-                        const uint32_t kb = sK + stage * L::KV_BYTES;
-#pragma unroll
-                        for (int kk = 0; kk < D / 16; ++kk) {
-                            const uint32_t off = (kk >> 2) * 16384u + (kk & 3) * 32u;
-                            const uint64_t ad = sw128_desc(sQ + off, 16u, 1024u);
-                            const uint64_t bd = sw128_desc(kb + off, 16u, 1024u);
-                            mma_bf16_ss(tmem + static_cast<uint32_t>(w) * 128u, ad, bd, IDESC_QK, kk > 0 ? 1u : 0u);
-                        }
-                        mma_commit(smem_u32(&ctl.s_full[w]));
-                        mma_commit(smem_u32(&ctl.k_empty[stage]));
-                        if (cl == nc - 1) mma_commit(smem_u32(&ctl.q_empty));
-                    } else {
-                        const int stage = c % V_STAGES;
-                        if (!wait_bar(smem_u32(&ctl.p_full[w]), n & 1, abort_flag) ||
-                            !wait_bar(smem_u32(&ctl.v_full[stage]), (c / V_STAGES) & 1, abort_flag)) {
-                            ok = false;
-                            break;
-                        }
-                        tc_fence_after();
-                        const uint32_t vb = sV + stage * L::KV_BYTES;
-                        const uint32_t pb = sP + w * L::P_BYTES;
-                        const uint32_t od = tmem + O_COL + static_cast<uint32_t>(w) * 128u;
-                        const bool first = cl < 2;   // group w's first chunk of the item
-#pragma unroll
-                        for (int kk = 0; kk < 8; ++kk) {
-                            const uint64_t ad = sw128_desc(pb + (kk >> 2) * 16384u + (kk & 3) * 32u, 16u, 1024u);
-                            const uint64_t bd = sw128_desc(vb + kk * 2048u, 16384u, 1024u);
-                            mma_bf16_ss(od, ad, bd, IDESC_PV, (first && kk == 0) ? 0u : 1u);
-                        }
-                        mma_commit(smem_u32(&ctl.v_empty[stage]));
-                        mma_commit(smem_u32(&ctl.p_free[w]));
-                    }
-                    if (w) ++n1; else ++n0;
-                }
-                if (!ok) break;
-                c_seq += nc;
-                ++item_seq;
-            }
-            if (qk_role) ctl.blocks_done = blocks;
-        }
-        __syncwarp();
-    } else {
+    if (warp >= FIRST_SOFTMAX_WARP) {
+        regs_inc<REGS_HIGH>();
         // =========================== softmax groups (warps 4..7: w = 0, 8..11: w = 1)
         // Group w takes the chunks c with c & 1 == w: its own S_w, P_w and
         // O_w, running maximum m and sum l.  At the end of an item the two
         // groups exchange (m, l) per row and each writes half of the output
         // columns: O = (O_0 2^(m_0-M) + O_1 2^(m_1-M)) / (l_0 2^(m_0-M) + l_1 2^(m_1-M)).
+        // A chunk's whole S row is loaded into registers first and S_w is
+        // released at once, so the next S = Q K^T into S_w overlaps this
+        // chunk's exponentials; everything after the load works on registers.
         const int w = (warp - FIRST_SOFTMAX_WARP) >> 2;
         const int quad = warp & 3;                 // TMEM lanes 32*quad ..
         const int row = quad * 32 + lane;          // query row in the 128-row tile
@@ -591,7 +329,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         bool ok = true;
         while (ok) {
             const int slot = item_seq & 1;
-            if (!wait_warp(smem_u32(&ctl.item_full[slot]), (item_seq >> 1) & 1, abort_flag)) break;
+            if (!wait_warp(smem_u32(&ctl.item_full[slot]), (item_seq >> 1) & 1, abort_flag, wlim)) break;
             const int bh = ctl.item[slot][0];
             const int qb = ctl.item[slot][1];
             const int cnt = ctl.item[slot][2];
@@ -607,73 +345,71 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                 // chunk c = c_seq + cl has c & 1 == w
                 const uint32_t c = c_seq + cl;
                 const int kst = c % KS;
-                if (!wait_warp(smem_u32(&ctl.k_full[kst]), (c / KS) & 1, abort_flag) ||
-                    !wait_warp(smem_u32(&ctl.s_full[w]), n & 1, abort_flag)) {
+                if (!wait_warp(smem_u32(&ctl.k_full[kst]), (c / KS) & 1, abort_flag, wlim) ||
+                    !wait_warp(smem_u32(&ctl.s_full[w]), n & 1, abort_flag, wlim)) {
                     ok = false;
                     break;
                 }
+                tc_fence_after();
+                uint32_t sv[4][32];   // this row's 128 raw scores of the chunk
+#pragma unroll
+                for (int q = 0; q < 4; ++q) tmem_ld32(sb + q * 32u, sv[q]);
+                tmem_wait_ld();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(&ctl.s_free[w]));   // S_w read: the next QK may overwrite it
                 const uint32_t* mrow = ctl.mask[kst][tgrp];
-                const uint32_t mw0 = mrow[0], mw1 = mrow[1], mw2 = mrow[2], mw3 = mrow[3];
-                const bool partial = (mw0 & mw1 & mw2 & mw3) != 0xFFFFFFFFu;   // chunk holds masked keys
+                uint32_t mw[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) mw[q] = mrow[q];
                 __syncwarp();
                 if (lane == 0) mbar_arrive(smem_u32(&ctl.k_empty[kst]));   // mask in registers: stage free
-                tc_fence_after();
-                // Exp pass: P = 2^(s*scale*log2e + negv), row sum on fp32 pairs, bf16 P row into P_w
-                // (128-byte swizzle, K-major operand), two TMEM loads in flight.
+                // Exp pass: P = 2^(s*scale*log2e + negv) on fp32 pairs, row sum on fp32 pairs, bf16 P row
+                // into P_w (128-byte swizzle, K-major operand).  Words whose 32 keys are all visible skip
+                // the mask tests; words with none skip the exponentials.
                 unsigned long long sm2[4];   // four chains of (even, odd) column sums
-                float mx[8];
                 auto exp_pass = [&](float negv) {
 #pragma unroll
                     for (int i = 0; i < 4; ++i) sm2[i] = 0ull;
                     const unsigned long long sl2x2 = f2_pack(sl2, sl2), negx2 = f2_pack(negv, negv);
-#pragma unroll 1
-                    for (int q2 = 0; q2 < 4; q2 += 2) {
-                        uint32_t v[2][32];
-                        tmem_ld32(sb + q2 * 32u, v[0]);
-                        tmem_ld32(sb + q2 * 32u + 32u, v[1]);
-                        tmem_wait_ld();
 #pragma unroll
-                        for (int hq = 0; hq < 2; ++hq) {
-                            const int q = q2 + hq;
-                            const uint32_t mword = q == 0 ? mw0 : (q == 1 ? mw1 : (q == 2 ? mw2 : mw3));
-                            uint32_t wv[16];
-                            if (mword == 0xFFFFFFFFu) {
-                                // every key of these 32 columns is visible
+                    for (int q = 0; q < 4; ++q) {
+                        const uint32_t mword = mw[q];
+                        uint32_t wv[16];
+                        if (mword == 0xFFFFFFFFu) {
 #pragma unroll
-                                for (int i = 0; i < 32; i += 2) {
-                                    const float s0 = __uint_as_float(v[hq][i]), s1 = __uint_as_float(v[hq][i + 1]);
-                                    float x0, x1;
-                                    f2_unpack(f2_fma(f2_pack(s0, s1), sl2x2, negx2), x0, x1);
-                                    const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
-                                    sm2[(i >> 1) & 3] = f2_add(sm2[(i >> 1) & 3], f2_pack(p0, p1));
-                                    wv[i >> 1] = pack_bf16x2(p0, p1);
-                                }
-                            } else if (mword == 0u) {
-                                // no visible key here: P = 0, nothing to the sum or the maximum
-#pragma unroll
-                                for (int i = 0; i < 16; ++i) wv[i] = 0u;
-                            } else {
-#pragma unroll
-                                for (int i = 0; i < 32; i += 2) {
-                                    const float s0 = __uint_as_float(v[hq][i]), s1 = __uint_as_float(v[hq][i + 1]);
-                                    float x0, x1;
-                                    f2_unpack(f2_fma(f2_pack(s0, s1), sl2x2, negx2), x0, x1);
-                                    const bool k0 = (mword >> i) & 1u, k1 = (mword >> (i + 1)) & 1u;
-                                    const float p0 = k0 ? ex2_approx(x0) : 0.f;
-                                    const float p1 = k1 ? ex2_approx(x1) : 0.f;
-                                    sm2[(i >> 1) & 3] = f2_add(sm2[(i >> 1) & 3], f2_pack(p0, p1));
-                                    wv[i >> 1] = pack_bf16x2(p0, p1);
-                                }
+                            for (int i = 0; i < 32; i += 2) {
+                                float x0, x1;
+                                f2_unpack(f2_fma(f2_pack(__uint_as_float(sv[q][i]), __uint_as_float(sv[q][i + 1])),
+                                                 sl2x2, negx2), x0, x1);
+                                const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+                                sm2[(i >> 1) & 3] = f2_add(sm2[(i >> 1) & 3], f2_pack(p0, p1));
+                                wv[i >> 1] = pack_bf16x2(p0, p1);
                             }
-                            const int half = q >> 1;
+                        } else if (mword == 0u) {
 #pragma unroll
-                            for (int k4 = 0; k4 < 4; ++k4) {
-                                const int chunk = (((q & 1) << 2) | k4) ^ (row & 7);
-                                const uint32_t addr = pbase + half * 16384u + chunk * 16u;
-                                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(wv[4 * k4]),
-                                             "r"(wv[4 * k4 + 1]), "r"(wv[4 * k4 + 2]), "r"(wv[4 * k4 + 3])
-                                             : "memory");
+                            for (int i = 0; i < 16; ++i) wv[i] = 0u;
+                        } else {
+#pragma unroll
+                            for (int i = 0; i < 32; i += 2) {
+                                float x0, x1;
+                                f2_unpack(f2_fma(f2_pack(__uint_as_float(sv[q][i]), __uint_as_float(sv[q][i + 1])),
+                                                 sl2x2, negx2), x0, x1);
+                                const bool k0 = (mword >> i) & 1u, k1 = (mword >> (i + 1)) & 1u;
+                                const float p0 = k0 ? ex2_approx(x0) : 0.f;
+                                const float p1 = k1 ? ex2_approx(x1) : 0.f;
+                                sm2[(i >> 1) & 3] = f2_add(sm2[(i >> 1) & 3], f2_pack(p0, p1));
+                                wv[i >> 1] = pack_bf16x2(p0, p1);
                             }
+                        }
+                        const int half = q >> 1;
+#pragma unroll
+                        for (int k4 = 0; k4 < 4; ++k4) {
+                            const int chunk = (((q & 1) << 2) | k4) ^ (row & 7);
+                            const uint32_t addr = pbase + half * 16384u + chunk * 16u;
+                            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(wv[4 * k4]),
+                                         "r"(wv[4 * k4 + 1]), "r"(wv[4 * k4 + 2]), "r"(wv[4 * k4 + 3])
+                                         : "memory");
                         }
                     }
                 };
@@ -690,30 +426,21 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                     }
                     tmem_wait_st();
                 };
-                // Row maximum of the visible raw scores of this chunk (scaled to log2 units).
+                // Row maximum of the visible raw scores of this chunk (scaled to log2 units); -inf for a
+                // row that sees no key of its block in this chunk.
                 auto max_pass = [&]() -> float {
+                    float mx[8];
 #pragma unroll
                     for (int i = 0; i < 8; ++i) mx[i] = -INFINITY;
 #pragma unroll
-                    for (int q2 = 0; q2 < 4; q2 += 2) {
-                        uint32_t sr[2][32];
-                        tmem_ld32(sb + q2 * 32u, sr[0]);
-                        tmem_ld32(sb + q2 * 32u + 32u, sr[1]);
-                        tmem_wait_ld();
-                        if (partial) {
-                            const uint32_t mwa = q2 == 0 ? mw0 : mw2, mwb = q2 == 0 ? mw1 : mw3;
+                    for (int q = 0; q < 4; ++q) {
+                        const uint32_t mword = mw[q];
 #pragma unroll
-                            for (int i = 0; i < 32; ++i) {
-                                if (!((mwa >> i) & 1u)) sr[0][i] = 0xFF800000u;
-                                if (!((mwb >> i) & 1u)) sr[1][i] = 0xFF800000u;
-                            }
+                        for (int i = 0; i < 32; i += 2) {
+                            const float a0 = ((mword >> i) & 1u) ? __uint_as_float(sv[q][i]) : -INFINITY;
+                            const float a1 = ((mword >> (i + 1)) & 1u) ? __uint_as_float(sv[q][i + 1]) : -INFINITY;
+                            mx[(i >> 1) & 7] = fmax3(mx[(i >> 1) & 7], a0, a1);
                         }
-#pragma unroll
-                        for (int hq = 0; hq < 2; ++hq)
-#pragma unroll
-                            for (int i = 0; i < 32; i += 2)
-                                mx[(i >> 1) & 7] = fmax3(mx[(i >> 1) & 7], __uint_as_float(sr[hq][i]),
-                                                         __uint_as_float(sr[hq][i + 1]));
                     }
                     return fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
                                  fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * sl2;
@@ -724,45 +451,41 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                     for (int i = 0; i < 4; ++i) f2_unpack(sm2[i], sm[2 * i], sm[2 * i + 1]);
                     return ((sm[0] + sm[1]) + (sm[2] + sm[3])) + ((sm[4] + sm[5]) + (sm[6] + sm[7]));
                 };
+                // P_w and O_w were last used by this group's previous PV
+                if (!wait_warp(smem_u32(&ctl.p_free[w]), (n & 1) ^ 1, abort_flag, wlim)) {
+                    ok = false;
+                    break;
+                }
+                // The group's first chunk of an item takes the row maximum first and computes P against
+                // it (a row may see no key of its block in a chunk: it keeps max -inf, P 0).  Later chunks
+                // make one pass against the running reference maximum; while a row's sum stays at or
+                // below RESCALE_SUM_LIMIT no P of it can overflow anything.  Otherwise (or for a row that
+                // had seen no key yet) the chunk is redone from the registers: exact maximum, O rescaled,
+                // P recomputed against it.
                 float alpha = 1.0f;
                 float sum;
-                if (!mine_any) {
-                    // the group's first chunk of the item: row maximum first, then P against it
-                    // (a row may see no key of its block in a chunk: it keeps max -inf, P 0)
-                    m_ref = max_pass();
-                    // P_w was last used by this group's previous PV
-                    if (!wait_warp(smem_u32(&ctl.p_free[w]), (n & 1) ^ 1, abort_flag)) {
-                        ok = false;
-                        break;
-                    }
-                    exp_pass(-m_ref);
-                    sum = chunk_sum();
-                } else {
-                    // later chunks: one pass against the running reference maximum.  While a row's sum
-                    // stays below 2^RESCALE_LOG2_SUM no P of it can overflow anything; otherwise (or for
-                    // a row that had seen no key yet) the chunk is redone: exact maximum, O rescaled,
-                    // P recomputed against it.
-                    if (!wait_warp(smem_u32(&ctl.p_free[w]), (n & 1) ^ 1, abort_flag)) {
-                        ok = false;
-                        break;
-                    }
-                    exp_pass(-m_ref);
-                    sum = chunk_sum();
-                    const bool big = !(sum <= RESCALE_SUM_LIMIT);
-                    if (__any_sync(0xffffffffu, big)) {
+                bool big = false;
+                bool exact = !mine_any;
+                for (;;) {
+                    if (exact) {
                         const float mxs = max_pass();
-                        const bool grow = big && mxs > m_ref;
-                        const float m_new = grow ? mxs : m_ref;
-                        alpha = grow ? ex2_approx(m_ref - m_new) : 1.0f;
-                        m_ref = m_new;
-                        rescale_o(alpha);
-                        exp_pass(-m_ref);
-                        sum = chunk_sum();
+                        if (!mine_any) {
+                            m_ref = mxs;
+                        } else {
+                            const bool grow = big && mxs > m_ref;
+                            const float m_new = grow ? mxs : m_ref;
+                            alpha = grow ? ex2_approx(m_ref - m_new) : 1.0f;
+                            m_ref = m_new;
+                            rescale_o(alpha);
+                        }
                     }
+                    exp_pass(-m_ref);
+                    sum = chunk_sum();
+                    if (exact) break;
+                    big = !(sum <= RESCALE_SUM_LIMIT);
+                    if (!__any_sync(0xffffffffu, big)) break;
+                    exact = true;
                 }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(smem_u32(&ctl.s_free[w]));   // S_w consumed
                 l = l * alpha + sum;
                 fence_proxy_async_smem();
                 tc_fence_before();
@@ -773,13 +496,13 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
             }
             if (!ok) break;
             // ---- epilogue: wait for this group's last PV, swap (m, l), merge
-            if (mine_any && !wait_warp(smem_u32(&ctl.p_free[w]), (n & 1) ^ 1, abort_flag)) break;
-            if (!wait_warp(smem_u32(&ctl.mrg_empty), (item_seq & 1) ^ 1, abort_flag)) break;
+            if (mine_any && !wait_warp(smem_u32(&ctl.p_free[w]), (n & 1) ^ 1, abort_flag, wlim)) break;
+            if (!wait_warp(smem_u32(&ctl.mrg_empty), (item_seq & 1) ^ 1, abort_flag, wlim)) break;
             ctl.mrg_m[w][row] = m_ref;
             ctl.mrg_l[w][row] = l;
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(&ctl.mrg_full));
-            if (!wait_warp(smem_u32(&ctl.mrg_full), item_seq & 1, abort_flag)) break;
+            if (!wait_warp(smem_u32(&ctl.mrg_full), item_seq & 1, abort_flag, wlim)) break;
             const float m0 = ctl.mrg_m[0][row], m1 = ctl.mrg_m[1][row];
             const float l0 = ctl.mrg_l[0][row], l1 = ctl.mrg_l[1][row];
             __syncwarp();
@@ -854,6 +577,317 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
             if (lane == 0) mbar_arrive(smem_u32(&ctl.o_free));
             c_seq += nc;
             ++item_seq;
+        }
+    } else {
+        regs_dec<REGS_LOW>();
+        if (warp == 0) {
+            // =========================== K producer: items, Q tile, K blocks, masks
+            // Column col = q*32 + lane of a chunk is token `off` of slot `slot`;
+            // its frame / row / col offsets inside the tile never change.
+            int c_slot[4], c_of[4], c_oy[4], c_ox[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int col = q * 32 + lane;
+                c_slot[q] = col / bs;
+                const int off = col - c_slot[q] * bs;
+                c_ox[q] = off % g.tw;
+                c_oy[q] = (off / g.tw) % g.th;
+                c_of[q] = off / (g.tw * g.th);
+            }
+            int item_seq = 0;
+            uint32_t c_seq = 0;      // K chunks loaded
+            uint32_t q_fills = 0;    // Q tiles loaded
+            bool ok = true;
+            while (ok) {
+                const int slot = item_seq & 1;
+                if (!wait_warp(smem_u32(&ctl.item_empty[slot]), ((item_seq >> 1) & 1) ^ 1, abort_flag, wlim)) break;
+                int t = 0;
+                if (lane == 0) t = atomicAdd(a.counter, 1);
+                t = __shfl_sync(0xffffffffu, t, 0);
+                if (t >= a.total_items) {
+                    if (lane == 0) {
+                        ctl.item[slot][3] = 0;
+                        mbar_arrive(smem_u32(&ctl.item_full[slot]));
+                    }
+                    break;
+                }
+                const int G = GRP ? a.G : 1;
+                const int units = GRP ? a.ngroups : g.nb;
+                const int hs = t / units;
+                const int r = t - hs * units;
+                const int bh = __ldg(a.head_order + hs);
+                const int u = __ldg(a.item_order + static_cast<long long>(bh) * units + r);
+                const int qb = u * G;                     // first query block of the tile
+                const int nq = min(G, g.nb - qb);         // query blocks in the tile
+                int cnt = GRP ? __ldg(a.gcnt + static_cast<long long>(bh) * a.ngroups + u)
+                              : __ldg(a.kv_cnt + static_cast<long long>(bh) * g.nb + qb);
+                if (cnt < 1 || cnt > g.nb) {
+                    if (lane == 0) record_status(FVATTN_ERR_BOUNDS);
+                    cnt = cnt < 1 ? 1 : g.nb;
+                }
+                if (lane == 0) {
+                    ctl.item[slot][0] = bh;
+                    ctl.item[slot][1] = qb;
+                    ctl.item[slot][2] = cnt;
+                    ctl.item[slot][3] = 1;
+                    mbar_arrive(smem_u32(&ctl.item_full[slot]));
+                }
+                if (!wait_warp(smem_u32(&ctl.q_empty), (item_seq & 1) ^ 1, abort_flag, wlim)) break;
+                const int row_base = bh * static_cast<int>(g.Npad);
+                ++q_fills;
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(smem_u32(&ctl.q_full), static_cast<uint32_t>(nq * bs * D * 2));
+                    for (int tq = 0; tq < (GRP ? nq : 1); ++tq)
+#pragma unroll
+                        for (int h = 0; h < D / 64; ++h)
+                            tma_load_2d(sQ + h * 16384u + static_cast<uint32_t>(tq * bs) * 128u, &tmQ, h * 64,
+                                        row_base + (qb + tq) * bs, smem_u32(&ctl.q_full));
+                }
+                const int32_t* list = a.kv_idx + (static_cast<long long>(bh) * g.nb + qb) * g.nb;
+                UnionWalk uw;
+                if (GRP) uw.init(a.gbits + (static_cast<long long>(bh) * a.ngroups + u) * G * a.nwords, G, a.nwords, lane);
+                const int nc = (cnt + bpc - 1) / bpc;
+                // chunk cl's blocks (lane s < nblk: slot s) and membership bits, one chunk ahead
+                int j_next = 0, n_next = 0;
+                uint32_t m_next = 0u;
+                if (GRP) {
+                    n_next = union_chunk<true>(uw, bpc, lane, j_next, m_next);
+                } else {
+                    n_next = min(bpc, cnt);
+                    j_next = chunk_block(list, 0, bpc, n_next, lane, g.nb);
+                    m_next = 1u;
+                }
+                for (int cl = 0; cl < nc; ++cl, ++c_seq) {
+                    const int stage = c_seq % KS;
+                    const int nblk = n_next;
+                    const int j = j_next;
+                    const uint32_t mem = m_next;
+                    if (cl + 1 < nc) {
+                        if (GRP) {
+                            n_next = union_chunk<true>(uw, bpc, lane, j_next, m_next);
+                        } else {
+                            n_next = min(bpc, cnt - (cl + 1) * bpc);
+                            j_next = chunk_block(list, cl + 1, bpc, n_next, lane, g.nb);
+                        }
+                    }
+                    const int ext = lane < nblk ? __ldg(a.ext + j) : 0;
+                    if (!wait_warp(smem_u32(&ctl.k_empty[stage]), ((c_seq / KS) & 1) ^ 1, abort_flag, wlim)) {
+                        ok = false;
+                        break;
+                    }
+                    if (GRP) {
+                        // per query block t of the tile: key column real and its block in t's list.
+                        // Real-token bits once per 32-column word; a word lies in one slot when
+                        // bs >= 32, so its membership bits are warp-uniform there.
+                        uint32_t pad[4], mq[4];
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            const int e = __shfl_sync(0xffffffffu, ext, c_slot[q]);
+                            mq[q] = __shfl_sync(0xffffffffu, mem, c_slot[q]);
+                            pad[q] = __ballot_sync(0xffffffffu, (c_of[q] < (e & 255)) && (c_oy[q] < ((e >> 8) & 255)) &&
+                                                                    (c_ox[q] < (e >> 16)));
+                        }
+                        for (int tq = 0; tq < G; ++tq) {
+                            uint32_t words[4];
+#pragma unroll
+                            for (int q = 0; q < 4; ++q)
+                                words[q] = bs >= 32 ? (((mq[q] >> tq) & 1u) ? pad[q] : 0u)
+                                                    : (pad[q] & __ballot_sync(0xffffffffu, (mq[q] >> tq) & 1u));
+                            if (lane == 0) {
+#pragma unroll
+                                for (int q = 0; q < 4; ++q) ctl.mask[stage][tq][q] = words[q];
+                            }
+                        }
+                    } else {
+                        (void)mem;
+                        uint32_t words[4];
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            const int e = __shfl_sync(0xffffffffu, ext, c_slot[q]);
+                            const bool valid = (c_of[q] < (e & 255)) && (c_oy[q] < ((e >> 8) & 255)) && (c_ox[q] < (e >> 16));
+                            words[q] = __ballot_sync(0xffffffffu, valid);
+                        }
+                        if (lane == 0) {
+#pragma unroll
+                            for (int q = 0; q < 4; ++q) ctl.mask[stage][0][q] = words[q];
+                        }
+                    }
+                    const uint32_t bar = smem_u32(&ctl.k_full[stage]);
+                    if (lane == 0) mbar_arrive_expect_tx(bar, static_cast<uint32_t>(nblk * bs * D * 2));
+                    __syncwarp();
+                    if (lane < nblk) {
+                        const uint32_t kb = sK + stage * L::KV_BYTES + lane * bs * 128u;
+#pragma unroll
+                        for (int h = 0; h < D / 64; ++h) tma_load_2d(kb + h * 16384u, &tmK, h * 64, row_base + j * bs, bar);
+                    }
+                }
+                ++item_seq;
+            }
+            // On the way out (also after an abort): wait for this warp's own loads in flight, the last
+            // fill of every stage, so no copy into shared memory outlives the CTA.
+            if (lane == 0) {
+                if (q_fills > 0) wait_bar_drain(smem_u32(&ctl.q_full), (q_fills - 1) & 1, wlim);
+                for (int st = 0; st < KS; ++st) {
+                    const uint32_t fills = c_seq > static_cast<uint32_t>(st) ? (c_seq - st + KS - 1) / KS : 0u;
+                    if (fills > 0) wait_bar_drain(smem_u32(&ctl.k_full[st]), (fills - 1) & 1, wlim);
+                }
+            }
+            __syncwarp();
+        } else if (warp == 2) {
+            // =========================== V producer
+            int item_seq = 0;
+            uint32_t c_seq = 0;      // V chunks loaded
+            // fault injection: this warp leaves at once, loading and arriving nothing, so the PV issuer's
+            // wait for V must run out
+            bool ok = (a.hooks & FVATTN_HOOK_SKIP_V_LOADS) == 0;
+            while (ok) {
+                const int slot = item_seq & 1;
+                if (!wait_warp(smem_u32(&ctl.item_full[slot]), (item_seq >> 1) & 1, abort_flag, wlim)) break;
+                const int bh = ctl.item[slot][0];
+                const int qb = ctl.item[slot][1];
+                const int cnt = ctl.item[slot][2];
+                const int valid = ctl.item[slot][3];
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(&ctl.item_empty[slot]));
+                if (!valid) break;
+                const int row_base = bh * static_cast<int>(g.Npad);
+                const int G = GRP ? a.G : 1;
+                const int32_t* list = a.kv_idx + (static_cast<long long>(bh) * g.nb + qb) * g.nb;
+                UnionWalk uw;
+                if (GRP) uw.init(a.gbits + (static_cast<long long>(bh) * a.ngroups + qb / G) * G * a.nwords, G, a.nwords,
+                                 lane);
+                const int nc = (cnt + bpc - 1) / bpc;
+                int j_next = 0, n_next = 0;
+                uint32_t m_unused = 0u;
+                if (GRP) {
+                    n_next = union_chunk<false>(uw, bpc, lane, j_next, m_unused);
+                } else {
+                    n_next = min(bpc, cnt);
+                    j_next = chunk_block(list, 0, bpc, n_next, lane, g.nb);
+                }
+                for (int cl = 0; cl < nc; ++cl, ++c_seq) {
+                    const int stage = c_seq % V_STAGES;
+                    const int nblk = n_next;
+                    const int j = j_next;
+                    if (cl + 1 < nc) {
+                        if (GRP) {
+                            n_next = union_chunk<false>(uw, bpc, lane, j_next, m_unused);
+                        } else {
+                            n_next = min(bpc, cnt - (cl + 1) * bpc);
+                            j_next = chunk_block(list, cl + 1, bpc, n_next, lane, g.nb);
+                        }
+                    }
+                    if (!wait_warp(smem_u32(&ctl.v_empty[stage]), ((c_seq / V_STAGES) & 1) ^ 1, abort_flag, wlim)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t bar = smem_u32(&ctl.v_full[stage]);
+                    if (lane == 0) mbar_arrive_expect_tx(bar, static_cast<uint32_t>(nblk * bs * D * 2));
+                    __syncwarp();
+                    if (lane < nblk) {
+                        const uint32_t vb = sV + stage * L::KV_BYTES + lane * bs * 128u;
+#pragma unroll
+                        for (int h = 0; h < D / 64; ++h) tma_load_2d(vb + h * 16384u, &tmV, h * 64, row_base + j * bs, bar);
+                    }
+                }
+                ++item_seq;
+            }
+            if (lane == 0) {
+                for (int st = 0; st < V_STAGES; ++st) {
+                    const uint32_t fills =
+                        c_seq > static_cast<uint32_t>(st) ? (c_seq - st + V_STAGES - 1) / V_STAGES : 0u;
+                    if (fills > 0) wait_bar_drain(smem_u32(&ctl.v_full[st]), (fills - 1) & 1, wlim);
+                }
+            }
+            __syncwarp();
+        } else if (warp == 1 || warp == 3) {
+            // =========================== tensor-core issuers (one lane each)
+            // Chunk c of the CTA's stream goes to softmax group w = c & 1 (S_w,
+            // P_w, O_w).  Warp 1 issues S_w = Q K^T for every chunk, warp 3
+            // issues O_w += P_w V.  Two issuing threads keep the tensor pipe fed:
+            // while one waits on its barriers (a memory operation by the issuing
+            // thread stalls until its own MMAs drain) the other's MMAs run.
+            if (lane == 0) {
+                const bool qk_role = warp == 1;
+                constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, 128, false);
+                constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, D, true);
+                int item_seq = 0;
+                uint32_t c_seq = 0;
+                uint32_t n0 = 0u, n1 = 0u;   // chunks handled per group
+                unsigned long long blocks = 0;
+                bool ok = true;
+                while (ok) {
+                    const int slot = item_seq & 1;
+                    if (!wait_bar(smem_u32(&ctl.item_full[slot]), (item_seq >> 1) & 1, abort_flag, wlim)) break;
+                    const int valid = ctl.item[slot][3];
+                    const int cnt = ctl.item[slot][2];
+                    mbar_arrive(smem_u32(&ctl.item_empty[slot]));
+                    if (!valid) break;
+                    const int nc = (cnt + bpc - 1) / bpc;
+                    if (qk_role) {
+                        blocks += static_cast<unsigned long long>(cnt);
+                        if (!wait_bar(smem_u32(&ctl.q_full), item_seq & 1, abort_flag, wlim)) break;
+                    } else {
+                        // the item's first PV waits until the previous item's
+                        // epilogue has read both accumulators
+                        if (!wait_bar(smem_u32(&ctl.o_free), (item_seq & 1) ^ 1, abort_flag, wlim)) break;
+                    }
+                    for (int cl = 0; cl < nc; ++cl) {
+                        const uint32_t c = c_seq + cl;
+                        const int w = c & 1;
+                        const uint32_t n = w ? n1 : n0;
+                        if (qk_role) {
+                            const int stage = c % KS;
+                            if (!wait_bar(smem_u32(&ctl.k_full[stage]), (c / KS) & 1, abort_flag, wlim) ||
+                                !wait_bar(smem_u32(&ctl.s_free[w]), (n & 1) ^ 1, abort_flag, wlim)) {
+                                ok = false;
+                                break;
+                            }
+                            tc_fence_after();
+                            const uint32_t kb = sK + stage * L::KV_BYTES;
+#pragma unroll
+                            for (int kk = 0; kk < D / 16; ++kk) {
+                                const uint32_t off = (kk >> 2) * 16384u + (kk & 3) * 32u;
+                                const uint64_t ad = sw128_desc(sQ + off, 16u, 1024u);
+                                const uint64_t bd = sw128_desc(kb + off, 16u, 1024u);
+                                mma_bf16_ss(tmem + static_cast<uint32_t>(w) * 128u, ad, bd, IDESC_QK, kk > 0 ? 1u : 0u);
+                            }
+                            mma_commit(smem_u32(&ctl.s_full[w]));
+                            mma_commit(smem_u32(&ctl.k_empty[stage]));
+                            if (cl == nc - 1) mma_commit(smem_u32(&ctl.q_empty));
+                        } else {
+                            const int stage = c % V_STAGES;
+                            if (!wait_bar(smem_u32(&ctl.p_full[w]), n & 1, abort_flag, wlim) ||
+                                !wait_bar(smem_u32(&ctl.v_full[stage]), (c / V_STAGES) & 1, abort_flag, wlim)) {
+                                ok = false;
+                                break;
+                            }
+                            tc_fence_after();
+                            const uint32_t vb = sV + stage * L::KV_BYTES;
+                            const uint32_t pb = sP + w * L::P_BYTES;
+                            const uint32_t od = tmem + O_COL + static_cast<uint32_t>(w) * 128u;
+                            const bool first = cl < 2;   // group w's first chunk of the item
+#pragma unroll
+                            for (int kk = 0; kk < 8; ++kk) {
+                                const uint64_t ad = sw128_desc(pb + (kk >> 2) * 16384u + (kk & 3) * 32u, 16u, 1024u);
+                                const uint64_t bd = sw128_desc(vb + kk * 2048u, 16384u, 1024u);
+                                mma_bf16_ss(od, ad, bd, IDESC_PV, (first && kk == 0) ? 0u : 1u);
+                            }
+                            mma_commit(smem_u32(&ctl.v_empty[stage]));
+                            mma_commit(smem_u32(&ctl.p_free[w]));
+                        }
+                        if (w) ++n1; else ++n0;
+                    }
+                    if (!ok) break;
+                    c_seq += nc;
+                    ++item_seq;
+                }
+                if (qk_role) ctl.blocks_done = blocks;
+                // every MMA this thread issued has completed (and made its commits) before the TMEM release
+                mma_commit(smem_u32(&ctl.drain[qk_role ? 0 : 1]));
+                wait_bar_drain(smem_u32(&ctl.drain[qk_role ? 0 : 1]), 0, wlim);
+            }
+            __syncwarp();
         }
     }
 
@@ -1021,6 +1055,10 @@ static WsLayout ws_layout(const fvattn_geom& g) {
     return w;
 }
 
+// Fault-injection settings of fvattn_test_hook (0: normal operation).
+static std::atomic<unsigned long long> g_hook_wait_limit_ns{0};
+static std::atomic<int> g_hook_flags{0};
+
 static int cached_num_sms() {
     int dev = 0, n = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return 0;
@@ -1037,6 +1075,12 @@ static int launch_attn(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
     if (cudaFuncSetAttribute(sparse_attn_kernel<D, GRP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(L::ALLOC)) != cudaSuccess)
         return FVATTN_ERR_CUDA;
+    // The warpgroups' register shares (setmaxnreg) must fit in what a CTA is
+    // launched with, or the raising warpgroups would wait for ever.
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, sparse_attn_kernel<D, GRP>) != cudaSuccess) return FVATTN_ERR_CUDA;
+    if (static_cast<long long>(fa.numRegs) * ATT_THREADS < 128ll * REGS_LOW + 256ll * REGS_HIGH)
+        return FVATTN_ERR_UNSUPPORTED;
     sparse_attn_kernel<D, GRP><<<grid, ATT_THREADS, L::ALLOC, s>>>(tq, tk, tv, args);
     FV_CHECK_LAUNCH();
     return FVATTN_OK;
@@ -1052,6 +1096,13 @@ extern "C" size_t fvattn_attn_workspace_size(const fvattn_geom* gp) {
 }
 
 extern "C" int fvattn_num_sms(void) { return cached_num_sms(); }
+
+extern "C" int fvattn_test_hook(unsigned long long wait_limit_ns, int flags) {
+    if ((flags & ~FVATTN_HOOK_SKIP_V_LOADS) != 0) return FVATTN_ERR_INVALID;
+    g_hook_wait_limit_ns.store(wait_limit_ns);
+    g_hook_flags.store(flags);
+    return FVATTN_OK;
+}
 
 static int attn_impl(const fvattn_geom* gp, const void* q_t, const void* k_t, const void* v_t, const int32_t* kv_idx,
                      const int32_t* kv_cnt, float scale, void* o_t, int raster, unsigned long long* sm_stats,
@@ -1115,6 +1166,9 @@ static int attn_impl(const fvattn_geom* gp, const void* q_t, const void* k_t, co
     args.gcnt = gcnt;
     args.ext = ext;
     args.total_items = BH * units;
+    const unsigned long long hook_limit = g_hook_wait_limit_ns.load();
+    args.wait_limit_ns = hook_limit ? hook_limit : WAIT_LIMIT_NS;
+    args.hooks = g_hook_flags.load();
     int nsm = cached_num_sms();
     if (nsm <= 0) return FVATTN_ERR_CUDA;
     const int grid = nsm;
@@ -1138,3 +1192,5 @@ extern "C" int fvattn_sparse_attn_raster(const fvattn_geom* gp, const void* q_t,
                                          fvattn_stream_t stream) {
     return attn_impl(gp, q_t, k_t, v_t, kv_idx, kv_cnt, scale, o, 1, sm_stats, workspace, ws_bytes, stream);
 }
+
+int fv::take_status_attn() { return fv::take_tu_status(); }

@@ -27,12 +27,31 @@ inline Geo to_geo(const fvattn_geom& g) {
     return k;
 }
 
-// Device status word (FVATTN_OK or the first error a kernel recorded).
-extern __device__ int g_fvattn_status;
+// Device status word of this translation unit: FVATTN_OK or the first error
+// one of its kernels recorded.  Every .cu file is compiled as a whole
+// program (no relocatable device code: ptxas then honours the per-warpgroup
+// register budgets of setmaxnreg), so each owns one word;
+// fvattn_get_status reads and clears them all through the take_status_*
+// functions below.
+static __device__ int g_tu_status = 0;
 
 __device__ __forceinline__ void record_status(int code) {
-    atomicCAS(&g_fvattn_status, 0, code);
+    atomicCAS(&g_tu_status, 0, code);
 }
+
+// Host side: read this translation unit's status word on the current device
+// and clear it; FVATTN_ERR_CUDA if the copy fails.
+static inline int take_tu_status() {
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_tu_status, sizeof(int)) != cudaSuccess) return FVATTN_ERR_CUDA;
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_tu_status, &zero, sizeof(int)) != cudaSuccess) return FVATTN_ERR_CUDA;
+    return v;
+}
+
+// The status words of the files whose kernels record errors.
+int take_status_route();
+int take_status_attn();
 
 // Raster tile index of a block, and block of a raster tile (identities in
 // raster tile order).

@@ -245,6 +245,24 @@ __device__ __forceinline__ void pdl_launch_dependents() {
 // no-op when this grid was launched without the programmatic attribute).
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
+// ---------------------------------------------------------------- register split
+
+// Per-warpgroup register budget (setmaxnreg; every warp of the warpgroup
+// executes the same instruction).  .dec returns registers to the CTA's
+// pool, .inc takes them from it and waits until they are there: the
+// warpgroups' shares must add up to no more than the CTA was launched with.
+template <uint32_t N>
+__device__ __forceinline__ void regs_dec() {
+    static_assert(N >= 24 && N <= 256 && N % 8 == 0, "setmaxnreg count");
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
+template <uint32_t N>
+__device__ __forceinline__ void regs_inc() {
+    static_assert(N >= 24 && N <= 256 && N % 8 == 0, "setmaxnreg count");
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // ---------------------------------------------------------------- misc
 
 __device__ __forceinline__ float ex2_approx(float x) {

@@ -894,3 +894,5 @@ extern "C" int fvattn_reorder_route(const fvattn_geom* gp, const void* q, const 
     return route_impl(gp, q, k, q_tiled, k_tiled, p, k_floor, k_extra, scale, kv_idx, kv_cnt, q_pool, k_pool, logits,
                       workspace, ws_bytes, stream);
 }
+
+int fv::take_status_route() { return fv::take_tu_status(); }

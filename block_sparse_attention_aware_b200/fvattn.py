@@ -26,7 +26,7 @@ EXPORTED = ("fvattn_geom_init", "fvattn_block_order", "fvattn_copy_heads", "fvat
             "fvattn_attn_workspace_size",
             "fvattn_num_sms", "fvattn_sparse_attn", "fvattn_sparse_attn_raster", "fvattn_sparse_attn_noalloc",
             "fvattn_get_status",
-            "fvattn_status_string")
+            "fvattn_status_string", "fvattn_test_hook")
 
 
 class FVAttnError(RuntimeError):
@@ -89,6 +89,8 @@ def load(path: str = LIB_PATH):
     L.fvattn_get_status.restype = I
     L.fvattn_status_string.argtypes = [I]
     L.fvattn_status_string.restype = ctypes.c_char_p
+    L.fvattn_test_hook.argtypes = [ctypes.c_ulonglong, I]
+    L.fvattn_test_hook.restype = I
     _lib = L
     return L
 
@@ -369,6 +371,16 @@ def sparse_attn_noalloc(g: Geom, qt, kt, vt, kv_idx, kv_cnt, scale: Optional[flo
                                            _stream(stream))
     _check("fvattn_sparse_attn_noalloc", rc)
     return out
+
+
+HOOK_SKIP_V_LOADS = 1   # FVATTN_HOOK_SKIP_V_LOADS
+
+
+def test_hook(wait_limit_ns: int = 0, flags: int = 0) -> None:
+    """fvattn_test_hook: fault injection for failure-path tests (a shorter
+    wait limit; FVATTN_HOOK_SKIP_V_LOADS).  test_hook() restores normal
+    operation."""
+    _check("fvattn_test_hook", load().fvattn_test_hook(int(wait_limit_ns), int(flags)))
 
 
 def get_status(stream=None) -> int:

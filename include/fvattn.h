@@ -283,10 +283,29 @@ int fvattn_sparse_attn_noalloc(const fvattn_geom *g, const void *q_t, const void
                                const int32_t *kv_idx, const int32_t *kv_cnt, float scale,
                                void *o_t, unsigned long long *sm_stats, fvattn_stream_t stream);
 
-/* Synchronise `stream`, read and clear the device status word, and return
- * it (FVATTN_OK, FVATTN_ERR_TIMEOUT or FVATTN_ERR_BOUNDS), or
+/* Synchronise `stream`, read and clear the device status words (one per
+ * library source file whose kernels record errors), and return the first
+ * error found (FVATTN_OK, FVATTN_ERR_TIMEOUT or FVATTN_ERR_BOUNDS), or
  * FVATTN_ERR_CUDA if the synchronisation itself failed. */
 int fvattn_get_status(fvattn_stream_t stream);
+
+/* Fault injection for tests of the failure path (the pages have no
+ * counterpart; it exists so that a test can make a device wait run out
+ * without faulting, trapping or hanging the GPU).  Process-wide settings read
+ * by every later fvattn_sparse_attn launch (and its raster and no-alloc
+ * forms):
+ *   wait_limit_ns  bound of every wait inside the attention kernel, in
+ *                  nanoseconds; 0 restores the default (4 s)
+ *   flags          0, or FVATTN_HOOK_SKIP_V_LOADS: the kernel's V-loading
+ *                  warp leaves at once without loading or signalling
+ *                  anything, so the wait of the PV issuer for V runs out.
+ * A wait that runs out records FVATTN_ERR_TIMEOUT; every role of the CTA
+ * then leaves its loop, waits for its own copies and MMAs in flight and
+ * releases its tensor memory, and the kernel returns (its output is
+ * unspecified).  Call fvattn_test_hook(0, 0) to return to normal operation.
+ * Returns FVATTN_ERR_INVALID for unknown flags. */
+#define FVATTN_HOOK_SKIP_V_LOADS 1
+int fvattn_test_hook(unsigned long long wait_limit_ns, int flags);
 
 /* Static string naming a status code. */
 const char *fvattn_status_string(int code);

@@ -27,7 +27,7 @@ def _declared():
 def test_exports_every_declared_symbol(fv):
     lib = fv.load()
     names = _declared()
-    assert len(names) == 17
+    assert len(names) == 18
     assert sorted(fv.EXPORTED) == names
     for n in names:
         assert hasattr(lib, n), n
@@ -157,3 +157,13 @@ def test_route_kernel_launches(fv):
     assert lib.fvattn_route_kernel_launches(None) == 0
     for B, H in ((1, 40), (2, 40), (1, 1)):
         assert fv.route_kernel_launches(fv.geom(B, H, 128, 21, 45, 80, 2, 8, 8)) == 3
+
+
+def test_test_hook_rejects_unknown_flags(fv):
+    """fvattn_test_hook (fault injection for failure-path tests) accepts only
+    the documented flag and is reset by (0, 0); no GPU needed."""
+    lib = fv.load()
+    assert lib.fvattn_test_hook(0, 2) == fv.ERR_INVALID
+    assert lib.fvattn_test_hook(0, -1) == fv.ERR_INVALID
+    assert lib.fvattn_test_hook(1000, fv.HOOK_SKIP_V_LOADS) == fv.OK
+    assert lib.fvattn_test_hook(0, 0) == fv.OK
