@@ -66,14 +66,19 @@ constexpr uint32_t O_COL = 256;          // S_w at columns 128*w, O_w at 256 + 1
 constexpr float RESCALE_SUM_LIMIT = 1073741824.0f;   // 2^30
 constexpr int MAX_GROUP = 8;             // query blocks per tile at bs = 16
 // Register split: the launch gives every thread LAUNCH_REGS; the producer and
-// issuer warpgroup drops to REGS_LOW and the two softmax warpgroups (which
-// hold a whole 128-column S row) rise to REGS_HIGH.  One warpgroup at
-// REGS_LOW plus two at REGS_HIGH must fit in what the CTA was launched with;
-// the host checks the compiled register count before every launch.
+// issuer warpgroup drops to RegSplit::LOW and the two softmax warpgroups
+// (which hold a whole 128-column S row) rise to RegSplit::HIGH.  One
+// warpgroup at LOW plus two at HIGH must fit in what the CTA was launched
+// with; the host checks the compiled register count before every launch.
+// The bs = 128 kernel computes half of a chunk's exponentials before it needs
+// P_w (more live registers in the softmax); the query-group kernel keeps more
+// for its producer, which walks the union of the group's lists.
 constexpr int LAUNCH_REGS = 168;          // 65536 / 384 rounded down to a multiple of 8
-constexpr int REGS_LOW = 88;
-constexpr int REGS_HIGH = 208;
-static_assert(128 * REGS_LOW + 256 * REGS_HIGH <= ATT_THREADS * LAUNCH_REGS, "register split");
+template <bool GRP> struct RegSplit {
+    static constexpr int LOW = GRP ? 88 : 72;
+    static constexpr int HIGH = GRP ? 208 : 216;
+    static_assert(128 * LOW + 256 * HIGH <= ATT_THREADS * LAUNCH_REGS, "register split");
+};
 
 struct AttnArgs {
     Geo g;
@@ -305,7 +310,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     const uint32_t tmem = ctl.tmem_base;
 
     if (warp >= FIRST_SOFTMAX_WARP) {
-        regs_inc<REGS_HIGH>();
+        regs_inc<RegSplit<GRP>::HIGH>();
         // =========================== softmax groups (warps 4..7: w = 0, 8..11: w = 1)
         // Group w takes the chunks c with c & 1 == w: its own S_w, P_w and
         // O_w, running maximum m and sum l.  At the end of an item the two
@@ -368,50 +373,82 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                 // into P_w (128-byte swizzle, K-major operand).  Words whose 32 keys are all visible skip
                 // the mask tests; words with none skip the exponentials.
                 unsigned long long sm2[4];   // four chains of (even, odd) column sums
-                auto exp_pass = [&](float negv) {
+                // bs = 128: the first two quarters of the row (keys 0..63) are computed before P_w is
+                // needed, so the wait for the group's previous PV to release P_w overlaps them.  Query
+                // groups wait first and store each quarter as it is computed.
+                bool pw_free = false;
+                auto exp_quarter = [&](int q, const unsigned long long sl2x2, const unsigned long long negx2,
+                                       uint32_t (&wv)[16]) {
+                    const uint32_t mword = mw[q];
+                    if (mword == 0xFFFFFFFFu) {
+#pragma unroll
+                        for (int i = 0; i < 32; i += 2) {
+                            float x0, x1;
+                            f2_unpack(f2_fma(f2_pack(__uint_as_float(sv[q][i]), __uint_as_float(sv[q][i + 1])),
+                                             sl2x2, negx2), x0, x1);
+                            const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+                            sm2[(i >> 1) & 3] = f2_add(sm2[(i >> 1) & 3], f2_pack(p0, p1));
+                            wv[i >> 1] = pack_bf16x2(p0, p1);
+                        }
+                    } else if (mword == 0u) {
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) wv[i] = 0u;
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 32; i += 2) {
+                            float x0, x1;
+                            f2_unpack(f2_fma(f2_pack(__uint_as_float(sv[q][i]), __uint_as_float(sv[q][i + 1])),
+                                             sl2x2, negx2), x0, x1);
+                            const bool k0 = (mword >> i) & 1u, k1 = (mword >> (i + 1)) & 1u;
+                            const float p0 = k0 ? ex2_approx(x0) : 0.f;
+                            const float p1 = k1 ? ex2_approx(x1) : 0.f;
+                            sm2[(i >> 1) & 3] = f2_add(sm2[(i >> 1) & 3], f2_pack(p0, p1));
+                            wv[i >> 1] = pack_bf16x2(p0, p1);
+                        }
+                    }
+                };
+                auto store_quarter = [&](int q, const uint32_t (&wv)[16]) {
+                    const int half = q >> 1;
+#pragma unroll
+                    for (int k4 = 0; k4 < 4; ++k4) {
+                        const int chunk = (((q & 1) << 2) | k4) ^ (row & 7);
+                        const uint32_t addr = pbase + half * 16384u + chunk * 16u;
+                        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(wv[4 * k4]),
+                                     "r"(wv[4 * k4 + 1]), "r"(wv[4 * k4 + 2]), "r"(wv[4 * k4 + 3])
+                                     : "memory");
+                    }
+                };
+                // false: the CTA aborted while waiting for P_w
+                auto exp_pass = [&](float negv) -> bool {
 #pragma unroll
                     for (int i = 0; i < 4; ++i) sm2[i] = 0ull;
                     const unsigned long long sl2x2 = f2_pack(sl2, sl2), negx2 = f2_pack(negv, negv);
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const uint32_t mword = mw[q];
-                        uint32_t wv[16];
-                        if (mword == 0xFFFFFFFFu) {
-#pragma unroll
-                            for (int i = 0; i < 32; i += 2) {
-                                float x0, x1;
-                                f2_unpack(f2_fma(f2_pack(__uint_as_float(sv[q][i]), __uint_as_float(sv[q][i + 1])),
-                                                 sl2x2, negx2), x0, x1);
-                                const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
-                                sm2[(i >> 1) & 3] = f2_add(sm2[(i >> 1) & 3], f2_pack(p0, p1));
-                                wv[i >> 1] = pack_bf16x2(p0, p1);
-                            }
-                        } else if (mword == 0u) {
-#pragma unroll
-                            for (int i = 0; i < 16; ++i) wv[i] = 0u;
-                        } else {
-#pragma unroll
-                            for (int i = 0; i < 32; i += 2) {
-                                float x0, x1;
-                                f2_unpack(f2_fma(f2_pack(__uint_as_float(sv[q][i]), __uint_as_float(sv[q][i + 1])),
-                                                 sl2x2, negx2), x0, x1);
-                                const bool k0 = (mword >> i) & 1u, k1 = (mword >> (i + 1)) & 1u;
-                                const float p0 = k0 ? ex2_approx(x0) : 0.f;
-                                const float p1 = k1 ? ex2_approx(x1) : 0.f;
-                                sm2[(i >> 1) & 3] = f2_add(sm2[(i >> 1) & 3], f2_pack(p0, p1));
-                                wv[i >> 1] = pack_bf16x2(p0, p1);
-                            }
+                    uint32_t w0[16], w1[16];
+                    if (GRP) {
+                        if (!pw_free) {
+                            if (!wait_warp(smem_u32(&ctl.p_free[w]), (n & 1) ^ 1, abort_flag, wlim)) return false;
+                            pw_free = true;
                         }
-                        const int half = q >> 1;
 #pragma unroll
-                        for (int k4 = 0; k4 < 4; ++k4) {
-                            const int chunk = (((q & 1) << 2) | k4) ^ (row & 7);
-                            const uint32_t addr = pbase + half * 16384u + chunk * 16u;
-                            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(wv[4 * k4]),
-                                         "r"(wv[4 * k4 + 1]), "r"(wv[4 * k4 + 2]), "r"(wv[4 * k4 + 3])
-                                         : "memory");
+                        for (int q = 0; q < 4; ++q) {
+                            exp_quarter(q, sl2x2, negx2, w0);
+                            store_quarter(q, w0);
                         }
+                        return true;
                     }
+                    exp_quarter(0, sl2x2, negx2, w0);
+                    exp_quarter(1, sl2x2, negx2, w1);
+                    if (!pw_free) {
+                        if (!wait_warp(smem_u32(&ctl.p_free[w]), (n & 1) ^ 1, abort_flag, wlim)) return false;
+                        pw_free = true;
+                    }
+                    store_quarter(0, w0);
+                    store_quarter(1, w1);
+                    exp_quarter(2, sl2x2, negx2, w0);
+                    store_quarter(2, w0);
+                    exp_quarter(3, sl2x2, negx2, w1);
+                    store_quarter(3, w1);
+                    return true;
                 };
                 auto rescale_o = [&](float alpha) {
                     tc_fence_after();
@@ -451,11 +488,6 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                     for (int i = 0; i < 4; ++i) f2_unpack(sm2[i], sm[2 * i], sm[2 * i + 1]);
                     return ((sm[0] + sm[1]) + (sm[2] + sm[3])) + ((sm[4] + sm[5]) + (sm[6] + sm[7]));
                 };
-                // P_w and O_w were last used by this group's previous PV
-                if (!wait_warp(smem_u32(&ctl.p_free[w]), (n & 1) ^ 1, abort_flag, wlim)) {
-                    ok = false;
-                    break;
-                }
                 // The group's first chunk of an item takes the row maximum first and computes P against
                 // it (a row may see no key of its block in a chunk: it keeps max -inf, P 0).  Later chunks
                 // make one pass against the running reference maximum; while a row's sum stays at or
@@ -476,16 +508,20 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                             const float m_new = grow ? mxs : m_ref;
                             alpha = grow ? ex2_approx(m_ref - m_new) : 1.0f;
                             m_ref = m_new;
-                            rescale_o(alpha);
+                            rescale_o(alpha);   // O_w is quiet: the first exp pass waited for the previous PV
                         }
                     }
-                    exp_pass(-m_ref);
+                    if (!exp_pass(-m_ref)) {
+                        ok = false;
+                        break;
+                    }
                     sum = chunk_sum();
                     if (exact) break;
                     big = !(sum <= RESCALE_SUM_LIMIT);
                     if (!__any_sync(0xffffffffu, big)) break;
                     exact = true;
                 }
+                if (!ok) break;
                 l = l * alpha + sum;
                 fence_proxy_async_smem();
                 tc_fence_before();
@@ -579,7 +615,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
             ++item_seq;
         }
     } else {
-        regs_dec<REGS_LOW>();
+        regs_dec<RegSplit<GRP>::LOW>();
         if (warp == 0) {
             // =========================== K producer: items, Q tile, K blocks, masks
             // Column col = q*32 + lane of a chunk is token `off` of slot `slot`;
@@ -1079,7 +1115,7 @@ static int launch_attn(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
     // launched with, or the raising warpgroups would wait for ever.
     cudaFuncAttributes fa;
     if (cudaFuncGetAttributes(&fa, sparse_attn_kernel<D, GRP>) != cudaSuccess) return FVATTN_ERR_CUDA;
-    if (static_cast<long long>(fa.numRegs) * ATT_THREADS < 128ll * REGS_LOW + 256ll * REGS_HIGH)
+    if (static_cast<long long>(fa.numRegs) * ATT_THREADS < 128ll * RegSplit<GRP>::LOW + 256ll * RegSplit<GRP>::HIGH)
         return FVATTN_ERR_UNSUPPORTED;
     sparse_attn_kernel<D, GRP><<<grid, ATT_THREADS, L::ALLOC, s>>>(tq, tk, tv, args);
     FV_CHECK_LAUNCH();
