@@ -24,11 +24,14 @@
 //   warps 4..11 softmax, two groups of four warps: chunk c goes to group
 //               c & 1, which owns S_(c&1) and O_(c&1) in TMEM and a P tile in
 //               shared memory.  One query row per thread (its TMEM lane);
-//               online softmax in fp32 (exp2 on the MUFU, eight independent
-//               max and sum chains); P rounded to bf16 in the 128-byte-swizzled
-//               K-major layout; O rescaled only when the row maximum grows by
-//               more than 2^8.  At the end of an item the groups swap (m, l)
-//               per row and each writes half of the output columns.
+//               online softmax in fp32 from registers (the whole S row is
+//               loaded and S_w released at once; exp2 on the MUFU; eight
+//               independent max and sum chains); P rounded to bf16 in the
+//               128-byte-swizzled K-major layout; a chunk is computed against
+//               the running reference maximum and redone, with O rescaled,
+//               only when a row sum passes RESCALE_SUM_LIMIT.  At the end of
+//               an item the groups swap (m, l) per row and each writes half
+//               of the output columns.
 // Query groups (bs < 128): one 128-row tile holds G = 128 / bs consecutive
 // query blocks (their rows are contiguous in the tiled layout), so the MMA
 // tile is never half empty.  The tile walks the union of the G kv lists in
