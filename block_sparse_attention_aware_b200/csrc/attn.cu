@@ -686,7 +686,8 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                 UnionWalk uw;
                 if (GRP) uw.init(a.gbits + (static_cast<long long>(bh) * a.ngroups + u) * G * a.nwords, G, a.nwords, lane);
                 const int nc = (cnt + bpc - 1) / bpc;
-                // chunk cl's blocks (lane s < nblk: slot s) and membership bits, one chunk ahead
+                // chunk cl's blocks (lane s < nblk: slot s), membership bits and real extents, one chunk
+                // ahead (the extent load is in flight while the current chunk is handled)
                 int j_next = 0, n_next = 0;
                 uint32_t m_next = 0u;
                 if (GRP) {
@@ -696,11 +697,13 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                     j_next = chunk_block(list, 0, bpc, n_next, lane, g.nb);
                     m_next = 1u;
                 }
+                int e_next = lane < n_next ? __ldg(a.ext + j_next) : 0;
                 for (int cl = 0; cl < nc; ++cl, ++c_seq) {
                     const int stage = c_seq % KS;
                     const int nblk = n_next;
                     const int j = j_next;
                     const uint32_t mem = m_next;
+                    const int ext = e_next;
                     if (cl + 1 < nc) {
                         if (GRP) {
                             n_next = union_chunk<true>(uw, bpc, lane, j_next, m_next);
@@ -708,8 +711,8 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                             n_next = min(bpc, cnt - (cl + 1) * bpc);
                             j_next = chunk_block(list, cl + 1, bpc, n_next, lane, g.nb);
                         }
+                        e_next = lane < n_next ? __ldg(a.ext + j_next) : 0;
                     }
-                    const int ext = lane < nblk ? __ldg(a.ext + j) : 0;
                     if (!wait_warp(smem_u32(&ctl.k_empty[stage]), ((c_seq / KS) & 1) ^ 1, abort_flag, wlim)) {
                         ok = false;
                         break;
