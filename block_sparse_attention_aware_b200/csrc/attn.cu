@@ -353,8 +353,8 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                 // chunk c = c_seq + cl has c & 1 == w
                 const uint32_t c = c_seq + cl;
                 const int kst = c % KS;
-                if (!wait_warp(smem_u32(&ctl.k_full[kst]), (c / KS) & 1, abort_flag, wlim) ||
-                    !wait_warp(smem_u32(&ctl.s_full[w]), n & 1, abort_flag, wlim)) {
+                if (!wait_warp2(smem_u32(&ctl.k_full[kst]), (c / KS) & 1, smem_u32(&ctl.s_full[w]), n & 1,
+                                abort_flag, wlim)) {
                     ok = false;
                     break;
                 }
@@ -880,8 +880,8 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                         const uint32_t n = w ? n1 : n0;
                         if (qk_role) {
                             const int stage = c % KS;
-                            if (!wait_bar(smem_u32(&ctl.k_full[stage]), (c / KS) & 1, abort_flag, wlim) ||
-                                !wait_bar(smem_u32(&ctl.s_free[w]), (n & 1) ^ 1, abort_flag, wlim)) {
+                            if (!wait_bar2(smem_u32(&ctl.k_full[stage]), (c / KS) & 1, smem_u32(&ctl.s_free[w]),
+                                           (n & 1) ^ 1, abort_flag, wlim)) {
                                 ok = false;
                                 break;
                             }
@@ -899,8 +899,8 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                             if (cl == nc - 1) mma_commit(smem_u32(&ctl.q_empty));
                         } else {
                             const int stage = c % V_STAGES;
-                            if (!wait_bar(smem_u32(&ctl.p_full[w]), n & 1, abort_flag, wlim) ||
-                                !wait_bar(smem_u32(&ctl.v_full[stage]), (c / V_STAGES) & 1, abort_flag, wlim)) {
+                            if (!wait_bar2(smem_u32(&ctl.p_full[w]), n & 1, smem_u32(&ctl.v_full[stage]),
+                                           (c / V_STAGES) & 1, abort_flag, wlim)) {
                                 ok = false;
                                 break;
                             }

@@ -50,6 +50,23 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
+// Two mbarrier phases tried in one go (both tries are issued before either
+// result is used, so their latencies overlap); bit 0: first phase complete,
+// bit 1: second.
+__device__ __forceinline__ uint32_t mbar_try_wait2(uint32_t bar1, uint32_t parity1, uint32_t bar2,
+                                                   uint32_t parity2) {
+    uint32_t a, b;
+    asm volatile("{\n\t.reg .pred p, q;\n\t"
+                 "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%2], %3;\n\t"
+                 "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 q, [%4], %5;\n\t"
+                 "selp.u32 %0, 1, 0, p;\n\t"
+                 "selp.u32 %1, 2, 0, q;\n\t}"
+                 : "=r"(a), "=r"(b)
+                 : "r"(bar1), "r"(parity1), "r"(bar2), "r"(parity2)
+                 : "memory");
+    return a | b;
+}
+
 // Non-blocking test of an mbarrier phase.
 __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
     uint32_t ok;

@@ -41,6 +41,44 @@ __device__ __forceinline__ bool wait_warp(uint32_t bar, uint32_t parity, volatil
     return __all_sync(0xffffffffu, ok);
 }
 
+// Waits for two phases, trying both together until both have completed.
+__device__ __forceinline__ bool wait_bar2(uint32_t bar1, uint32_t parity1, uint32_t bar2, uint32_t parity2,
+                                          volatile int* abort_flag, unsigned long long limit_ns = WAIT_LIMIT_NS) {
+    uint32_t done = mbar_try_wait2(bar1, parity1, bar2, parity2);
+    if (done == 3u) return true;
+    unsigned long long t0 = 0;
+    for (uint32_t it = 1;; ++it) {
+        if (done & 1u) {
+            if (mbar_try_wait(bar2, parity2)) return true;
+        } else if (done & 2u) {
+            if (mbar_try_wait(bar1, parity1)) {
+                done |= 1u;
+                if (done == 3u) return true;
+            }
+        } else {
+            done = mbar_try_wait2(bar1, parity1, bar2, parity2);
+            if (done == 3u) return true;
+        }
+        if ((it & 255u) == 0u) {
+            if (*abort_flag) return false;
+            unsigned long long now = global_timer_ns();
+            if (t0 == 0) {
+                t0 = now;
+            } else if (now - t0 > limit_ns) {
+                record_status(FVATTN_ERR_TIMEOUT);
+                *abort_flag = 1;
+                return false;
+            }
+        }
+    }
+}
+
+__device__ __forceinline__ bool wait_warp2(uint32_t bar1, uint32_t parity1, uint32_t bar2, uint32_t parity2,
+                                           volatile int* abort_flag, unsigned long long limit_ns = WAIT_LIMIT_NS) {
+    const bool ok = wait_bar2(bar1, parity1, bar2, parity2, abort_flag, limit_ns);
+    return __all_sync(0xffffffffu, ok);
+}
+
 // Drain wait used on the way out (ignores the abort flag): for copies or
 // MMAs already issued, which complete on their own.
 __device__ __forceinline__ bool wait_bar_drain(uint32_t bar, uint32_t parity,
