@@ -359,19 +359,21 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                     break;
                 }
                 tc_fence_after();
+                // the mask words are read while the S row comes out of tensor memory
+                const uint32_t* mrow = ctl.mask[kst][tgrp];
+                uint32_t mw[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) mw[q] = mrow[q];
                 uint32_t sv[4][32];   // this row's 128 raw scores of the chunk
 #pragma unroll
                 for (int q = 0; q < 4; ++q) tmem_ld32(sb + q * 32u, sv[q]);
                 tmem_wait_ld();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(smem_u32(&ctl.s_free[w]));   // S_w read: the next QK may overwrite it
-                const uint32_t* mrow = ctl.mask[kst][tgrp];
-                uint32_t mw[4];
-#pragma unroll
-                for (int q = 0; q < 4; ++q) mw[q] = mrow[q];
-                __syncwarp();
-                if (lane == 0) mbar_arrive(smem_u32(&ctl.k_empty[kst]));   // mask in registers: stage free
+                if (lane == 0) {
+                    mbar_arrive(smem_u32(&ctl.s_free[w]));    // S_w read: the next QK may overwrite it
+                    mbar_arrive(smem_u32(&ctl.k_empty[kst]));   // mask in registers: stage free
+                }
                 // Exp pass: P = 2^(s*scale*log2e + negv) on fp32 pairs, row sum on fp32 pairs, bf16 P row
                 // into P_w (128-byte swizzle, K-major operand).  Words whose 32 keys are all visible skip
                 // the mask tests; words with none skip the exponentials.
