@@ -35,9 +35,11 @@
 // Query groups (bs < 128): one 128-row tile holds G = 128 / bs consecutive
 // query blocks (their rows are contiguous in the tiled layout), so the MMA
 // tile is never half empty.  The tile walks the union of the G kv lists in
-// ascending block order, from per-block membership bitmaps built by
-// group_bits_kernel; each chunk carries one key mask per query block of the
-// tile, so a row only sees the keys of its own block's list.
+// ascending block order, read from a union list (block ids with their
+// membership bits) that group_union_kernel writes once per launch, so the
+// loading warps do no set arithmetic per chunk; each chunk carries one key
+// mask per query block of the tile, so a row only sees the keys of its own
+// block's list.
 // Every wait is bounded; a wait that runs out records FVATTN_ERR_TIMEOUT,
 // raises a CTA-wide abort flag and all roles leave their loops, so the CTA
 // always reaches the TMEM release.
@@ -89,11 +91,10 @@ struct AttnArgs {
     const int32_t* kv_cnt;
     // Query groups: G = 128 / bs consecutive query blocks share one 128-row
     // tile.  For G > 1 an item is (b*h, group) and walks the union of the
-    // group's kv lists, given as per-block membership bitmaps.
+    // group's kv lists in ascending block order.
     int G;                       // query blocks per tile (1 when bs = 128)
     int ngroups;                 // ceil(nb / G)
-    int nwords;                  // 32-bit words per bitmap, ceil(nb / 32)
-    const uint32_t* gbits;       // [B*H][ngroups][G][nwords] (G > 1)
+    const uint32_t* ulist;       // [B*H][ngroups][nb] union lists (G > 1): block | membership bits << 24
     const int32_t* gcnt;         // [B*H][ngroups] union sizes (G > 1)
     const int32_t* ext;          // [nb] real extent of each block, packed as block_extent
     const int32_t* head_order;   // [B*H] heads, heaviest first
@@ -177,60 +178,21 @@ __device__ __forceinline__ int chunk_block(const int32_t* list, int cl, int bpc,
     return j;
 }
 
-// Walk of the union of a query group's kv lists in ascending block order.
-// Lane t < G holds the current word of block t's membership bitmap; the
-// walk position (word index, bits left of the union word) is warp-uniform.
-struct UnionWalk {
-    const uint32_t* maps;   // [G][nwords]
-    int G, nwords, wi;
-    uint32_t word, rem, ahead;   // ahead: lane t's word wi + 1, loaded one word early
-
-    __device__ __forceinline__ void init(const uint32_t* m, int groups, int nw, int lane) {
-        maps = m;
-        G = groups;
-        nwords = nw;
-        wi = -1;
-        word = 0u;
-        rem = 0u;
-        ahead = lane < G ? __ldg(maps + lane * nwords) : 0u;
+// Slots of chunk cl of a query group's union list (lane s < nn: slot s):
+// block id and membership bits (bit t: in the list of the tile's query
+// block t), range-checked.
+__device__ __forceinline__ int union_slot(const uint32_t* ul, int cl, int bpc, int nn, int lane, int nb,
+                                          uint32_t& mem) {
+    uint32_t e = 0u;
+    if (lane < nn) e = __ldg(ul + cl * bpc + lane);
+    int j = static_cast<int>(e & 0xFFFFFFu);
+    mem = e >> 24;
+    if (lane < nn && j >= nb) {
+        record_status(FVATTN_ERR_BOUNDS);
+        j = 0;
+        mem = 0u;
     }
-    // Next union block j and (when WANT_MEM) its membership bits (bit t: in
-    // block t's list); false once the union is exhausted.  Warp-uniform.
-    template <bool WANT_MEM>
-    __device__ __forceinline__ bool next(int lane, int& j, uint32_t& mem) {
-        while (rem == 0u) {
-            if (++wi >= nwords) return false;
-            word = ahead;
-            ahead = (lane < G && wi + 1 < nwords) ? __ldg(maps + lane * nwords + wi + 1) : 0u;
-            rem = __reduce_or_sync(0xffffffffu, word);
-        }
-        const int bit = __ffs(static_cast<int>(rem)) - 1;
-        rem &= rem - 1u;
-        j = wi * 32 + bit;
-        if (WANT_MEM) mem = __ballot_sync(0xffffffffu, (word >> bit) & 1u);
-        return true;
-    }
-};
-
-// Slots of the next chunk of a group walk: lane s < (returned count) gets
-// slot s's block and (when WANT_MEM) membership bits.
-template <bool WANT_MEM>
-__device__ __forceinline__ int union_chunk(UnionWalk& u, int bpc, int lane, int& j, uint32_t& mem) {
-    int n = 0;
-    j = 0;
-    mem = 0u;
-    for (int s2 = 0; s2 < bpc; ++s2) {
-        int jj;
-        uint32_t mm;
-        mm = 0u;
-        if (!u.template next<WANT_MEM>(lane, jj, mm)) break;
-        if (lane == s2) {
-            j = jj;
-            mem = mm;
-        }
-        ++n;
-    }
-    return n;
+    return j;
 }
 
 // GRP: 128-row tiles of G = 128 / bs > 1 query blocks walking the union of
@@ -685,19 +647,17 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                                         row_base + (qb + tq) * bs, smem_u32(&ctl.q_full));
                 }
                 const int32_t* list = a.kv_idx + (static_cast<long long>(bh) * g.nb + qb) * g.nb;
-                UnionWalk uw;
-                if (GRP) uw.init(a.gbits + (static_cast<long long>(bh) * a.ngroups + u) * G * a.nwords, G, a.nwords, lane);
+                const uint32_t* ul = GRP ? a.ulist + (static_cast<long long>(bh) * a.ngroups + u) * g.nb : nullptr;
                 const int nc = (cnt + bpc - 1) / bpc;
                 // chunk cl's blocks (lane s < nblk: slot s), membership bits and real extents, one chunk
                 // ahead (the extent load is in flight while the current chunk is handled)
-                int j_next = 0, n_next = 0;
-                uint32_t m_next = 0u;
+                int j_next = 0;
+                uint32_t m_next = 1u;
+                int n_next = min(bpc, cnt);
                 if (GRP) {
-                    n_next = union_chunk<true>(uw, bpc, lane, j_next, m_next);
+                    j_next = union_slot(ul, 0, bpc, n_next, lane, g.nb, m_next);
                 } else {
-                    n_next = min(bpc, cnt);
                     j_next = chunk_block(list, 0, bpc, n_next, lane, g.nb);
-                    m_next = 1u;
                 }
                 int e_next = lane < n_next ? __ldg(a.ext + j_next) : 0;
                 for (int cl = 0; cl < nc; ++cl, ++c_seq) {
@@ -707,10 +667,10 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                     const uint32_t mem = m_next;
                     const int ext = e_next;
                     if (cl + 1 < nc) {
+                        n_next = min(bpc, cnt - (cl + 1) * bpc);
                         if (GRP) {
-                            n_next = union_chunk<true>(uw, bpc, lane, j_next, m_next);
+                            j_next = union_slot(ul, cl + 1, bpc, n_next, lane, g.nb, m_next);
                         } else {
-                            n_next = min(bpc, cnt - (cl + 1) * bpc);
                             j_next = chunk_block(list, cl + 1, bpc, n_next, lane, g.nb);
                         }
                         e_next = lane < n_next ? __ldg(a.ext + j_next) : 0;
@@ -797,29 +757,20 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                 const int row_base = bh * static_cast<int>(g.Npad);
                 const int G = GRP ? a.G : 1;
                 const int32_t* list = a.kv_idx + (static_cast<long long>(bh) * g.nb + qb) * g.nb;
-                UnionWalk uw;
-                if (GRP) uw.init(a.gbits + (static_cast<long long>(bh) * a.ngroups + qb / G) * G * a.nwords, G, a.nwords,
-                                 lane);
+                const uint32_t* ul = GRP ? a.ulist + (static_cast<long long>(bh) * a.ngroups + qb / G) * g.nb : nullptr;
                 const int nc = (cnt + bpc - 1) / bpc;
-                int j_next = 0, n_next = 0;
                 uint32_t m_unused = 0u;
-                if (GRP) {
-                    n_next = union_chunk<false>(uw, bpc, lane, j_next, m_unused);
-                } else {
-                    n_next = min(bpc, cnt);
-                    j_next = chunk_block(list, 0, bpc, n_next, lane, g.nb);
-                }
+                int n_next = min(bpc, cnt);
+                int j_next = GRP ? union_slot(ul, 0, bpc, n_next, lane, g.nb, m_unused)
+                                 : chunk_block(list, 0, bpc, n_next, lane, g.nb);
                 for (int cl = 0; cl < nc; ++cl, ++c_seq) {
                     const int stage = c_seq % V_STAGES;
                     const int nblk = n_next;
                     const int j = j_next;
                     if (cl + 1 < nc) {
-                        if (GRP) {
-                            n_next = union_chunk<false>(uw, bpc, lane, j_next, m_unused);
-                        } else {
-                            n_next = min(bpc, cnt - (cl + 1) * bpc);
-                            j_next = chunk_block(list, cl + 1, bpc, n_next, lane, g.nb);
-                        }
+                        n_next = min(bpc, cnt - (cl + 1) * bpc);
+                        j_next = GRP ? union_slot(ul, cl + 1, bpc, n_next, lane, g.nb, m_unused)
+                                     : chunk_block(list, cl + 1, bpc, n_next, lane, g.nb);
                     }
                     if (!wait_warp(smem_u32(&ctl.v_empty[stage]), ((c_seq / V_STAGES) & 1) ^ 1, abort_flag, wlim)) {
                         ok = false;
@@ -949,15 +900,16 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
 
 // ------------------------------------------------------------------ work list
 
-// One warp per (b*h, query group) when G = 128 / bs > 1: membership bitmaps
-// of the group's G kv lists (bit j of map t: block j is in query block t's
-// list; order and repeats in a list do not matter) and the size of their
-// union, which is the number of kv blocks the group's tile walks.
-__global__ void __launch_bounds__(256) group_bits_kernel(Geo g, int G, int ngroups, int nwords,
-                                                         const int32_t* __restrict__ kv_idx,
-                                                         const int32_t* __restrict__ kv_cnt, uint32_t* __restrict__ gbits,
-                                                         int32_t* __restrict__ gcnt) {
-    extern __shared__ uint32_t gb_smem[];   // [8 warps][G * nwords]
+// One warp per (b*h, query group) when G = 128 / bs > 1: the union of the
+// group's G kv lists in ascending block order, each entry the block id with
+// its membership bits (bit t: the block is in query block t's list) above
+// bit 24, and the union's size, which is the number of kv blocks the group's
+// tile walks.  Order and repeats inside a list do not matter.
+__global__ void __launch_bounds__(256) group_union_kernel(Geo g, int G, int ngroups, int nwords,
+                                                          const int32_t* __restrict__ kv_idx,
+                                                          const int32_t* __restrict__ kv_cnt,
+                                                          uint32_t* __restrict__ ulist, int32_t* __restrict__ gcnt) {
+    extern __shared__ uint32_t gb_smem[];   // [8 warps][G * nwords] membership bitmaps
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const long long unit = static_cast<long long>(blockIdx.x) * 8 + warp;
     if (unit >= static_cast<long long>(g.B) * g.H * ngroups) return;
@@ -986,16 +938,31 @@ __global__ void __launch_bounds__(256) group_bits_kernel(Geo g, int G, int ngrou
         }
     }
     __syncwarp();
-    int un = 0;
-    for (int wd = lane; wd < nwords; wd += 32) {
-        uint32_t o = 0u;
-        for (int t = 0; t < G; ++t) o |= bits[t * nwords + wd];
-        un += __popc(o);
+    // lane l takes word 32r + l of round r; an exclusive scan of the words' union counts places them
+    uint32_t* dst = ulist + unit * nb;
+    int base = 0;
+    for (int w0 = 0; w0 < nwords; w0 += 32) {
+        const int wd = w0 + lane;
+        uint32_t un = 0u;
+        if (wd < nwords)
+            for (int t = 0; t < G; ++t) un |= bits[t * nwords + wd];
+        const int c = __popc(un);
+        int incl = c;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        int k = base + incl - c;
+        for (uint32_t r = un; r != 0u; r &= r - 1u) {
+            const int b = __ffs(static_cast<int>(r)) - 1;
+            uint32_t mem = 0u;
+            for (int t = 0; t < G; ++t) mem |= ((bits[t * nwords + wd] >> b) & 1u) << t;
+            dst[k++] = static_cast<uint32_t>(wd * 32 + b) | (mem << 24);
+        }
+        base += __shfl_sync(0xffffffffu, incl, 31);
     }
-    un = static_cast<int>(__reduce_add_sync(0xffffffffu, static_cast<unsigned int>(un)));
-    uint32_t* dst = gbits + unit * G * nwords;
-    for (int i = lane; i < G * nwords; i += 32) dst[i] = bits[i];
-    if (lane == 0) gcnt[unit] = un;
+    if (lane == 0) gcnt[unit] = base;
 }
 
 // One CTA per (b, h): order the head's `units` work units (query blocks, or
@@ -1069,10 +1036,10 @@ static bool make_tmap(CUtensorMap* m, const void* base, long long rows, int D, i
                         static_cast<unsigned long long>(D), 64u, static_cast<unsigned>(bs));
 }
 
-// Workspace: work list (item order, head cost and order, counter) and, when
-// G = 128 / bs > 1, the query groups' membership bitmaps and union sizes.
+// Workspace: work list (item order, head cost and order, counter), block
+// extents and, when G = 128 / bs > 1, the query groups' union lists and sizes.
 struct WsLayout {
-    size_t item_order, head_cost, head_order, counter, ext, gbits, gcnt, total;
+    size_t item_order, head_cost, head_order, counter, ext, ulist, gcnt, total;
     int G, ngroups, nwords;
 };
 
@@ -1089,11 +1056,11 @@ static WsLayout ws_layout(const fvattn_geom& g) {
     w.head_order = w.head_cost + al256(sizeof(long long) * BH);
     w.counter = w.head_order + al256(sizeof(int32_t) * BH);
     w.ext = w.counter + 256;
-    w.gbits = w.ext + al256(sizeof(int32_t) * g.nb);
-    w.gcnt = w.gbits;
-    w.total = w.gbits;
+    w.ulist = w.ext + al256(sizeof(int32_t) * g.nb);
+    w.gcnt = w.ulist;
+    w.total = w.ulist;
     if (w.G > 1) {
-        w.gcnt = w.gbits + al256(sizeof(uint32_t) * BH * w.ngroups * w.G * w.nwords);
+        w.gcnt = w.ulist + al256(sizeof(uint32_t) * BH * w.ngroups * g.nb);
         w.total = w.gcnt + al256(sizeof(int32_t) * BH * w.ngroups);
     }
     return w;
@@ -1170,15 +1137,15 @@ static int attn_impl(const fvattn_geom* gp, const void* q_t, const void* k_t, co
     long long* head_cost = reinterpret_cast<long long*>(ws + wl.head_cost);
     int32_t* head_order = reinterpret_cast<int32_t*>(ws + wl.head_order);
     int* counter = reinterpret_cast<int*>(ws + wl.counter);
-    uint32_t* gbits = wl.G > 1 ? reinterpret_cast<uint32_t*>(ws + wl.gbits) : nullptr;
+    uint32_t* ulist = wl.G > 1 ? reinterpret_cast<uint32_t*>(ws + wl.ulist) : nullptr;
     int32_t* gcnt = wl.G > 1 ? reinterpret_cast<int32_t*>(ws + wl.gcnt) : nullptr;
     const int BH = g.B * g.H;
     const int units = wl.G > 1 ? wl.ngroups : g.nb;
 
     if (wl.G > 1) {
         const long long warps = static_cast<long long>(BH) * wl.ngroups;
-        group_bits_kernel<<<static_cast<unsigned>((warps + 7) / 8), 256, sizeof(uint32_t) * 8 * wl.G * wl.nwords, s>>>(
-            g, wl.G, wl.ngroups, wl.nwords, kv_idx, kv_cnt, gbits, gcnt);
+        group_union_kernel<<<static_cast<unsigned>((warps + 7) / 8), 256, sizeof(uint32_t) * 8 * wl.G * wl.nwords, s>>>(
+            g, wl.G, wl.ngroups, wl.nwords, kv_idx, kv_cnt, ulist, gcnt);
         FV_CHECK_LAUNCH();
     }
     worklist_head_kernel<<<BH, 256, sizeof(int) * (g.nb + 2), s>>>(g, units, wl.G > 1 ? gcnt : kv_cnt, item_order,
@@ -1205,8 +1172,7 @@ static int attn_impl(const fvattn_geom* gp, const void* q_t, const void* k_t, co
     args.scale_log2 = scale * 1.4426950408889634f;
     args.G = wl.G;
     args.ngroups = wl.ngroups;
-    args.nwords = wl.nwords;
-    args.gbits = gbits;
+    args.ulist = ulist;
     args.gcnt = gcnt;
     args.ext = ext;
     args.total_items = BH * units;

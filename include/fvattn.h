@@ -202,8 +202,9 @@ int fvattn_copy_heads(const fvattn_geom *g, int h0, int nh, const void *src, voi
 int fvattn_route_kernel_launches(const fvattn_geom *g);
 
 /* Bytes of device workspace fvattn_sparse_attn needs: the work list (item
- * order, head cost and order, counter) and, for bs < 128, the query groups'
- * kv-list membership bitmaps and union sizes. */
+ * order, head cost and order, counter), the blocks' real extents and, for
+ * bs < 128, the union of each query group's kv lists (nb entries of 4 bytes
+ * per group: 255 MB for the 40-head CFG layer at nb = 1260) and its size. */
 size_t fvattn_attn_workspace_size(const fvattn_geom *g);
 
 /* Number of CTAs (one per SM) the persistent attention kernel launches on
@@ -256,8 +257,9 @@ int fvattn_sparse_attn_raster(const fvattn_geom *g, const void *q_t, const void 
 /* Maximum scratch, in bytes, of fvattn_sparse_attn_noalloc (2 MiB): enough
  * for fvattn_attn_workspace_size(g) of up to about 500 000 work items
  * (B*H*nb) at bs = 128 (e.g. B*H <= 200 at nb = 2560).  For bs < 128 the
- * query groups' bitmaps (about B*H*nb*ceil(nb/32)*4 bytes) count too: a
- * 40-head layer at bs = 64 fits up to nb = 608. */
+ * query groups' union lists (B*H*ceil(nb*bs/128)*nb*4 bytes) count too: a
+ * 40-head layer fits up to nb = 160 at bs = 64, 224 at bs = 32 and 318 at
+ * bs = 16. */
 #define FVATTN_NOALLOC_SCRATCH_BYTES (2u * 1024u * 1024u)
 
 /* fvattn_sparse_attn without a workspace argument, for callers that cannot
