@@ -35,9 +35,9 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 WORKLOAD = "720p"
 
 # DRAM bytes (read + write) of one sparse_attn_kernel<128, 0> launch on the 720p layer: an ncu capture
-# of the same layer restricted to 4 heads read 376.0 MB and wrote 77.0 MB; K/V reuse stays inside a
+# of the same layer restricted to 4 heads read 383.7 MB and wrote 75.6 MB; K/V reuse stays inside a
 # head, so traffic scales with the head count (x10 for 40 heads).
-ATTN_TRAFFIC_720P = {"bytes": (376.000256e6 + 77.03936e6) * 10,
+ATTN_TRAFFIC_720P = {"bytes": (383.733504e6 + 75.581184e6) * 10,
                      "how": "ncu dram__bytes_read.sum + dram__bytes_write.sum of the 4-head 720p layer, x10 heads"}
 
 
