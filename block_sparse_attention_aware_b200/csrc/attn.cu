@@ -77,7 +77,7 @@ constexpr int MAX_GROUP = 8;             // query blocks per tile at bs = 16
 // with; the host checks the compiled register count before every launch.
 // The bs = 128 kernel computes half of a chunk's exponentials before it needs
 // P_w (more live registers in the softmax); the query-group kernel keeps more
-// for its producer, which walks the union of the group's lists.
+// for its producer, which builds one key mask per query block of the tile.
 constexpr int LAUNCH_REGS = 168;          // 65536 / 384 rounded down to a multiple of 8
 template <bool GRP> struct RegSplit {
     static constexpr int LOW = GRP ? 88 : 72;

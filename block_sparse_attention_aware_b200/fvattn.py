@@ -446,8 +446,8 @@ class Layer:
 
     def kernel_launches(self) -> int:
         """Kernels one __call__ (unfused inverse) launches: reorders, routing,
-        the work list (plus the query-group bitmaps for bs < 128), attention,
-        inverse reorder."""
+        the work list (plus the query groups' union lists for bs < 128),
+        attention, inverse reorder."""
         reorders = 1 if self.fused_route else 3
         worklist = 2 + (1 if self.g.bs < 128 else 0)
         return reorders + route_kernel_launches(self.g) + worklist + 1 + 1
