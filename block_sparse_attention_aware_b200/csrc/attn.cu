@@ -75,13 +75,12 @@ constexpr int MAX_GROUP = 8;             // query blocks per tile at bs = 16
 // (which hold a whole 128-column S row) rise to RegSplit::HIGH.  One
 // warpgroup at LOW plus two at HIGH must fit in what the CTA was launched
 // with; the host checks the compiled register count before every launch.
-// The bs = 128 kernel computes half of a chunk's exponentials before it needs
-// P_w (more live registers in the softmax); the query-group kernel keeps more
-// for its producer, which builds one key mask per query block of the tile.
+// The softmax computes half of a chunk's exponentials before it needs P_w,
+// which takes more live registers there.
 constexpr int LAUNCH_REGS = 168;          // 65536 / 384 rounded down to a multiple of 8
 template <bool GRP> struct RegSplit {
-    static constexpr int LOW = GRP ? 88 : 72;
-    static constexpr int HIGH = GRP ? 208 : 216;
+    static constexpr int LOW = 72;
+    static constexpr int HIGH = 216;
     static_assert(128 * LOW + 256 * HIGH <= ATT_THREADS * LAUNCH_REGS, "register split");
 };
 
@@ -340,9 +339,8 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                 // into P_w (128-byte swizzle, K-major operand).  Words whose 32 keys are all visible skip
                 // the mask tests; words with none skip the exponentials.
                 unsigned long long sm2[4];   // four chains of (even, odd) column sums
-                // bs = 128: the first two quarters of the row (keys 0..63) are computed before P_w is
-                // needed, so the wait for the group's previous PV to release P_w overlaps them.  Query
-                // groups wait first and store each quarter as it is computed.
+                // The first two quarters of the row (keys 0..63) are computed before P_w is needed, so
+                // the wait for the group's previous PV to release P_w overlaps them.
                 bool pw_free = false;
                 auto exp_quarter = [&](int q, const unsigned long long sl2x2, const unsigned long long negx2,
                                        uint32_t (&wv)[16]) {
@@ -391,18 +389,6 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                     for (int i = 0; i < 4; ++i) sm2[i] = 0ull;
                     const unsigned long long sl2x2 = f2_pack(sl2, sl2), negx2 = f2_pack(negv, negv);
                     uint32_t w0[16], w1[16];
-                    if (GRP) {
-                        if (!pw_free) {
-                            if (!wait_warp(smem_u32(&ctl.p_free[w]), (n & 1) ^ 1, abort_flag, wlim)) return false;
-                            pw_free = true;
-                        }
-#pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            exp_quarter(q, sl2x2, negx2, w0);
-                            store_quarter(q, w0);
-                        }
-                        return true;
-                    }
                     exp_quarter(0, sl2x2, negx2, w0);
                     exp_quarter(1, sl2x2, negx2, w1);
                     if (!pw_free) {
