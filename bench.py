@@ -581,7 +581,7 @@ def run_fvattn(args):
         kh = k.cpu().pin_memory()
         vh = v.cpu().pin_memory()
         oh = torch.empty_like(qh).pin_memory()
-        groups = args.e2e_groups or fvattn.default_head_groups(g.H)
+        groups = args.e2e_groups or fvattn.default_head_group_sizes(g.H)
         pipe = fvattn.HostPipeline(fvattn.geom_of(w), w.p, w.k, groups=groups, device=dev, order=args.order,
                                    fused_route=fused)
         pipe(qh, kh, vh, oh)
@@ -598,7 +598,7 @@ def run_fvattn(args):
         te /= args.e2e_steps
         line["e2e"] = {"value": flops_all / te / 1e12, "unit": "TFLOP/s", "ms_per_step": te * 1e3,
                        "h2d_bytes_per_step": 3 * raster_bytes, "d2h_bytes_per_step": raster_bytes,
-                       "steps": args.e2e_steps, "head_groups": groups,
+                       "steps": args.e2e_steps, "head_groups": pipe.sizes,
                        "how": "fvattn.HostPipeline: per head group, 2-D H2D copies of Q/K/V, the layer's calls "
                               "(Q/K reorder + routing in one pass, V reorder, attention, inverse reorder), "
                               "2-D D2H copy of O; groups overlap on two copy streams and the compute stream"}
@@ -632,8 +632,9 @@ def main():
     ap.add_argument("--stack", action="store_true",
                     help="also time every seeded layer of a multi-layer workload once (cfg720p: 40 layers)")
     ap.add_argument("--e2e-groups", type=int, default=0,
-                    help="head groups of the end-to-end pipeline (uploads, compute and downloads overlap); "
-                         "0: fvattn.default_head_groups (two heads a group: 20 for 40 heads)")
+                    help="equal head groups of the end-to-end pipeline (uploads, compute and downloads "
+                         "overlap); 0: fvattn.default_head_group_sizes (two heads a group, one in the first "
+                         "and the last: 21 groups for 40 heads)")
     ap.add_argument("--unfused-route", action="store_true",
                     help="time the step with separate reorders and routing instead of the fused call")
     ap.add_argument("--heads", type=int, default=0,

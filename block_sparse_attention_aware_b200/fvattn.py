@@ -11,7 +11,7 @@ import ctypes
 import math
 import os
 from dataclasses import dataclass
-from typing import Optional
+from typing import List, Optional
 
 import torch
 
@@ -475,42 +475,53 @@ class Layer:
         return self.restore(stream)
 
 
-def default_head_groups(H: int) -> int:
-    """Head groups for HostPipeline: two heads per group when H is even,
-    otherwise the most groups with at least two heads each (one group when
-    no divisor of H allows that).  Smaller groups leave less of the first
-    upload and the last download outside the overlap."""
-    best = 1
-    for groups in range(1, H + 1):
-        if H % groups == 0 and H // groups >= 2:
-            best = groups
-    return best
+def default_head_group_sizes(H: int) -> List[int]:
+    """Head-group sizes for HostPipeline: two heads a group, except the first
+    and the last group, which hold one head each.  Before the first group's
+    routing can start, its Q and K must be uploaded. After the last group's
+    compute, its output must be downloaded.  Neither overlaps any compute,
+    so both groups are kept small.  For 40 heads: 1, 2 x 19, 1 (21 groups)."""
+    if H < 1:
+        raise ValueError(f"{H} heads")
+    if H <= 2:
+        return [1] * H
+    m = (H - 2) // 2
+    return [1] + [2] * m + [1] * (H - 1 - 2 * m)
 
 
 class HostPipeline:
     """End to end from page-locked host buffers, pipelined by head groups.
 
-    Heads are independent through every step, so the layer is run as
-    `groups` head slices on two rotating sets of device buffers: the upload
-    of slice i+1 (one copy stream), the library calls on slice i (the
-    compute stream) and the download of slice i-1 (another copy stream)
-    overlap.  Within a slice, Q and K are uploaded first and routed while V
-    is still on its way.  The output equals one whole-layer call bit for
-    bit."""
+    Heads are independent through every step, so the layer is run as head
+    slices: the upload of slice i+1 (one copy stream), the library calls on
+    slice i (the compute stream) and the download of slice i-1 (another copy
+    stream) overlap.  Within a slice, Q and K are uploaded first and routed
+    while V is still on its way.  `groups` is None (default_head_group_sizes),
+    a number of equal groups, or a list of group sizes in heads.  Slices of
+    one size rotate over two sets of device buffers.  The output equals one
+    whole-layer call bit for bit."""
 
-    def __init__(self, g: Geom, p: float, k: int, groups: Optional[int] = None, device="cuda",
+    def __init__(self, g: Geom, p: float, k: int, groups=None, device="cuda",
                  order: str = "raster", fused_route: bool = True):
         if groups is None:
-            groups = default_head_groups(g.H)
-        if groups < 1 or g.H % groups:
-            raise ValueError(f"{g.H} heads do not split into {groups} equal groups")
-        self.g, self.groups, self.nh = g, groups, g.H // groups
-        gs = geom(g.B, self.nh, g.D, g.F, g.Hs, g.Ws, g.tf, g.th, g.tw)
-        self.layers = [Layer(gs, p, k, device=device, order=order, fused_route=fused_route)
-                       for _ in range(min(2, groups))]
-        shape = (g.B, g.N, self.nh, g.D)
-        self.inputs = [[torch.empty(shape, dtype=torch.bfloat16, device=device) for _ in range(3)]
-                       for _ in self.layers]
+            sizes = default_head_group_sizes(g.H)
+        elif isinstance(groups, int):
+            if groups < 1 or g.H % groups:
+                raise ValueError(f"{g.H} heads do not split into {groups} equal groups")
+            sizes = [g.H // groups] * groups
+        else:
+            sizes = [int(x) for x in groups]
+            if not sizes or min(sizes) < 1 or sum(sizes) != g.H:
+                raise ValueError(f"group sizes {sizes} do not partition {g.H} heads")
+        self.g, self.sizes, self.groups = g, sizes, len(sizes)
+        # per group size: one or two (Layer, device Q/K/V slices) buffer sets
+        self.sets = {}
+        for nh in sorted(set(sizes)):
+            gs = geom(g.B, nh, g.D, g.F, g.Hs, g.Ws, g.tf, g.th, g.tw)
+            shape = (g.B, g.N, nh, g.D)
+            self.sets[nh] = [(Layer(gs, p, k, device=device, order=order, fused_route=fused_route),
+                              [torch.empty(shape, dtype=torch.bfloat16, device=device) for _ in range(3)])
+                             for _ in range(min(2, sizes.count(nh)))]
         self.up = torch.cuda.Stream(device=device)
         self.down = torch.cuda.Stream(device=device)
 
@@ -522,17 +533,21 @@ class HostPipeline:
         start.record(s)
         self.up.wait_event(start)
         self.down.wait_event(start)
-        freed = [None] * len(self.layers)     # download of the slice that last used a buffer set
+        freed = {}        # buffer set -> download of the slice that last used it
+        seen = {}         # group size -> slices of that size so far
         done = None
-        for i in range(self.groups):
-            b = i % len(self.layers)
-            lay, (qd, kd, vd) = self.layers[b], self.inputs[b]
-            if freed[b] is not None:
+        h0 = 0
+        for nh in self.sizes:
+            sets = self.sets[nh]
+            b = (nh, seen.get(nh, 0) % len(sets))
+            seen[nh] = seen.get(nh, 0) + 1
+            lay, (qd, kd, vd) = sets[b[1]]
+            if b in freed:
                 self.up.wait_event(freed[b])
             uploaded = []
             for pair in (((q_host, qd), (k_host, kd)), ((v_host, vd),)):
                 for src, dst in pair:
-                    _check("fvattn_copy_heads", L.fvattn_copy_heads(ctypes.byref(g), i * self.nh, self.nh,
+                    _check("fvattn_copy_heads", L.fvattn_copy_heads(ctypes.byref(g), h0, nh,
                                                                     ctypes.c_void_p(src.data_ptr()), _ptr(dst), 1,
                                                                     _stream(self.up)))
                 uploaded.append(torch.cuda.Event())
@@ -546,12 +561,13 @@ class HostPipeline:
             computed = torch.cuda.Event()
             computed.record(s)
             self.down.wait_event(computed)
-            _check("fvattn_copy_heads", L.fvattn_copy_heads(ctypes.byref(g), i * self.nh, self.nh, _ptr(out),
+            _check("fvattn_copy_heads", L.fvattn_copy_heads(ctypes.byref(g), h0, nh, _ptr(out),
                                                             ctypes.c_void_p(o_host.data_ptr()), 0,
                                                             _stream(self.down)))
             done = torch.cuda.Event()
             done.record(self.down)
             freed[b] = done
+            h0 += nh
         s.wait_event(done)
         return o_host
 

@@ -4,12 +4,21 @@ import pytest
 from block_sparse_attention_aware_b200 import fvattn
 
 
-@pytest.mark.parametrize("H,want", [(40, 20), (4, 2), (2, 1), (1, 1), (3, 1), (6, 3), (9, 3), (7, 1), (12, 6)])
-def test_default_head_groups(H, want):
-    groups = fvattn.default_head_groups(H)
-    assert groups == want
-    assert H % groups == 0
-    assert groups == 1 or H // groups >= 2
+@pytest.mark.parametrize("H", [1, 2, 3, 4, 5, 6, 7, 9, 12, 40])
+def test_default_head_group_sizes(H):
+    sizes = fvattn.default_head_group_sizes(H)
+    assert sum(sizes) == H
+    assert sizes[0] == 1 and sizes[-1] == 1
+    assert all(s in (1, 2) for s in sizes)
+    # the middle groups hold two heads each (one leftover head joins the end)
+    assert all(s == 2 for s in sizes[1:-2])
+    if H == 40:
+        assert sizes == [1] + [2] * 19 + [1]
+
+
+def test_head_group_sizes_rejected():
+    with pytest.raises(ValueError):
+        fvattn.default_head_group_sizes(0)
 
 
 @pytest.fixture(scope="module")
