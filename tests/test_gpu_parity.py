@@ -359,10 +359,10 @@ def test_fused_inverse_reorder_matches_oracle_hilbert(fv, orc, name, w):
     _raster_vs_oracle(fv, orc, w)
 
 
-@pytest.mark.parametrize("groups", [2, 4])
+@pytest.mark.parametrize("groups", [2, 4, None, [1, 3], [2, 1, 1]], ids=["2", "4", "default", "1-3", "2-1-1"])
 def test_host_pipeline_matches_whole_layer(fv, groups):
     """The head-group pipeline from page-locked host buffers writes the same
-    bits as one whole-layer call."""
+    bits as one whole-layer call, for equal and for uneven group sizes."""
     w = synth.custom_workload(B=2, H=4, D=128, F=3, Hs=16, Ws=24, tf=2, th=8, tw=8, seed=51, p=0.8, k=2,
                               qscale="fixed", qscale_values=(0.5, 2.0, 6.0, 1.0))
     g = fv.geom_of(w)
