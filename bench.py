@@ -39,6 +39,11 @@ WORKLOAD = "720p"
 # head, so traffic scales with the head count (x10 for 40 heads).
 ATTN_TRAFFIC_720P = {"bytes": (383.733504e6 + 75.581184e6) * 10,
                      "how": "ncu dram__bytes_read.sum + dram__bytes_write.sum of the 4-head 720p layer, x10 heads"}
+# The CFG 720p layer (B=2, 64-token blocks) restricted to 4 heads: 627.3 MB read, 152.1 MB written.
+ATTN_TRAFFIC_CFG720P = {"bytes": (627.297792e6 + 152.127744e6) * 10,
+                        "how": "ncu dram__bytes_read.sum + dram__bytes_write.sum of the 4-head CFG 720p layer, "
+                               "x10 heads"}
+ATTN_TRAFFIC = {"720p": ATTN_TRAFFIC_720P, "cfg720p": ATTN_TRAFFIC_CFG720P}
 
 
 def load_peaks():
@@ -534,8 +539,8 @@ def run_fvattn(args):
         "stages_gbs": gbs,
         "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": sustained, "unit": "TFLOP/s",
                      "frac": attn_tflops / sustained,
-                     "traffic": ATTN_TRAFFIC_720P["bytes"] if (w.name == "720p" and not args.heads) else None,
-                     "traffic_how": ATTN_TRAFFIC_720P["how"] if (w.name == "720p" and not args.heads) else None,
+                     "traffic": ATTN_TRAFFIC[w.name]["bytes"] if (w.name in ATTN_TRAFFIC and not args.heads) else None,
+                     "traffic_how": ATTN_TRAFFIC[w.name]["how"] if (w.name in ATTN_TRAFFIC and not args.heads) else None,
                      "algorithmic_bytes_per_launch": 4 * tiled_bytes,
                      "kernel": f"sparse_attn_kernel<{g.D}, {int(g.bs < 128)}>",
                      "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside back-to-back steps)",
