@@ -21,6 +21,15 @@ def test_head_group_sizes_rejected():
         fvattn.default_head_group_sizes(0)
 
 
+@pytest.mark.parametrize("groups", [3, 0, [1, 2], [2, 2, 1], [0, 4], []])
+def test_host_pipeline_rejects_bad_groups(fv, groups):
+    """HostPipeline checks its head grouping before it allocates anything:
+    equal groups must divide H, and a list of sizes must partition it."""
+    g = fv.geom(1, 4, 64, 2, 8, 8, 2, 2, 4)
+    with pytest.raises(ValueError):
+        fv.HostPipeline(g, 0.9, 2, groups=groups, device="cpu")
+
+
 @pytest.fixture(scope="module")
 def fv():
     from block_sparse_attention_aware_b200 import build
